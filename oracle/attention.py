@@ -1,0 +1,213 @@
+"""Plain float64 attention: the definition written out, no tiling, no online softmax.
+
+TEST INFRASTRUCTURE ONLY (see the package docstring).  Nothing here is shared
+with the CUDA path: the two meet only on the seeded bf16 inputs.
+
+Sources (page title and section):
+  * "注意力优化：FlashAttention 与稀疏注意力", 核心公式 / 公式速览:
+      S = Q K^T / sqrt(d_k); A = row softmax of S (each row sums to 1);
+      output row i = sum_j A_ij V_j; a disallowed key j gets logit -inf
+      before the softmax, so its weight is 0.
+  * "高效注意力" §3 (MQA/GQA): several query heads share one K/V head.
+  * "高效注意力" §4 and "大模型高效注意力机制全解析" §3.2.1 (sliding_window):
+      each token attends to a window of nearby tokens.  Read here as the
+      causal band  i - w < j <= i  (w keys, the query itself included).
+  * "缩放定律与高效注意力" §3.3: the backward pass needs only O and the per-row
+      logsumexp; the gradient formulas themselves are the textbook softmax
+      gradient (the pages do not print them).
+
+Conventions (the readings the pages leave open):
+  * Layout [B, H, L, d]; query head h reads K/V head h // (Hq // Hkv).
+  * Causal alignment is top-left: key j visible to query i iff j <= i.
+  * `scale` multiplies Q K^T; LSE is the natural log of sum_j exp(scale*S_ij)
+    over visible j.
+  * A row with no visible key has O = 0, LSE = -inf, dQ = 0 (no NaN).
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+# Rows per block when a head is evaluated in row blocks (bounds memory only;
+# every row is still the plain definition over its visible columns).
+_ROW_BLOCK_ELEMS = 1 << 24
+
+
+def visible_mask(Lq: int, Lk: int, causal: bool, window: int) -> np.ndarray:
+    """Boolean [Lq, Lk]: True where key j is visible to query i."""
+    i = np.arange(Lq)[:, None]
+    j = np.arange(Lk)[None, :]
+    vis = np.ones((Lq, Lk), dtype=bool)
+    if causal:
+        vis &= j <= i
+    if window > 0:
+        vis &= j > i - window
+    return vis
+
+
+def visible_band(r0: int, r1: int, Lk: int, causal: bool, window: int) -> tuple[int, int]:
+    """Columns [lo, hi) that can be visible to any row in [r0, r1)."""
+    hi = min(Lk, r1) if causal else Lk
+    lo = max(0, r0 - window + 1) if window > 0 else 0
+    return lo, max(lo, hi)
+
+
+def _f64(x) -> np.ndarray:
+    if x.dtype == np.uint16:  # bf16 bits: widen exactly
+        x = (x.astype(np.uint32) << 16).view(np.float32)
+    return np.asarray(x, dtype=np.float64)
+
+
+def attention_weights(q, k, scale: float, vis: np.ndarray):
+    """Scores, weights and logsumexp for one head.
+
+    q [Lq, d], k [Lk, d] float64; vis [Lq, Lk] bool.
+    Returns (A, lse): A[i, j] = exp(S_ij) / sum_vis exp(S_ij) on visible
+    entries and exactly 0 elsewhere; lse[i] = log sum_vis exp(S_ij).
+    """
+    S = scale * (q @ k.T)
+    S = np.where(vis, S, -np.inf)
+    m = S.max(axis=1, keepdims=True)
+    m = np.where(np.isfinite(m), m, 0.0)          # fully masked row: any shift works
+    E = np.where(vis, np.exp(S - m), 0.0)
+    l = E.sum(axis=1, keepdims=True)
+    A = np.divide(E, l, out=np.zeros_like(E), where=l > 0)
+    with np.errstate(divide="ignore"):
+        lse = np.where(l[:, 0] > 0, m[:, 0] + np.log(l[:, 0]), -np.inf)
+    return A, lse
+
+
+def _head_fwd(qh, kh, vh, scale, causal, window, rows=None):
+    """O and LSE for the rows `rows` (default: all) of one head."""
+    Lq, Lk = qh.shape[0], kh.shape[0]
+    rows = np.arange(Lq) if rows is None else np.asarray(rows)
+    O = np.zeros((rows.size, vh.shape[1]))
+    lse = np.full(rows.size, -np.inf)
+    if rows.size == 0:
+        return O, lse
+    # Contiguous runs of rows are evaluated block by block over their band.
+    step = max(1, _ROW_BLOCK_ELEMS // max(1, Lk))
+    start = 0
+    while start < rows.size:
+        stop = min(rows.size, start + step)
+        blk = rows[start:stop]
+        r0, r1 = int(blk.min()), int(blk.max()) + 1
+        lo, hi = visible_band(r0, r1, Lk, causal, window)
+        vis = _band_mask(blk, lo, hi, causal, window)
+        A, l = attention_weights(qh[blk], kh[lo:hi], scale, vis)
+        O[start:stop] = A @ vh[lo:hi]
+        lse[start:stop] = l
+        start = stop
+    return O, lse
+
+
+def _band_mask(rows, lo, hi, causal, window):
+    i = np.asarray(rows)[:, None]
+    j = np.arange(lo, hi)[None, :]
+    vis = np.ones((i.shape[0], hi - lo), dtype=bool)
+    if causal:
+        vis &= j <= i
+    if window > 0:
+        vis &= j > i - window
+    return vis
+
+
+def _group(Hq: int, Hkv: int) -> int:
+    if Hkv <= 0 or Hq % Hkv:
+        raise ValueError("Hq must be a multiple of Hkv")
+    return Hq // Hkv
+
+
+def _kv_head(h: int, Hq: int, Hkv: int) -> int:
+    """K/V head read by query head h: contiguous groups of Hq/Hkv query heads."""
+    return h // _group(Hq, Hkv)
+
+
+def attn_fwd(q, k, v, scale: float, causal: bool = False, window: int = 0, heads=None):
+    """O [B,Hq,Lq,d] and LSE [B,Hq,Lq] in float64.
+
+    q: [B,Hq,Lq,d]; k, v: [B,Hkv,Lk,d] (float or bf16 bits as uint16).
+    heads: optional list of (b, h) to evaluate; other heads are left NaN.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Hq, Lq, d = q.shape
+    Hkv = k.shape[1]
+    O = np.full((B, Hq, Lq, v.shape[-1]), np.nan)
+    lse = np.full((B, Hq, Lq), np.nan)
+    todo = heads if heads is not None else [(b, h) for b in range(B) for h in range(Hq)]
+    for b, h in todo:
+        g = _kv_head(h, Hq, Hkv)
+        O[b, h], lse[b, h] = _head_fwd(q[b, h], k[b, g], v[b, g], scale, causal, window)
+    return O, lse
+
+
+def attn_fwd_rows(q, k, v, scale, causal, window, b, h, rows):
+    """O and LSE for selected rows of one head (sampled checks at full size).
+
+    Each row is evaluated from the definition over all of its visible keys.
+    """
+    Hq, Hkv = q.shape[1], k.shape[1]
+    g = _kv_head(h, Hq, Hkv)
+    rows = np.sort(np.asarray(rows))
+    qh = _f64(q[b, h])
+    kh = _f64(k[b, g])
+    vh = _f64(v[b, g])
+    Lk = kh.shape[0]
+    O = np.zeros((rows.size, qh.shape[1]))
+    lse = np.zeros(rows.size)
+    for n, i in enumerate(rows):
+        lo, hi = visible_band(int(i), int(i) + 1, Lk, causal, window)
+        vis = _band_mask([i], lo, hi, causal, window)
+        A, l = attention_weights(qh[i:i + 1], kh[lo:hi], scale, vis)
+        O[n] = (A @ vh[lo:hi])[0]
+        lse[n] = l[0]
+    return O, lse
+
+
+def _head_bwd(qh, kh, vh, doh, scale, causal, window):
+    """dQ, dK, dV for one (query head, kv head) pair; textbook softmax gradient."""
+    Lq, Lk = qh.shape[0], kh.shape[0]
+    dq = np.zeros_like(qh)
+    dk = np.zeros_like(kh)
+    dv = np.zeros_like(vh)
+    step = max(1, _ROW_BLOCK_ELEMS // max(1, Lk))
+    for r0 in range(0, Lq, step):
+        r1 = min(Lq, r0 + step)
+        lo, hi = visible_band(r0, r1, Lk, causal, window)
+        vis = _band_mask(np.arange(r0, r1), lo, hi, causal, window)
+        A, _ = attention_weights(qh[r0:r1], kh[lo:hi], scale, vis)
+        O = A @ vh[lo:hi]
+        dO = doh[r0:r1]
+        dv[lo:hi] += A.T @ dO                       # dV = A^T dO
+        dP = dO @ vh[lo:hi].T                        # dP = dO V^T
+        D = np.sum(dO * O, axis=1, keepdims=True)    # D_i = dO_i . O_i = sum_j A_ij dP_ij
+        dS = A * (dP - D)                            # softmax Jacobian applied row by row
+        dq[r0:r1] = scale * (dS @ kh[lo:hi])         # S = scale Q K^T
+        dk[lo:hi] += scale * (dS.T @ qh[r0:r1])
+    return dq, dk, dv
+
+
+def attn_bwd(q, k, v, do, scale: float, causal: bool = False, window: int = 0, heads=None):
+    """dQ [B,Hq,Lq,d], dK and dV [B,Hkv,Lk,d] in float64.
+
+    dK/dV of a K/V head are summed over the query heads that share it.
+    heads: optional list of (b, hkv): only those K/V heads (and all query
+    heads of their groups) are evaluated; the rest is left NaN.
+    """
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    B, Hq, Lq, d = q.shape
+    Hkv = k.shape[1]
+    _group(Hq, Hkv)
+    dq = np.full(q.shape, np.nan)
+    dk = np.full(k.shape, np.nan)
+    dv = np.full(v.shape, np.nan)
+    todo = heads if heads is not None else [(b, g) for b in range(B) for g in range(Hkv)]
+    for b, g in todo:
+        dk[b, g] = 0.0
+        dv[b, g] = 0.0
+        for h in (h for h in range(Hq) if _kv_head(h, Hq, Hkv) == g):
+            dqh, dkh, dvh = _head_bwd(q[b, h], k[b, g], v[b, g], do[b, h], scale, causal, window)
+            dq[b, h] = dqh
+            dk[b, g] += dkh
+            dv[b, g] += dvh
+    return dq, dk, dv

@@ -1,0 +1,380 @@
+"""Pins for the float64 oracle, checked against facts the pages and mathematics fix.
+
+Every test here runs on the CPU.  Each pin is chosen so that a plausible slip
+in the oracle (a dropped mask, a wrong sign, a transposed operand, a missing
+scale, a wrong GQA head mapping) makes at least one of them fail; the last
+group of tests plants such slips and checks that.
+"""
+
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import attention as oa
+from synth import make_shape_inputs, bf16_bits_to_f32
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+RNG = np.random.default_rng(2024)
+
+
+def _rand(*shape):
+    return RNG.standard_normal(shape)
+
+
+# ---------------------------------------------------------------- worked example
+def test_golden_hand_worked_example():
+    """Hand-derived 3x3 example (fixture cites the definition it follows)."""
+    g = json.load(open(os.path.join(GOLDEN, "hand_worked_3x3.json")))
+    q = np.array(g["q"], float)[None, None]
+    k = np.array(g["k"], float)[None, None]
+    v = np.array(g["v"], float)[None, None]
+    for case in g["cases"]:
+        O, lse = oracle.attn_fwd(q, k, v, g["scale"], case["causal"], case["window"])
+        np.testing.assert_allclose(O[0, 0], np.array(case["O"]), rtol=0, atol=1e-14)
+        np.testing.assert_allclose(lse[0, 0], np.array(case["LSE"]), rtol=0, atol=1e-14)
+    bw = g["backward"]
+    dq, dk, dv = oracle.attn_bwd(q, k, v, np.array(bw["dO"], float)[None, None],
+                                 g["scale"], bw["causal"], bw["window"])
+    np.testing.assert_allclose(dq[0, 0], bw["dQ"], atol=1e-14)
+    np.testing.assert_allclose(dk[0, 0], bw["dK"], atol=1e-14)
+    np.testing.assert_allclose(dv[0, 0], bw["dV"], atol=1e-14)
+
+
+# ---------------------------------------------------------------- invariants
+MASKS = [(False, 0), (True, 0), (True, 5), (True, 1), (True, 64)]
+
+
+@pytest.mark.parametrize("causal,window", MASKS)
+def test_rows_sum_to_one_masked_exact_zero(causal, window):
+    """Each row of A sums to 1; invisible entries are exactly 0 (-inf logit)."""
+    Lq, Lk, d = 37, 37, 8
+    q, k = _rand(Lq, d), _rand(Lk, d)
+    vis = oracle.visible_mask(Lq, Lk, causal, window)
+    A, _ = oracle.attention_weights(q, k, 0.7, vis)
+    np.testing.assert_allclose(A.sum(1), 1.0, atol=1e-14)
+    assert np.all(A[~vis] == 0.0)
+    assert np.all(A[vis] > 0.0)
+
+
+def test_visible_mask_definition():
+    """Causal: j <= i.  Window w: i - w < j <= i (w keys including self)."""
+    vis = oracle.visible_mask(6, 6, True, 3)
+    for i in range(6):
+        assert list(np.nonzero(vis[i])[0]) == list(range(max(0, i - 2), i + 1))
+    assert oracle.visible_mask(4, 4, False, 0).all()
+    assert (oracle.visible_mask(5, 5, True, 0) == np.tril(np.ones((5, 5), bool))).all()
+
+
+@pytest.mark.parametrize("causal,window", MASKS)
+def test_output_in_convex_hull(causal, window):
+    """Output row i is a convex combination of the visible V rows."""
+    Lq = Lk = 29
+    d = 6
+    q, k, v = _rand(1, 1, Lq, d), _rand(1, 1, Lk, d), _rand(1, 1, Lk, d)
+    O, _ = oracle.attn_fwd(q, k, v, 0.4, causal, window)
+    vis = oracle.visible_mask(Lq, Lk, causal, window)
+    for i in range(Lq):
+        vv = v[0, 0][vis[i]]
+        assert np.all(O[0, 0, i] <= vv.max(0) + 1e-12)
+        assert np.all(O[0, 0, i] >= vv.min(0) - 1e-12)
+
+
+@pytest.mark.parametrize("causal,window", MASKS)
+def test_zero_query_gives_mean_of_visible(causal, window):
+    """Q = 0: all visible logits equal, so O_i is the mean of visible V and LSE = ln(count)."""
+    Lq = Lk = 23
+    d = 5
+    q = np.zeros((1, 1, Lq, d))
+    k, v = _rand(1, 1, Lk, d), _rand(1, 1, Lk, d)
+    O, lse = oracle.attn_fwd(q, k, v, 1.3, causal, window)
+    vis = oracle.visible_mask(Lq, Lk, causal, window)
+    for i in range(Lq):
+        np.testing.assert_allclose(O[0, 0, i], v[0, 0][vis[i]].mean(0), atol=1e-14)
+        assert abs(lse[0, 0, i] - math.log(vis[i].sum())) < 1e-14
+
+
+def test_single_visible_key_returns_that_row():
+    """Causal row 0 and window w=1 each see one key: O_i = V_j exactly, LSE = S_ij."""
+    L, d = 11, 7
+    q, k, v = _rand(1, 1, L, d), _rand(1, 1, L, d), _rand(1, 1, L, d)
+    O, lse = oracle.attn_fwd(q, k, v, 0.3, True, 0)
+    assert np.array_equal(O[0, 0, 0], v[0, 0, 0])
+    assert abs(lse[0, 0, 0] - 0.3 * q[0, 0, 0] @ k[0, 0, 0]) < 1e-14
+    O, lse = oracle.attn_fwd(q, k, v, 0.3, True, 1)
+    assert np.array_equal(O[0, 0], v[0, 0])
+    np.testing.assert_allclose(lse[0, 0], 0.3 * np.sum(q[0, 0] * k[0, 0], 1), atol=1e-14)
+
+
+def test_value_shift_and_score_shift_invariance():
+    """V + 1 c^T gives O + 1 c^T; a per-row constant added to the logits changes nothing."""
+    L, d = 19, 4
+    q, k, v = _rand(1, 1, L, d), _rand(1, 1, L, d), _rand(1, 1, L, d)
+    c = _rand(d)
+    O, lse = oracle.attn_fwd(q, k, v, 0.5, True, 7)
+    O2, _ = oracle.attn_fwd(q, k, v + c, 0.5, True, 7)
+    np.testing.assert_allclose(O2, O + c, atol=1e-13)
+    # Give every key the same component along u; shifting q along u adds a
+    # per-row constant to its logits.
+    u = np.zeros(d + 1)
+    u[-1] = 1.0
+    k1 = np.concatenate([k, np.ones((1, 1, L, 1))], -1)
+    v1 = v
+    q1 = np.concatenate([q, np.zeros((1, 1, L, 1))], -1)
+    q2 = q1 + 3.0 * u
+    Oa, la = oracle.attn_fwd(q1, k1, v1, 0.5, True, 7)
+    Ob, lb = oracle.attn_fwd(q2, k1, v1, 0.5, True, 7)
+    np.testing.assert_allclose(Ob, Oa, atol=1e-13)
+    np.testing.assert_allclose(lb, la + 1.5, atol=1e-13)
+
+
+def _online_softmax_attention(q, k, v, scale, vis, block):
+    """The streaming recurrence of "高效注意力：FlashAttention 与线性注意力" (原理与机制):
+    keep a running max m and running sum l per row; merge each key block by
+    rescaling the old sum and the old output by e^{m_old - m_new}."""
+    Lq, d = q.shape[0], v.shape[1]
+    m = np.full(Lq, -np.inf)
+    l = np.zeros(Lq)
+    acc = np.zeros((Lq, d))
+    for j0 in range(0, k.shape[0], block):
+        s = scale * q @ k[j0:j0 + block].T
+        s = np.where(vis[:, j0:j0 + block], s, -np.inf)
+        m_new = np.maximum(m, s.max(1))
+        safe = np.where(np.isfinite(m_new), m_new, 0.0)
+        alpha = np.where(np.isfinite(m), np.exp(m - safe), 0.0)
+        p = np.exp(s - safe[:, None])
+        l = l * alpha + p.sum(1)
+        acc = acc * alpha[:, None] + p @ v[j0:j0 + block]
+        m = m_new
+    O = np.divide(acc, l[:, None], out=np.zeros_like(acc), where=l[:, None] > 0)
+    with np.errstate(divide="ignore"):
+        lse = np.where(l > 0, m + np.log(l), -np.inf)
+    return O, lse
+
+
+@pytest.mark.parametrize("block", [1, 3, 7, 16, 64])
+@pytest.mark.parametrize("causal,window", MASKS)
+def test_block_split_online_softmax_equals_full(block, causal, window):
+    L, d = 45, 8
+    q, k, v = _rand(L, d), _rand(L, d), _rand(L, d)
+    vis = oracle.visible_mask(L, L, causal, window)
+    O, lse = oracle.attn_fwd(q[None, None], k[None, None], v[None, None], 0.35, causal, window)
+    O2, lse2 = _online_softmax_attention(q, k, v, 0.35, vis, block)
+    np.testing.assert_allclose(O2, O[0, 0], atol=1e-12)
+    np.testing.assert_allclose(lse2, lse[0, 0], atol=1e-12)
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(4, 2), (6, 1), (8, 8), (32, 8)])
+def test_gqa_equals_mha_with_repeated_kv(Hq, Hkv):
+    """Query head h uses K/V head h // (Hq/Hkv): equal to MHA with K/V repeated."""
+    B, L, d = 2, 13, 4
+    q = _rand(B, Hq, L, d)
+    k, v = _rand(B, Hkv, L, d), _rand(B, Hkv, L, d)
+    G = Hq // Hkv
+    kr, vr = np.repeat(k, G, axis=1), np.repeat(v, G, axis=1)
+    O, lse = oracle.attn_fwd(q, k, v, 0.5, True, 4)
+    Or, lser = oracle.attn_fwd(q, kr, vr, 0.5, True, 4)
+    np.testing.assert_array_equal(O, Or)
+    np.testing.assert_array_equal(lse, lser)
+    do = _rand(B, Hq, L, d)
+    dq, dk, dv = oracle.attn_bwd(q, k, v, do, 0.5, True, 4)
+    dqr, dkr, dvr = oracle.attn_bwd(q, kr, vr, do, 0.5, True, 4)
+    np.testing.assert_allclose(dq, dqr, atol=1e-14)
+    np.testing.assert_allclose(dk, dkr.reshape(B, Hkv, G, L, d).sum(2), atol=1e-13)
+    np.testing.assert_allclose(dv, dvr.reshape(B, Hkv, G, L, d).sum(2), atol=1e-13)
+
+
+# ---------------------------------------------------------------- backward
+def _loss(q, k, v, R, scale, causal, window):
+    O, _ = oracle.attn_fwd(q, k, v, scale, causal, window)
+    return float(np.sum(O * R))
+
+
+@pytest.mark.parametrize("Hq,Hkv,L,causal,window", [
+    (2, 2, 9, False, 0), (2, 2, 9, True, 0), (2, 1, 8, True, 3), (2, 2, 7, True, 1),
+    (4, 2, 6, False, 0),
+])
+def test_backward_matches_finite_differences(Hq, Hkv, L, causal, window):
+    """Gradient of <R, O> against central differences, float64, to 1e-6."""
+    rng = np.random.default_rng(7)
+    d = 4
+    q = rng.standard_normal((1, Hq, L, d))
+    k = rng.standard_normal((1, Hkv, L, d))
+    v = rng.standard_normal((1, Hkv, L, d))
+    R = rng.standard_normal((1, Hq, L, d))
+    scale = 0.6
+    dq, dk, dv = oracle.attn_bwd(q, k, v, R, scale, causal, window)
+    eps = 1e-5
+    for X, G in ((q, dq), (k, dk), (v, dv)):
+        num = np.zeros_like(X)
+        it = np.nditer(X, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            old = X[idx]
+            X[idx] = old + eps
+            fp = _loss(q, k, v, R, scale, causal, window)
+            X[idx] = old - eps
+            fm = _loss(q, k, v, R, scale, causal, window)
+            X[idx] = old
+            num[idx] = (fp - fm) / (2 * eps)
+        np.testing.assert_allclose(G, num, atol=1e-6, rtol=0)
+
+
+def test_fully_masked_rows_are_zero():
+    """Lq > Lk with a window leaves late rows with no visible key: O=0, LSE=-inf, dQ=0."""
+    Lq, Lk, d, w = 12, 4, 3, 3
+    q, k, v = _rand(1, 1, Lq, d), _rand(1, 1, Lk, d), _rand(1, 1, Lk, d)
+    vis = oracle.visible_mask(Lq, Lk, True, w)
+    dead = ~vis.any(1)
+    assert dead.sum() > 0
+    O, lse = oracle.attn_fwd(q, k, v, 0.5, True, w)
+    assert np.all(O[0, 0][dead] == 0) and np.all(np.isneginf(lse[0, 0][dead]))
+    assert np.all(np.isfinite(O))
+    dq, dk, dv = oracle.attn_bwd(q, k, v, _rand(1, 1, Lq, d), 0.5, True, w)
+    assert np.all(dq[0, 0][dead] == 0)
+    assert np.all(np.isfinite(dk)) and np.all(np.isfinite(dv))
+
+
+def test_row_blocking_is_invisible(monkeypatch):
+    """Evaluating a head in small row blocks over their bands gives the same numbers."""
+    L, d = 70, 8
+    q, k, v, do = (_rand(1, 2, L, d) for _ in range(4))
+    ref = oracle.attn_fwd(q, k, v, 0.4, True, 9)
+    refb = oracle.attn_bwd(q, k, v, do, 0.4, True, 9)
+    monkeypatch.setattr(oa, "_ROW_BLOCK_ELEMS", 3 * L)
+    blk = oracle.attn_fwd(q, k, v, 0.4, True, 9)
+    blkb = oracle.attn_bwd(q, k, v, do, 0.4, True, 9)
+    for a, b in zip(ref + refb, blk + blkb):
+        np.testing.assert_allclose(a, b, atol=1e-14)
+    rows = np.array([0, 5, 33, 69])
+    Orow, lrow = oracle.attn_fwd_rows(q, k, v, 0.4, True, 9, 0, 1, rows)
+    np.testing.assert_allclose(Orow, ref[0][0, 1, rows], atol=1e-14)
+    np.testing.assert_allclose(lrow, ref[1][0, 1, rows], atol=1e-14)
+
+
+# ---------------------------------------------------------------- library cross-checks
+torch = pytest.importorskip("torch")
+
+
+@pytest.mark.parametrize("Hq,Hkv,causal,window", [
+    (4, 4, False, 0), (4, 4, True, 0), (4, 2, True, 0), (4, 1, True, 6), (2, 2, True, 1),
+])
+def test_matches_torch_sdpa_float64(Hq, Hkv, causal, window):
+    """Special case that reduces to a library routine: torch CPU float64 SDPA (test only)."""
+    B, L, d = 2, 33, 16
+    q, k, v = _rand(B, Hq, L, d), _rand(B, Hkv, L, d), _rand(B, Hkv, L, d)
+    O, _ = oracle.attn_fwd(q, k, v, 0.25, causal, window)
+    tq, tk, tv = (torch.from_numpy(x) for x in (q, k, v))
+    G = Hq // Hkv
+    tk, tv = tk.repeat_interleave(G, 1), tv.repeat_interleave(G, 1)
+    mask = torch.from_numpy(oracle.visible_mask(L, L, causal, window))
+    ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=mask, scale=0.25)
+    np.testing.assert_allclose(O, ref.numpy(), atol=1e-12)
+
+
+def test_pages_fp32_experiment_magnitude():
+    """"缩放定律与高效注意力" 实验 1: B=2,H=4,L=128,d=32, seed 42, fp32 manual vs fused
+    attention differ by about 4.5e-7 (rounding order only).  Both fp32 results sit
+    within that order of magnitude of the exact float64 oracle."""
+    torch.manual_seed(42)
+    B, H, L, d = 2, 4, 128, 32
+    q, k, v = [torch.randn(B, H, L, d) for _ in range(3)]
+    manual = (q @ k.transpose(-2, -1) / d ** 0.5).softmax(-1) @ v
+    fused = torch.nn.functional.scaled_dot_product_attention(q, k, v)
+    exact, _ = oracle.attn_fwd(q.double().numpy(), k.double().numpy(), v.double().numpy(),
+                               1 / math.sqrt(d))
+    e1 = np.abs(manual.double().numpy() - exact).max()
+    e2 = np.abs(fused.double().numpy() - exact).max()
+    assert e1 < 5e-6 and e2 < 5e-6
+    assert (manual - fused).abs().max().item() < 5e-6
+
+
+# ---------------------------------------------------------------- input recipe
+def test_bf16_rounding_matches_torch():
+    """The generator's float32 -> bf16 rounding is round-to-nearest-even."""
+    from synth import f32_to_bf16_bits
+    x = np.random.default_rng(3).standard_normal(10000).astype(np.float32) * 37
+    x[:4] = [1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -0.0, 65504.0]
+    ours = f32_to_bf16_bits(x)
+    ref = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(ours, ref)
+
+
+def test_inputs_are_seeded_and_exact_bf16():
+    a = make_shape_inputs(1, 2, 1, 5, 5, 8, seed=11, with_do=True)
+    b = make_shape_inputs(1, 2, 1, 5, 5, 8, seed=11, with_do=True)
+    for n in "q", "k", "v", "do":
+        assert np.array_equal(a[n], b[n])
+    x = bf16_bits_to_f32(a["q"])
+    assert np.array_equal(x.view(np.uint32) & 0xFFFF, np.zeros_like(x, dtype=np.uint32))
+
+
+# ---------------------------------------------------------------- planted slips
+def _pins_pass():
+    """Run a compact subset of the pins; False if any fails."""
+    checks = [test_golden_hand_worked_example,
+              lambda: test_zero_query_gives_mean_of_visible(True, 5),
+              lambda: test_gqa_equals_mha_with_repeated_kv(4, 2),
+              lambda: test_backward_matches_finite_differences(2, 1, 8, True, 3),
+              lambda: test_matches_torch_sdpa_float64(4, 2, True, 0)]
+    for c in checks:
+        try:
+            c()
+        except AssertionError:
+            return False
+    return True
+
+
+def test_pins_pass_unmodified():
+    assert _pins_pass()
+
+
+@pytest.mark.parametrize("slip", ["transpose", "no_mask", "dS_sign", "dk_no_scale", "gqa_map"])
+def test_pins_catch_planted_slips(monkeypatch, slip):
+    """Plant a plausible mistake in the oracle (CPU only) and check a pin fails."""
+    if slip == "transpose":
+        orig = oa.attention_weights
+        monkeypatch.setattr(oa, "attention_weights",
+                            lambda q, k, s, vis: _transposed_weights(orig, q, k, s, vis))
+    elif slip == "no_mask":
+        orig = oa.attention_weights
+        monkeypatch.setattr(oa, "attention_weights",
+                            lambda q, k, s, vis: orig(q, k, s, np.ones_like(vis)))
+    elif slip == "dS_sign":
+        monkeypatch.setattr(oa, "_head_bwd", _bwd_with(lambda A, dP, D: A * (dP + D)))
+    elif slip == "dk_no_scale":
+        monkeypatch.setattr(oa, "_head_bwd", _bwd_with(None, dk_scale=False))
+    elif slip == "gqa_map":
+        monkeypatch.setattr(oa, "_kv_head", lambda h, Hq, Hkv: h % Hkv)
+    assert not _pins_pass()
+
+
+def _transposed_weights(orig, q, k, s, vis):
+    # scores built as K Q^T instead of Q K^T (only changes square, unmasked cases)
+    if q.shape[0] == k.shape[0]:
+        S = s * (k @ q.T)
+        S = np.where(vis, S, -np.inf)
+        m = np.max(S, 1, keepdims=True)
+        m = np.where(np.isfinite(m), m, 0)
+        E = np.where(vis, np.exp(S - m), 0)
+        l = E.sum(1, keepdims=True)
+        A = np.divide(E, l, out=np.zeros_like(E), where=l > 0)
+        with np.errstate(divide="ignore"):
+            return A, np.where(l[:, 0] > 0, m[:, 0] + np.log(l[:, 0]), -np.inf)
+    return orig(q, k, s, vis)
+
+
+def _bwd_with(ds_fn, dk_scale=True):
+    def head_bwd(qh, kh, vh, doh, scale, causal, window):
+        Lq, Lk = qh.shape[0], kh.shape[0]
+        vis = oracle.visible_mask(Lq, Lk, causal, window)
+        A, _ = oa.attention_weights(qh, kh, scale, vis)
+        O = A @ vh
+        dP = doh @ vh.T
+        D = np.sum(doh * O, 1, keepdims=True)
+        dS = ds_fn(A, dP, D) if ds_fn else A * (dP - D)
+        return scale * dS @ kh, (scale if dk_scale else 1.0) * dS.T @ qh, A.T @ doh
+    return head_bwd
