@@ -1,0 +1,133 @@
+/*
+ * tiledattn.h - C ABI of the tiled exact attention library (sm_100a, B200).
+ *
+ * The library computes exact scaled-dot-product attention
+ *
+ *     O = softmax(scale * Q K^T + mask) V
+ *
+ * ("注意力优化：FlashAttention 与稀疏注意力", 核心公式: S = QK^T/sqrt(d_k), a row
+ * softmax whose rows sum to 1, output row i = sum_j A_ij V_j, and disallowed
+ * keys set to -inf before the softmax), tile by tile with an online softmax so
+ * that the score matrix never reaches device memory ("缩放定律与高效注意力"
+ * §3.2, tiling and the incremental max/sum; "高效注意力：FlashAttention 与线性
+ * 注意力", 原理与机制: the running max and sum rescaled by e^{m_old - m_new}).
+ * The backward pass recomputes the scores from the saved output and per-row
+ * logsumexp ("缩放定律与高效注意力" §3.3).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Tensors are contiguous, row-major, [B, H, L, d]; Q/O/dO/dQ have H = Hq,
+ *    K/V/dK/dV have H = Hkv.  bf16 tensors hold IEEE bfloat16 bit patterns.
+ *  - GQA/MQA ("高效注意力" §3): Hq must be a multiple of Hkv; query head h
+ *    reads K/V head h / (Hq / Hkv) (contiguous groups).
+ *  - Masks: causal = 1 makes key j visible to query i only if j <= i (top-left
+ *    alignment).  window = w > 0 (requires causal = 1) further restricts it to
+ *    i - w < j <= i: the w most recent keys including i itself ("高效注意力"
+ *    §4, sliding-window attention).  window = 0 means no window.
+ *  - A query row that sees no key gets O = 0 and LSE = -inf (and dQ = 0).
+ *  - LSE is the natural logarithm of sum_j exp(scale * q_i . k_j) over visible j.
+ *  - Supported head dimension: d = 64 or d = 128 (d_k = d_v = d).
+ *  - Every device pointer must be 16-byte aligned and point to memory of the
+ *    current CUDA device.  All buffers are owned by the caller; the library
+ *    allocates nothing and keeps no pointer after a call returns.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Calls are asynchronous on that stream.  Argument errors are detected and
+ *    returned before anything is launched; launch failures return
+ *    ATTN_ERR_CUDA.  No C++ exception crosses this interface.
+ *  - Every device-side wait is bounded.  If a kernel gives up waiting, it
+ *    records ATTN_ERR_TIMEOUT in a per-device error word, which
+ *    attn_get_device_error() reports; its outputs are then undefined.
+ *  - Empty problems (B, Hq, Lq = 0) are valid and launch nothing.  Lk = 0 is
+ *    valid: every row sees no key.
+ */
+#ifndef TILEDATTN_H
+#define TILEDATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ATTN_API __attribute__((visibility("default")))
+#else
+#define ATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = 1, /* null/misaligned pointer, negative size, bad mask, Hq % Hkv != 0 */
+  ATTN_ERR_UNSUPPORTED = 2, /* valid but not implemented (head dim other than 64/128, too large) */
+  ATTN_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed */
+  ATTN_ERR_TIMEOUT = 4      /* a kernel abandoned a bounded wait (see attn_get_device_error) */
+} attn_status;
+
+/*
+ * Forward pass ("缩放定律与高效注意力" §3.2; output O and the per-row logsumexp
+ * that §3.3 says the backward pass needs).
+ *
+ *  q    bf16 [B, Hq,  Lq, d]   input
+ *  k    bf16 [B, Hkv, Lk, d]   input
+ *  v    bf16 [B, Hkv, Lk, d]   input
+ *  o    bf16 [B, Hq,  Lq, d]   output (rounded to nearest even from fp32)
+ *  lse  fp32 [B, Hq,  Lq]      output, natural log
+ *  scale  multiplies Q K^T (1/sqrt(d) for standard attention); must be finite
+ *
+ * Returns ATTN_OK or an attn_status error code.
+ */
+ATTN_API int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Lq,
+             int Lk, int d, float scale, int causal, int window, void* stream);
+
+/*
+ * Bytes of device workspace attn_bwd needs for this shape: the per-row
+ * D_i = dO_i . O_i (fp32 [B,Hq,Lq]) and an fp32 dQ accumulator [B,Hq,Lq,d].
+ * Returns 0 for an empty problem or invalid sizes.
+ */
+ATTN_API size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int Lq, int Lk, int d);
+
+/*
+ * Backward pass by recomputation ("缩放定律与高效注意力" §3.3: only O and the
+ * per-row logsumexp are kept; Q, K, V are re-read and the scores rebuilt tile
+ * by tile).  Gradients are the textbook softmax gradient:
+ *   D_i = dO_i . O_i,  P = exp(scale*S - LSE),  dV = P^T dO,  dP = dO V^T,
+ *   dS = P * (dP - D),  dQ = scale * dS K,  dK = scale * dS^T Q.
+ *
+ *  q, k, v, o, lse   the forward's inputs and outputs (same shapes as above)
+ *  dO   bf16 [B, Hq, Lq, d]   upstream gradient
+ *  dq   bf16 [B, Hq, Lq, d]   output
+ *  dk   bf16 [B, Hkv, Lk, d]  output, summed over the Hq/Hkv query heads of a group
+ *  dv   bf16 [B, Hkv, Lk, d]  output, summed likewise
+ *  workspace  device buffer of at least attn_bwd_workspace_size(...) bytes,
+ *             256-byte aligned; its contents on entry do not matter
+ */
+ATTN_API int attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO, void* dq,
+             void* dk, void* dv, int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale, int causal, int window,
+             void* workspace, size_t workspace_bytes, void* stream);
+
+/* Static, human-readable name of a status code. */
+ATTN_API const char* attn_status_string(int status);
+
+/*
+ * Synchronises `stream`, then reads and clears the current device's error
+ * word.  Returns ATTN_OK, ATTN_ERR_TIMEOUT if a kernel gave up a bounded wait
+ * since the last call, or ATTN_ERR_CUDA if the synchronisation failed.
+ * If `site` is not NULL it receives the internal wait-site id of a timeout.
+ */
+ATTN_API int attn_get_device_error(void* stream, int* site);
+
+/*
+ * Self-test of the bounded-wait mechanism: launches one CTA that waits on a
+ * barrier nothing ever completes, with a limit of `limit_ns` nanoseconds.
+ * The kernel gives up, records ATTN_ERR_TIMEOUT and exits normally; the
+ * caller then sees it through attn_get_device_error().  Returns the launch
+ * status.  No counterpart on the pages: it exists to test failure handling.
+ */
+ATTN_API int attn_selftest_wait_timeout(int64_t limit_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TILEDATTN_H */

@@ -1,0 +1,99 @@
+"""The C-ABI library: loads, exports every declared symbol, validates arguments.
+
+Runs on the CPU: only calls that must fail validation (or are empty) are made,
+and those return before touching the GPU.
+"""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            names += re.findall(r"^ATTN_API\s+[\w\s\*]+?\b(\w+)\(", text, re.M)
+    return names
+
+
+@pytest.fixture(scope="module")
+def ta():
+    from tiled_exact_attention_02_b200 import build
+    build.build()
+    import tiled_exact_attention_02_b200 as ta
+    return ta
+
+
+def test_every_declared_symbol_is_exported(ta):
+    names = _declared()
+    assert {"attn_fwd", "attn_bwd", "attn_bwd_workspace_size", "attn_status_string",
+            "attn_get_device_error"} <= set(names)
+    lib = ctypes.CDLL(ta.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(ta):
+    assert ta.status_string(0) == "ATTN_OK"
+    assert ta.status_string(1) == "ATTN_ERR_INVALID_ARG"
+    assert ta.status_string(4) == "ATTN_ERR_TIMEOUT"
+    assert ta.status_string(77) == "ATTN_ERR_UNKNOWN"
+
+
+P = 1 << 20  # a 16-byte aligned fake address: never dereferenced, validation fails first
+
+
+def _fwd(ta, B=1, Hq=2, Hkv=2, Lq=8, Lk=8, d=64, scale=0.125, causal=0, window=0, q=P, k=P, v=P, o=P, lse=P):
+    return ta.lib.attn_fwd(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, scale, causal, window, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(d=96), 2), (dict(d=256), 2), (dict(Hq=3, Hkv=2), 1), (dict(Hkv=0), 1),
+    (dict(B=-1), 1), (dict(Lq=-5), 1), (dict(window=4), 1), (dict(causal=1, window=-1), 1),
+    (dict(causal=2), 1), (dict(scale=0.0), 1), (dict(scale=-1.0), 1), (dict(scale=float("nan")), 1),
+    (dict(scale=float("inf")), 1), (dict(q=0), 1), (dict(o=P + 8), 1), (dict(lse=P + 4), 1),
+    (dict(k=0), 1), (dict(v=P + 2), 1),
+])
+def test_fwd_rejects_bad_arguments(ta, kw, status):
+    assert _fwd(ta, **kw) == status
+
+
+@pytest.mark.parametrize("kw", [dict(B=0), dict(Hq=0, Hkv=0), dict(Lq=0)])
+def test_fwd_empty_problem_is_a_no_op(ta, kw):
+    assert _fwd(ta, q=0, k=0, v=0, o=0, lse=0, **kw) == 0
+
+
+def _bwd(ta, B=1, Hq=2, Hkv=1, Lq=8, Lk=8, d=128, scale=0.1, causal=1, window=0, ptrs=None, ws=P, wsb=1 << 20):
+    p = ptrs or [P] * 9
+    return ta.lib.attn_bwd(*p, B, Hq, Hkv, Lq, Lk, d, scale, causal, window, ws, wsb, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(d=80), 2), (dict(Hq=3), 1), (dict(window=3, causal=0), 1), (dict(ws=0), 1),
+    (dict(wsb=16), 1), (dict(ptrs=[P] * 5 + [0] + [P] * 3), 1), (dict(ptrs=[P] * 8 + [P + 1]), 1),
+    (dict(scale=0.0), 1), (dict(ws=P + 64), 1),
+])
+def test_bwd_rejects_bad_arguments(ta, kw, status):
+    assert _bwd(ta, **kw) == status
+
+
+def test_bwd_workspace_size(ta):
+    n = ta.bwd_workspace_size(2, 4, 2, 100, 50, 64)
+    rows = 2 * 4 * 100
+    assert n == -(-rows * 4 // 256) * 256 + -(-rows * 64 * 4 // 256) * 256
+    assert ta.bwd_workspace_size(0, 4, 2, 100, 50, 64) == 0
+    assert ta.bwd_workspace_size(1, 3, 2, 100, 50, 64) == 0
+    assert ta.bwd_workspace_size(1, 4, 2, 100, 50, 72) == 0
+
+
+def test_binding_has_no_cpu_path(ta):
+    """The binding only marshals: no numpy/torch attention math in the package."""
+    src = open(os.path.join(ROOT, "tiled_exact_attention_02_b200", "__init__.py")).read()
+    for banned in ("softmax", "oracle", "matmul", "@", "scaled_dot_product"):
+        assert banned not in src.replace("@staticmethod", ""), banned

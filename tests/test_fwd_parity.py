@@ -1,0 +1,127 @@
+"""Forward parity: the CUDA path (through the C ABI) against the float64 oracle.
+
+Same seeded bf16 inputs on both sides.  Tolerances: O max-abs 1e-2 and
+relative Frobenius 5e-3; LSE 1e-5 relative (absolute below |LSE| = 1).
+"""
+
+import numpy as np
+import pytest
+
+import oracle
+from synth import WORKLOADS, make_inputs, make_shape_inputs
+from tests._util import check_lse, check_o, to_dev, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def ta():
+    import torch
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    import tiled_exact_attention_02_b200 as ta
+    return ta
+
+
+def run_fwd(ta, x, causal, window, scale):
+    q, k, v = (to_dev(x[n]) for n in "qkv")
+    o, lse = ta.attention(q, k, v, causal, window, scale)
+    st, site = ta.device_error()
+    assert st == 0, f"device error {st} at site {site}"
+    return to_f64(o), to_f64(lse)
+
+
+# (B, Hq, Hkv, Lq, Lk, d, causal, window): tails, partial tiles, masks, groups
+EDGE = [
+    (1, 1, 1, 1, 1, 64, False, 0),
+    (1, 2, 2, 7, 7, 128, True, 0),
+    (1, 2, 1, 129, 129, 64, True, 0),
+    (2, 4, 2, 200, 200, 128, True, 0),
+    (1, 2, 2, 100, 333, 128, False, 0),
+    (1, 2, 2, 333, 100, 64, False, 0),
+    (1, 4, 4, 257, 257, 64, True, 1),
+    (1, 2, 2, 384, 384, 128, True, 1000),
+    (1, 8, 1, 256, 256, 128, True, 0),
+    (1, 6, 2, 300, 300, 128, True, 64),
+    (1, 3, 3, 640, 640, 128, True, 130),
+    (1, 2, 2, 300, 100, 128, True, 50),
+    (2, 2, 2, 513, 513, 64, False, 0),
+    (1, 4, 2, 1000, 1000, 128, True, 0),
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Lq,Lk,d,causal,window", EDGE)
+def test_fwd_edge_shapes(ta, B, Hq, Hkv, Lq, Lk, d, causal, window):
+    x = make_shape_inputs(B, Hq, Hkv, Lq, Lk, d, seed=Lq * 7 + Lk + d)
+    scale = d ** -0.5
+    o, lse = run_fwd(ta, x, causal, window, scale)
+    ro, rl = oracle.attn_fwd(x["q"], x["k"], x["v"], scale, causal, window)
+    check_o(o, ro, "O")
+    check_lse(lse, rl, "LSE")
+
+
+def test_fwd_no_keys(ta):
+    """Lk = 0: every row sees nothing: O = 0, LSE = -inf."""
+    import torch
+    x = make_shape_inputs(1, 2, 2, 50, 1, 64, seed=5)
+    q = to_dev(x["q"])
+    k = torch.empty((1, 2, 0, 64), dtype=torch.bfloat16, device="cuda")
+    o, lse = ta.attention(q, k, k, False, 0, 0.125)
+    assert torch.all(o == 0) and torch.all(torch.isneginf(lse))
+
+
+def test_fwd_sharp_softmax_rescales(ta):
+    """Large logits (Q scaled by 8) force the lazy rescale path many times per row.
+
+    Far sharper than any benchmark workload, so the max-abs bound is derived
+    from the arithmetic instead: P enters P.V rounded to bf16 (relative error
+    <= 2^-9 per weight, so <= 2^-9 max|V| on a convex combination) and O is
+    rounded to bf16 once more (<= 2^-9 |O| <= 2^-9 max|V|).
+    """
+    x = make_shape_inputs(1, 2, 2, 1024, 1024, 128, seed=99, q_mult=8.0)
+    o, lse = run_fwd(ta, x, True, 0, 128 ** -0.5)
+    ro, rl = oracle.attn_fwd(x["q"], x["k"], x["v"], 128 ** -0.5, True, 0)
+    vmax = float(np.max(np.abs(oracle.attention._f64(x["v"]))))
+    assert np.max(np.abs(o - ro)) <= 2.0 ** -8 * vmax * 1.05
+    from tests._util import rel_fro
+    assert rel_fro(o, ro) <= 5e-3
+    check_lse(lse, rl, "LSE")
+
+
+def test_fwd_single_head_128(ta):
+    w = WORKLOADS["single_head_128"]
+    x = make_inputs(w)
+    o, lse = run_fwd(ta, x, w.causal, w.window, w.scale)
+    ro, rl = oracle.attn_fwd(x["q"], x["k"], x["v"], w.scale, w.causal, w.window)
+    check_o(o, ro, "O")
+    check_lse(lse, rl, "LSE")
+
+
+@pytest.mark.parametrize("name,heads", [
+    ("mha_causal_4096", [(0, 0), (1, 31), (0, 17)]),
+    ("gqa_causal_8192", [(0, 0), (3, 31), (2, 9)]),
+    ("gqa_window_32768", [(0, 0), (0, 21)]),
+])
+def test_fwd_full_size_sampled_heads(ta, name, heads):
+    """Full-size workloads in the benchmark's launch configuration; whole heads
+    (independent units) are compared against the oracle."""
+    w = WORKLOADS[name]
+    x = make_inputs(w)
+    o, lse = run_fwd(ta, x, w.causal, w.window, w.scale)
+    ro, rl = oracle.attn_fwd(x["q"], x["k"], x["v"], w.scale, w.causal, w.window, heads=heads)
+    for b, h in heads:
+        check_o(o[b, h], ro[b, h], f"{name} O[{b},{h}]")
+        check_lse(lse[b, h], rl[b, h], f"{name} LSE[{b},{h}]")
+    assert np.all(np.isfinite(o))
+
+
+def test_bounded_wait_reports_timeout(ta):
+    """A wait that nothing completes gives up and reports ATTN_ERR_TIMEOUT;
+    the context stays usable afterwards."""
+    assert ta.lib.attn_selftest_wait_timeout(50_000_000, None) == 0
+    st, site = ta.device_error()
+    assert st == ta.ATTN_ERR_TIMEOUT and site == 1000
+    assert ta.device_error()[0] == 0
+    x = make_shape_inputs(1, 1, 1, 64, 64, 64, seed=1)
+    o, lse = run_fwd(ta, x, True, 0, 0.125)
+    ro, rl = oracle.attn_fwd(x["q"], x["k"], x["v"], 0.125, True, 0)
+    check_o(o, ro)

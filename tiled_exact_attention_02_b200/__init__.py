@@ -1,0 +1,182 @@
+"""Python binding of libtiledattn.so: argument marshalling only.
+
+Every step of the computation runs in the CUDA kernels behind the C ABI
+(include/tiledattn.h).  PyTorch provides device memory and the current
+stream.  There is no CPU fallback: if the library is missing, importing the
+binding raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libtiledattn.so")
+HEADER = os.path.join(os.path.dirname(HERE), "include", "tiledattn.h")
+
+ATTN_OK = 0
+ATTN_ERR_INVALID_ARG = 1
+ATTN_ERR_UNSUPPORTED = 2
+ATTN_ERR_CUDA = 3
+ATTN_ERR_TIMEOUT = 4
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is not built; run `python -m tiled_exact_attention_02_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, vp]
+    lib.attn_fwd.restype = i
+    lib.attn_bwd_workspace_size.argtypes = [i, i, i, i, i, i]
+    lib.attn_bwd_workspace_size.restype = sz
+    lib.attn_bwd.argtypes = [vp] * 9 + [i] * 6 + [f, i, i, vp, sz, vp]
+    lib.attn_bwd.restype = i
+    lib.attn_status_string.argtypes = [i]
+    lib.attn_status_string.restype = ctypes.c_char_p
+    lib.attn_get_device_error.argtypes = [vp, ctypes.POINTER(i)]
+    lib.attn_get_device_error.restype = i
+    lib.attn_selftest_wait_timeout.argtypes = [ctypes.c_int64, vp]
+    lib.attn_selftest_wait_timeout.restype = i
+    return lib
+
+
+lib = _load()
+
+
+def status_string(status: int) -> str:
+    return lib.attn_status_string(int(status)).decode()
+
+
+def _stream_ptr(stream) -> int:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+def _check(status: int, what: str) -> None:
+    if status != ATTN_OK:
+        raise AttnError(status, what)
+
+
+def _shapes(q, k):
+    B, Hq, Lq, d = q.shape
+    Bk, Hkv, Lk, dk = k.shape
+    if Bk != B or dk != d:
+        raise ValueError(f"shape mismatch q{tuple(q.shape)} k{tuple(k.shape)}")
+    return B, Hq, Hkv, Lq, Lk, d
+
+
+def _require(t, name, dtype=None):
+    import torch
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def fwd(q, k, v, o, lse, causal: bool = False, window: int = 0, scale: float | None = None, stream=None):
+    """attn_fwd on torch tensors (bf16 q/k/v/o, fp32 lse), asynchronous on `stream`."""
+    import torch
+    for n, t in (("q", q), ("k", k), ("v", v), ("o", o)):
+        _require(t, n, torch.bfloat16)
+    _require(lse, "lse", torch.float32)
+    B, Hq, Hkv, Lq, Lk, d = _shapes(q, k)
+    if tuple(v.shape) != tuple(k.shape) or tuple(o.shape) != tuple(q.shape) or tuple(lse.shape) != (B, Hq, Lq):
+        raise ValueError("v/o/lse shape mismatch")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    st = lib.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                      B, Hq, Hkv, Lq, Lk, d, scale, int(bool(causal)), int(window), _stream_ptr(stream))
+    _check(st, "attn_fwd")
+
+
+def bwd_workspace_size(B, Hq, Hkv, Lq, Lk, d) -> int:
+    return int(lib.attn_bwd_workspace_size(B, Hq, Hkv, Lq, Lk, d))
+
+
+def bwd(q, k, v, o, lse, do, dq, dk, dv, workspace, causal: bool = False, window: int = 0,
+        scale: float | None = None, stream=None):
+    """attn_bwd on torch tensors; `workspace` is a uint8 CUDA tensor."""
+    import torch
+    for n, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do), ("dq", dq), ("dk", dk), ("dv", dv)):
+        _require(t, n, torch.bfloat16)
+    _require(lse, "lse", torch.float32)
+    _require(workspace, "workspace")
+    B, Hq, Hkv, Lq, Lk, d = _shapes(q, k)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    st = lib.attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
+                      dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv, Lq, Lk, d, scale,
+                      int(bool(causal)), int(window), workspace.data_ptr(),
+                      workspace.numel() * workspace.element_size(), _stream_ptr(stream))
+    _check(st, "attn_bwd")
+
+
+def device_error(stream=None) -> tuple[int, int]:
+    """(status, site) of the current device's error word; clears it."""
+    site = ctypes.c_int(0)
+    st = lib.attn_get_device_error(_stream_ptr(stream), ctypes.byref(site))
+    return st, site.value
+
+
+def attention(q, k, v, causal: bool = False, window: int = 0, scale: float | None = None):
+    """Allocate O and LSE with torch and run the forward pass."""
+    import torch
+    B, Hq, Hkv, Lq, Lk, d = _shapes(q, k)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
+    fwd(q, k, v, o, lse, causal, window, scale)
+    return o, lse
+
+
+def attention_backward(q, k, v, o, lse, do, causal: bool = False, window: int = 0, scale: float | None = None):
+    """Allocate dQ/dK/dV and the workspace with torch and run the backward pass."""
+    import torch
+    B, Hq, Hkv, Lq, Lk, d = _shapes(q, k)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(max(1, bwd_workspace_size(B, Hq, Hkv, Lq, Lk, d)), dtype=torch.uint8, device=q.device)
+    bwd(q, k, v, o, lse, do, dq, dk, dv, ws, causal, window, scale)
+    return dq, dk, dv
+
+
+def _autograd_function():
+    import torch
+
+    class TiledAttention(torch.autograd.Function):
+        """autograd wrapper: forward saves O and LSE; backward recomputes."""
+
+        @staticmethod
+        def forward(ctx, q, k, v, causal=False, window=0, scale=None):
+            o, lse = attention(q, k, v, causal, window, scale)
+            ctx.save_for_backward(q, k, v, o, lse)
+            ctx.args = (causal, window, scale)
+            return o
+
+        @staticmethod
+        def backward(ctx, do):
+            q, k, v, o, lse = ctx.saved_tensors
+            dq, dk, dv = attention_backward(q, k, v, o, lse, do.contiguous(), *ctx.args)
+            return dq, dk, dv, None, None, None
+
+    return TiledAttention
+
+
+def tiled_attention(q, k, v, causal: bool = False, window: int = 0, scale: float | None = None):
+    """Differentiable attention (torch autograd) backed by the CUDA kernels."""
+    global _TiledAttention
+    try:
+        fn = _TiledAttention
+    except NameError:
+        fn = _TiledAttention = _autograd_function()
+    return fn.apply(q, k, v, causal, window, scale)

@@ -1,0 +1,187 @@
+// api.cu - the C ABI: argument validation, TMA descriptors, launches, and the
+// per-device error word.  See include/tiledattn.h for the contract.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/tiledattn.h"
+#include "attn_kernels.h"
+#include "sm100.cuh"
+
+namespace tea {
+
+// Error word of each device the library runs on: kernels record a bounded
+// wait they gave up on; attn_get_device_error reads and clears it.
+__device__ int g_dev_err;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s without progress
+
+std::mutex g_mu;
+int* g_err_addr[kMaxDevices];
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+// Resolve the driver's tensor-map encoder once (no link-time libcuda dependency).
+int get_encoder(EncodeTiledFn* fn) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_encode) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !p)
+      return ATTN_ERR_CUDA;
+    g_encode = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  *fn = g_encode;
+  return ATTN_OK;
+}
+
+// Device address of the current device's error word (looked up once per device).
+int get_err_word(int** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_err_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_dev_err) != cudaSuccess) return ATTN_ERR_CUDA;
+    g_err_addr[dev] = static_cast<int*>(p);
+  }
+  *out = g_err_addr[dev];
+  return ATTN_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shared shape checks.  Returns ATTN_OK, or the error to report.
+int check_shape(int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale, int causal, int window) {
+  if (B < 0 || Hq < 0 || Hkv < 0 || Lq < 0 || Lk < 0) return ATTN_ERR_INVALID_ARG;
+  if (Hkv == 0 && Hq > 0) return ATTN_ERR_INVALID_ARG;
+  if (Hkv > 0 && Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (Hq == 0 && Hkv > 0) return ATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (window < 0) return ATTN_ERR_INVALID_ARG;
+  if (window > 0 && !causal) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || scale <= 0.f) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  // Index arithmetic limits: rows per tensor and grid size stay in int range.
+  if ((int64_t)B * Hq > (1 << 24) || (int64_t)B * Hkv > (1 << 24)) return ATTN_ERR_UNSUPPORTED;
+  if (Lq > (1 << 28) || Lk > (1 << 28)) return ATTN_ERR_UNSUPPORTED;
+  if ((int64_t)B * Hq * ((Lq + 127) / 128) >= (int64_t)1 << 31) return ATTN_ERR_UNSUPPORTED;
+  return ATTN_OK;
+}
+
+// 3-D map over a [BH, L, d] bf16 tensor, box 64 x 128 x 1, 128-byte swizzle.
+// Rows past L inside a box read as zero.
+int make_map(EncodeTiledFn enc, CUtensorMap* m, const void* ptr, int BH, int L, int d) {
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)(L > 0 ? L : 1), (cuuint64_t)(BH > 0 ? BH : 1)};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)d * 2 * (cuuint64_t)(L > 0 ? L : 1)};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+__global__ void selftest_wait_kernel(int* err, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  const WaitGuard g{err, &abort_flag, limit_ns, 0};
+  // Nothing ever arrives on `bar`: the wait must give up by itself.
+  mbar_wait(&bar, 0, g, 1000);
+  __syncthreads();
+}
+
+}  // namespace
+}  // namespace tea
+
+using namespace tea;
+
+extern "C" {
+
+const char* attn_status_string(int status) {
+  switch (status) {
+    case ATTN_OK: return "ATTN_OK";
+    case ATTN_ERR_INVALID_ARG: return "ATTN_ERR_INVALID_ARG";
+    case ATTN_ERR_UNSUPPORTED: return "ATTN_ERR_UNSUPPORTED";
+    case ATTN_ERR_CUDA: return "ATTN_ERR_CUDA";
+    case ATTN_ERR_TIMEOUT: return "ATTN_ERR_TIMEOUT";
+    default: return "ATTN_ERR_UNKNOWN";
+  }
+}
+
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Lq,
+             int Lk, int d, float scale, int causal, int window, void* stream) {
+  int st = check_shape(B, Hq, Hkv, Lq, Lk, d, scale, causal, window);
+  if (st != ATTN_OK) return st;
+  if (B == 0 || Hq == 0 || Lq == 0) return ATTN_OK;
+  if (!q || !o || !lse || !aligned16(q) || !aligned16(o) || !aligned16(lse)) return ATTN_ERR_INVALID_ARG;
+  if (Lk > 0 && (!k || !v || !aligned16(k) || !aligned16(v))) return ATTN_ERR_INVALID_ARG;
+  EncodeTiledFn enc;
+  if ((st = get_encoder(&enc)) != ATTN_OK) return st;
+  FwdParams P;
+  memset(&P, 0, sizeof(P));
+  P.prob = Problem{B, Hq, Hkv, Lq, Lk, d, causal, window, scale};
+  // With Lk == 0 nothing reads K/V; map Q's memory so the descriptors stay valid.
+  const void* kp = Lk > 0 ? k : q;
+  const void* vp = Lk > 0 ? v : q;
+  if ((st = make_map(enc, &P.tm_q, q, B * Hq, Lq, d)) != ATTN_OK) return st;
+  if ((st = make_map(enc, &P.tm_k, kp, Lk > 0 ? B * Hkv : B * Hq, Lk > 0 ? Lk : Lq, d)) != ATTN_OK) return st;
+  if ((st = make_map(enc, &P.tm_v, vp, Lk > 0 ? B * Hkv : B * Hq, Lk > 0 ? Lk : Lq, d)) != ATTN_OK) return st;
+  P.o = o;
+  P.lse = lse;
+  P.scale_log2 = scale * 1.4426950408889634f;
+  fwd_plan(P.prob, &P.n_units, &P.pair_heads);
+  if ((st = get_err_word(&P.err)) != ATTN_OK) return st;
+  P.limit_ns = kWaitLimitNs;
+  return launch_fwd(P, static_cast<cudaStream_t>(stream)) == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int Lq, int Lk, int d) {
+  if (check_shape(B, Hq, Hkv, Lq, Lk, d, 1.f, 0, 0) != ATTN_OK) return 0;
+  if (B == 0 || Hq == 0 || Lq == 0) return 0;
+  const size_t rows = (size_t)B * Hq * Lq;
+  const size_t dsz = (rows * 4 + 255) / 256 * 256;   // D, fp32
+  const size_t dq = (rows * d * 4 + 255) / 256 * 256; // dQ accumulator, fp32
+  return dsz + dq;
+}
+
+int attn_get_device_error(void* stream, int* site) {
+  int* addr = nullptr;
+  int st = get_err_word(&addr);
+  if (st != ATTN_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return ATTN_ERR_CUDA;
+  int word = 0;
+  if (cudaMemcpyFromSymbol(&word, g_dev_err, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_dev_err, &zero, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (site) *site = word >> 8;
+  return (word & 0xFF) == DEV_TIMEOUT ? ATTN_ERR_TIMEOUT : ATTN_OK;
+}
+
+int attn_selftest_wait_timeout(int64_t limit_ns, void* stream) {
+  if (limit_ns <= 0 || limit_ns > (int64_t)10000000000ll) return ATTN_ERR_INVALID_ARG;
+  int* err = nullptr;
+  int st = get_err_word(&err);
+  if (st != ATTN_OK) return st;
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(err, (uint64_t)limit_ns);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,446 @@
+// attn_fwd.cu - forward attention kernel for sm_100a.
+//
+// Algorithm ("缩放定律与高效注意力" §3.2; "高效注意力：FlashAttention 与线性注意力",
+// 原理与机制): for a tile of 128 query rows, stream the visible key/value tiles
+// of 128 keys, compute S = Q K^T on the tensor cores into tensor memory, keep
+// a running row max m and row sum l, turn S into P = exp(scale*S - m) and
+// accumulate O += P V, rescaling O and l by e^{m_old - m_new} when m grows.
+// Only O (divided by l) and LSE = m + log l leave the chip.
+//
+// B200 mapping (one CTA per SM, 384 threads, 12 warps):
+//   warp 0      TMA producer: two Q tiles, then a ring of K/V tiles
+//   warp 1      tcgen05 issuer (one elected thread) and TMEM owner
+//   warps 4-7   softmax for query slot 0 (thread = query row)
+//   warps 8-11  softmax for query slot 1
+// A CTA holds two query tiles ("slots") that share every K/V tile it loads:
+// two heads of one GQA group at the same rows when the group size is even
+// (K/V reuse across the group), otherwise two consecutive row tiles of one
+// head.  Tensor memory (512 columns): S0 | S1 | O0 | O1, 128 columns each; the
+// bf16 P of a slot overwrites the first 64 columns of its S after S has been
+// read, and feeds the P.V MMA straight from tensor memory.  While one slot's
+// softmax runs, the tensor cores work on the other slot's P.V and next
+// Q.K^T, so the exponentials of one slot overlap the MMAs of the other.
+//
+// Rescaling is lazy: a row's reference max is only raised when the new max
+// exceeds it by more than 8 (in log2 units).  Any reference value gives the
+// same O/l; keeping p <= 2^8 bounds the bf16 P and fp32 accumulators.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+#include <cmath>
+
+#include "sm100.cuh"
+#include "attn_common.cuh"
+#include "attn_kernels.h"
+
+namespace tea {
+
+namespace fwd {
+
+constexpr int BM = 128;        // query rows per slot
+constexpr int BN = 128;        // keys per K/V tile
+constexpr int THREADS = 384;
+constexpr int PANEL = 16384;   // one 128-row x 128-byte swizzled panel
+constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
+
+template <int D>
+struct Cfg {
+  static constexpr int PANELS = D / 64;
+  static constexpr int TILE = BM * D * 2;         // bytes of one Q, K or V tile
+  static constexpr int NST = D == 128 ? 4 : 8;    // K/V ring stages
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_KV = 2 * TILE;
+  static constexpr int OFF_BAR = OFF_KV + NST * TILE;
+  static constexpr int SMEM = OFF_BAR + 512 + 1024;  // barriers + alignment slack
+};
+
+struct Bars {
+  uint64_t q_full[2];
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t o_full[2];
+  uint64_t drain;
+  uint64_t kv_full[8];
+  uint64_t kv_empty[8];
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+// TMEM columns of slot s: S (and P) at s_col(s), O at o_col(s).
+__device__ __forceinline__ uint32_t s_col(int s) { return 128u * s; }
+__device__ __forceinline__ uint32_t o_col(int s) { return 256u + 128u * s; }
+
+// One CTA's work: two query tiles (slots).
+struct Unit {
+  int b, kvh;
+  int head[2];
+  int q0[2];
+  int lo[2], hi[2];  // key tile range per slot (empty: lo == hi)
+  int ulo, uhi;      // union of the two ranges
+};
+
+__device__ __forceinline__ Unit decode_unit(const FwdParams& P, int idx) {
+  const Problem& p = P.prob;
+  Unit u;
+  const int G = p.Hq / p.Hkv;
+  const int nqt = cdiv(p.Lq, BM);
+  if (P.pair_heads) {
+    // Two heads of one GQA group, same query rows.  Heavy (late) rows first.
+    const int per_q = p.B * (p.Hq / 2);
+    const int qi = nqt - 1 - idx / per_q;
+    const int rem = idx % per_q;
+    u.b = rem / (p.Hq / 2);
+    const int hp = rem % (p.Hq / 2);
+    u.head[0] = 2 * hp;
+    u.head[1] = 2 * hp + 1;
+    u.q0[0] = u.q0[1] = qi * BM;
+  } else {
+    const int nqp = cdiv(nqt, 2);
+    const int per_q = p.B * p.Hq;
+    const int qp = nqp - 1 - idx / per_q;
+    const int rem = idx % per_q;
+    u.b = rem / p.Hq;
+    u.head[0] = u.head[1] = rem % p.Hq;
+    u.q0[0] = qp * 2 * BM;
+    u.q0[1] = qp * 2 * BM + BM;
+  }
+  u.kvh = u.head[0] / G;
+  u.ulo = 1 << 30;
+  u.uhi = 0;
+  for (int s = 0; s < 2; s++) {
+    kv_tile_range(p, u.q0[s], u.q0[s] + BM, BN, u.lo[s], u.hi[s]);
+    if (u.lo[s] < u.hi[s]) {
+      u.ulo = imin(u.ulo, u.lo[s]);
+      u.uhi = imax(u.uhi, u.hi[s]);
+    }
+  }
+  if (u.uhi == 0) u.ulo = 0;
+  return u;
+}
+
+__device__ __forceinline__ bool active(const Unit& u, int s, int j) { return j >= u.lo[s] && j < u.hi[s]; }
+
+// ------------------------------------------------------------------ producer
+template <int D>
+__device__ void producer(const FwdParams& P, const Unit& u, uint8_t* smem, Bars& bars, const WaitGuard& g) {
+  using C = Cfg<D>;
+  const Problem& p = P.prob;
+  tma_prefetch_desc(&P.tm_q);
+  tma_prefetch_desc(&P.tm_k);
+  tma_prefetch_desc(&P.tm_v);
+#pragma unroll
+  for (int s = 0; s < 2; s++) {
+    if (u.lo[s] >= u.hi[s]) continue;
+    mbar_arrive_expect_tx(&bars.q_full[s], C::TILE);
+    for (int pnl = 0; pnl < C::PANELS; pnl++)
+      tma_load_3d(smem + C::OFF_Q + s * C::TILE + pnl * PANEL, &P.tm_q, &bars.q_full[s], pnl * 64, u.q0[s],
+                  u.b * p.Hq + u.head[s]);
+  }
+  int issued = 0;
+  for (int j = u.ulo; j < u.uhi; j++) {
+    for (int which = 0; which < 2; which++) {
+      const int r = 2 * (j - u.ulo) + which;
+      const int st = r % C::NST;
+      const uint32_t ph = (r / C::NST) & 1;
+      if (!mbar_wait(&bars.kv_empty[st], ph ^ 1, g, 1)) goto drain;
+      mbar_arrive_expect_tx(&bars.kv_full[st], C::TILE);
+      for (int pnl = 0; pnl < C::PANELS; pnl++)
+        tma_load_3d(smem + C::OFF_KV + st * C::TILE + pnl * PANEL, which ? &P.tm_v : &P.tm_k, &bars.kv_full[st],
+                    pnl * 64, j * BN, u.b * p.Hkv + u.kvh);
+      issued = r + 1;
+    }
+  }
+  return;
+drain:
+  // A wait was abandoned: let every copy this warp started land before the
+  // CTA exits (bounded, independent of the other roles).
+  {
+    WaitGuard g2 = g;
+    for (int r = imax(0, issued - C::NST); r < issued; r++) mbar_wait_ignore_abort(&bars.kv_full[r % C::NST], (r / C::NST) & 1, g2);
+#pragma unroll
+    for (int s = 0; s < 2; s++)
+      if (u.lo[s] < u.hi[s]) mbar_wait_ignore_abort(&bars.q_full[s], 0, g2);
+  }
+}
+
+// ------------------------------------------------------------------ MMA issuer
+template <int D>
+__device__ void mma_issuer(const FwdParams& P, const Unit& u, uint8_t* smem, Bars& bars, uint32_t tmem,
+                           const WaitGuard& g) {
+  using C = Cfg<D>;
+  const uint32_t idesc_qk = idesc_bf16_f32(BM, BN, 0, 0);
+  const uint32_t idesc_pv = idesc_bf16_f32(BM, D, 0, 1);
+  const uint32_t q_addr = smem_u32(smem + C::OFF_Q);
+  const uint32_t kv_addr = smem_u32(smem + C::OFF_KV);
+  if (u.uhi <= u.ulo) return;
+
+  auto stage_of = [&](int j, int which) { return (2 * (j - u.ulo) + which) % C::NST; };
+  auto phase_of = [&](int j, int which) { return (uint32_t)(((2 * (j - u.ulo) + which) / C::NST) & 1); };
+
+  auto issue_s = [&](int s, int j) {
+    const uint32_t qa = q_addr + s * C::TILE;
+    const uint32_t ka = kv_addr + stage_of(j, 0) * C::TILE;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; kk++) {
+      const uint32_t off = (kk / 4) * PANEL + (kk % 4) * 32;
+      mma_ss(tmem + s_col(s), sw128_desc(qa + off, 16, 1024), sw128_desc(ka + off, 16, 1024), idesc_qk, kk > 0);
+    }
+    mma_commit(&bars.s_full[s]);
+  };
+
+#pragma unroll
+  for (int s = 0; s < 2; s++)
+    if (u.lo[s] < u.hi[s] && !mbar_wait(&bars.q_full[s], 0, g, 10)) goto out;
+
+  // Prologue: S for the first tile.
+  if (!mbar_wait(&bars.kv_full[stage_of(u.ulo, 0)], phase_of(u.ulo, 0), g, 11)) goto out;
+  tc_fence_after();
+#pragma unroll
+  for (int s = 0; s < 2; s++)
+    if (active(u, s, u.ulo)) issue_s(s, u.ulo);
+  mma_commit(&bars.kv_empty[stage_of(u.ulo, 0)]);
+
+  for (int j = u.ulo; j < u.uhi; j++) {
+    if (!mbar_wait(&bars.kv_full[stage_of(j, 1)], phase_of(j, 1), g, 12)) goto out;
+    const bool next = j + 1 < u.uhi;
+    if (next) {
+      if (!mbar_wait(&bars.kv_full[stage_of(j + 1, 0)], phase_of(j + 1, 0), g, 13)) goto out;
+    }
+    const uint32_t va = kv_addr + stage_of(j, 1) * C::TILE;
+#pragma unroll
+    for (int s = 0; s < 2; s++) {
+      if (active(u, s, j)) {
+        if (!mbar_wait(&bars.p_full[s], (j - u.lo[s]) & 1, g, 14 + s)) goto out;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; kk++)
+          mma_ts(tmem + o_col(s), tmem + s_col(s) + kk * 8, sw128_desc(va + kk * 2048, PANEL, 1024), idesc_pv,
+                 (j > u.lo[s]) || kk > 0);
+        if (j == u.hi[s] - 1) mma_commit(&bars.o_full[s]);
+      }
+      if (next && active(u, s, j + 1)) issue_s(s, j + 1);
+    }
+    mma_commit(&bars.kv_empty[stage_of(j, 1)]);
+    if (next) mma_commit(&bars.kv_empty[stage_of(j + 1, 0)]);
+  }
+out:
+  // Drain: wait until every MMA this thread issued has completed.
+  mma_commit(&bars.drain);
+  mbar_wait_ignore_abort(&bars.drain, 0, g);
+}
+
+// ------------------------------------------------------------------ softmax
+// One warpgroup per slot; thread `row` owns query row q0 + row and TMEM lane
+// `row` (warp w of the group may only touch lanes 32*(w%4) .. +31).
+template <int D>
+__device__ void softmax_slot(const FwdParams& P, const Unit& u, int s, Bars& bars, uint32_t tmem,
+                             const WaitGuard& g) {
+  const Problem& p = P.prob;
+  const int wl = (threadIdx.x / 32) % 4;
+  const int lane = threadIdx.x % 32;
+  const int row = wl * 32 + lane;
+  // Slot fields as scalars (a runtime index into Unit would put it in local memory).
+  const int lo_s = s ? u.lo[1] : u.lo[0];
+  const int hi_s = s ? u.hi[1] : u.hi[0];
+  const int head_s = s ? u.head[1] : u.head[0];
+  const int q_row = (s ? u.q0[1] : u.q0[0]) + row;
+  int key_lo, key_hi;
+  row_key_range(p, q_row, key_lo, key_hi);
+  const float c = P.scale_log2;
+  const uint32_t lane_base = (uint32_t)(wl * 32) << 16;
+  const uint32_t t_s = tmem + lane_base + s_col(s);
+  const uint32_t t_o = tmem + lane_base + o_col(s);
+  float m = -INFINITY;  // reference max, log2 units (scaled)
+  float l = 0.f;        // running sum of exp2(c*S - m)
+
+  for (int j = lo_s; j < hi_s; j++) {
+    const int it = j - lo_s;
+    if (!mbar_wait(&bars.s_full[s], it & 1, g, 20 + s)) return;
+    tc_fence_after();
+    uint32_t x[BN];
+#pragma unroll
+    for (int q = 0; q < BN / 32; q++) tmem_ld32p(t_s + 32 * q, x + 32 * q);
+    tmem_wait_ld();
+
+    // Element-wise mask only on tiles that straddle this row's visible range.
+    const int key0 = j * BN;
+    if (key0 < key_lo || key0 + BN > key_hi) {
+#pragma unroll
+      for (int cc = 0; cc < BN; cc++) {
+        const int key = key0 + cc;
+        if (key < key_lo || key >= key_hi) x[cc] = __float_as_uint(-INFINITY);
+      }
+    }
+    float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+    for (int cc = 0; cc < BN; cc += 4) {
+      mx0 = fmaxf(mx0, __uint_as_float(x[cc]));
+      mx1 = fmaxf(mx1, __uint_as_float(x[cc + 1]));
+      mx2 = fmaxf(mx2, __uint_as_float(x[cc + 2]));
+      mx3 = fmaxf(mx3, __uint_as_float(x[cc + 3]));
+    }
+    const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+    const float m_cand = mx == -INFINITY ? -INFINITY : mx * c;
+    const float m_new = fmaxf(m, m_cand);
+    const bool need = m_new > m + RESCALE_THRESHOLD;
+    const float alpha = need ? ex2_approx(m - m_new) : 1.f;
+    if (need) {
+      l *= alpha;
+      m = m_new;
+    }
+    const float m_sub = m == -INFINITY ? 0.f : m;
+    float s0 = 0.f, s1 = 0.f;
+    // P packed two per 32-bit word, written over x[0 .. BN/2) as it goes
+    // (x[2cc], x[2cc+1] are dead once read).
+#pragma unroll
+    for (int cc = 0; cc < BN / 2; cc++) {
+      const float p0 = ex2_approx(fmaf(__uint_as_float(x[2 * cc]), c, -m_sub));
+      const float p1 = ex2_approx(fmaf(__uint_as_float(x[2 * cc + 1]), c, -m_sub));
+      s0 += p0;
+      s1 += p1;
+      x[cc] = pack_bf16x2(p0, p1);
+    }
+    l += s0 + s1;
+    // P (bf16, two per column) replaces the first BN/2 columns of S.
+    tmem_st32(t_s, x);
+    tmem_st32(t_s + 32, x + 32);
+    tmem_wait_st();
+    if (__any_sync(0xffffffffu, need) && it > 0) {
+      // O holds the sum over earlier tiles (the last P.V finished before this
+      // S was produced) and the next P.V waits for p_full: bring O to the new
+      // reference max now, after P is out of the registers.
+#pragma unroll
+      for (int q = 0; q < D / 32; q++) {
+        uint32_t o[32];
+        tmem_ld32p(t_o + 32 * q, o);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; e++) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+        tmem_st32(t_o + 32 * q, o);
+      }
+      tmem_wait_st();
+    }
+
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bars.p_full[s]);
+  }
+
+  // Epilogue: O / l in bf16 and the natural-log LSE.
+  const bool has = lo_s < hi_s;
+  if (has) {
+    if (!mbar_wait(&bars.o_full[s], 0, g, 22 + s)) return;
+    tc_fence_after();
+  }
+  const bool write = q_row < p.Lq;
+  const float inv_l = l > 0.f ? 1.f / l : 0.f;
+  const size_t row_off = ((size_t)(u.b * p.Hq + head_s) * p.Lq + q_row);
+  uint4* out = reinterpret_cast<uint4*>(static_cast<uint16_t*>(P.o) + row_off * D);
+#pragma unroll
+  for (int q = 0; q < D / 32; q++) {
+    uint32_t o[32];
+    if (has) {
+      tmem_ld32p(t_o + 32 * q, o);
+      tmem_wait_ld();
+    } else {
+#pragma unroll
+      for (int e = 0; e < 32; e++) o[e] = 0u;
+    }
+    uint32_t w[16];
+#pragma unroll
+    for (int e = 0; e < 16; e++)
+      w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
+    if (write) {
+#pragma unroll
+      for (int v = 0; v < 4; v++) out[q * 4 + v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+    }
+  }
+  if (write) P.lse[row_off] = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
+}
+
+// ------------------------------------------------------------------ kernel
+template <int D>
+__global__ void __launch_bounds__(THREADS, 1) attn_fwd_kernel(const __grid_constant__ FwdParams P) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  Bars& bars = *reinterpret_cast<Bars*>(smem + C::OFF_BAR);
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const Unit u = decode_unit(P, blockIdx.x);
+  const WaitGuard g{P.err, &bars.abort_flag, P.limit_ns, 0};
+
+  if (threadIdx.x == 0) {
+    bars.abort_flag = 0;
+    for (int s = 0; s < 2; s++) {
+      mbar_init(&bars.q_full[s], 1);
+      mbar_init(&bars.s_full[s], 1);
+      mbar_init(&bars.p_full[s], 4);
+      mbar_init(&bars.o_full[s], 1);
+    }
+    mbar_init(&bars.drain, 1);
+    for (int st = 0; st < C::NST; st++) {
+      mbar_init(&bars.kv_full[st], 1);
+      mbar_init(&bars.kv_empty[st], 1);
+    }
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars.tmem_base;
+
+  // Registers: launched at 168 per thread (384 x 168); the load/MMA group
+  // gives up to 80, each softmax group takes 208 (128*80 + 256*208 <= 384*168).
+  if (warp < 4) {
+    regs_dec<80>();
+    if (warp == 0) {
+      if (lane == 0) producer<D>(P, u, smem, bars, g);
+    } else if (warp == 1) {
+      if (lane == 0) mma_issuer<D>(P, u, smem, bars, tmem, g);
+    }
+  } else {
+    regs_inc<208>();
+    softmax_slot<D>(P, u, (warp - 4) / 4, bars, tmem, g);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace fwd
+
+void fwd_plan(const Problem& p, int* n_units, int* pair_heads) {
+  const int G = p.Hq / p.Hkv;
+  const int nqt = cdiv(p.Lq, fwd::BM);
+  if (G % 2 == 0) {
+    *pair_heads = 1;
+    *n_units = p.B * (p.Hq / 2) * nqt;
+  } else {
+    *pair_heads = 0;
+    *n_units = p.B * p.Hq * cdiv(nqt, 2);
+  }
+}
+
+template <int D>
+static cudaError_t launch_fwd_d(const FwdParams& P, cudaStream_t stream) {
+  constexpr int smem = fwd::Cfg<D>::SMEM;
+  cudaError_t e = cudaFuncSetAttribute(fwd::attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  fwd::attn_fwd_kernel<D><<<P.n_units, fwd::THREADS, smem, stream>>>(P);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fwd(const FwdParams& P, cudaStream_t stream) {
+  if (P.n_units <= 0) return cudaSuccess;
+  return P.prob.d == 128 ? launch_fwd_d<128>(P, stream) : launch_fwd_d<64>(P, stream);
+}
+
+}  // namespace tea
