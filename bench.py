@@ -1,0 +1,355 @@
+"""Benchmark: exact causal attention forward + backward on B200.
+
+One step = the whole hot path on one batch: attn_fwd (O, LSE) then the
+recompute backward (attn_bwd_preprocess, attn_bwd_main, attn_bwd_finalize),
+on the fwd+bwd workload B=2, Hq=Hkv=32, L=4096, d=128, causal, synthetic
+bf16 N(0,1) inputs.  Metric: algorithmic mask-adjusted TFLOP/s over fwd+bwd
+(forward 4*d*visible_pairs*B*Hq; backward 2.5x that).
+
+Multi-GPU (torchrun): the (batch, head) units are independent, so every rank
+runs its own batch of the same workload with no collective on the data path
+(weak scaling); the step time is the max over ranks.
+
+`--impl reference` times the float64 CPU oracle (a slow, plain restatement of
+the definition) on a bounded sample of the same workload instead.
+"""
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synth import WORKLOADS, make_inputs  # noqa: E402
+
+WORKLOAD = "mha_causal_fwdbwd"
+METRIC = "attention TFLOP/s (bf16, mask-adjusted) fwd+bwd and % of B200 dense BF16 peak"
+DOMINANT = "attn_bwd_main"
+PROFILE = os.path.join(ROOT, "profiles", "attn_bwd_main_mha_causal_4096.md")
+KERNEL_SRC = os.path.join(ROOT, "tiled_exact_attention_02_b200", "csrc", "attn_bwd.cu")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        p = json.load(open(path))
+        return p["bf16_tflops"], p.get("bf16_tflops_sustained", p["bf16_tflops"]), p["hbm_gbs"], "measured"
+    except Exception:
+        return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+def profile_traffic():
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary, if it was taken on the current kernel source (else None)."""
+    try:
+        text = open(PROFILE).read()
+        sha = hashlib.sha256(open(KERNEL_SRC, "rb").read()).hexdigest()[:16]
+        m_sha = re.search(r"source_sha256_16:\s*([0-9a-f]+)", text)
+        m_b = re.search(r"dram_bytes_per_launch_full:\s*([0-9.eE+]+)", text)
+        if m_sha and m_b and m_sha.group(1) == sha:
+            return float(m_b.group(1))
+    except OSError:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling during the timed region."""
+
+    def __init__(self, index):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--id={index}", f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                                       "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return None
+        self.p.terminate()
+        self.p.wait()
+        self.f.flush()
+        rows = [r.split(",") for r in open(self.f.name).read().strip().splitlines() if r.strip()]
+        os.unlink(self.f.name)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if len(r) > 8]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for n, v in zip(names, r[5:9]):
+                if v.strip() == "Active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": float(rows[0][2]) if len(rows[0]) > 2 else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def dist_setup(n_gpus):
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+ROWS_PER_UNIT = 512  # CPU sample unit: 512 query rows of one head, fwd + their bwd contributions
+
+
+def cpu_units(w):
+    return [(b, h, r0) for b in range(w.B) for h in range(w.Hq) for r0 in range(0, w.Lq, ROWS_PER_UNIT)]
+
+
+def unit_flops(w, r0):
+    """Algorithmic fwd+bwd FLOPs of query rows [r0, r0 + ROWS_PER_UNIT) of one head."""
+    pairs = 0
+    for i in range(r0, min(w.Lq, r0 + ROWS_PER_UNIT)):
+        hi = min(i + 1, w.Lk) if w.causal else w.Lk
+        lo = max(0, i - w.window + 1) if w.window > 0 else 0
+        pairs += max(0, hi - lo)
+    return 3.5 * 4.0 * w.d * pairs
+
+
+def oracle_sample(w, x, units):
+    """Time the float64 oracle on sample units; returns (seconds, algorithmic flops)."""
+    import oracle
+    t0 = time.perf_counter()
+    flops = 0.0
+    for b, h, r0 in units:
+        oracle.attn_row_block(x["q"], x["k"], x["v"], x["do"], w.scale, w.causal, w.window, b, h, r0,
+                              min(w.Lq, r0 + ROWS_PER_UNIT))
+        flops += unit_flops(w, r0)
+    return time.perf_counter() - t0, flops
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = WORKLOADS[WORKLOAD]
+    x = make_inputs(w)
+    units = cpu_units(w)
+    stride = 97  # walk the units in a fixed scattered order (mixes light and heavy causal rows)
+    for i in range(args.warmup):
+        oracle_sample(w, x, [units[(i * stride) % len(units)]])
+    secs, flops = 0.0, 0.0
+    for i in range(args.steps):
+        s, f = oracle_sample(w, x, [units[((args.warmup + i) * stride) % len(units)]])
+        secs += s
+        flops += f
+    value = flops / secs / 1e12
+    cores = host_cores()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.Lq, "d": w.d,
+                   "causal": w.causal, "window": w.window,
+                   "step_sample": f"{ROWS_PER_UNIT} query rows of one head, fwd + their bwd contributions"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{args.steps} units of {ROWS_PER_UNIT} query rows x 1 head of {WORKLOAD}, "
+                                   f"float64 numpy fwd+bwd, {secs:.1f} s"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    import tiled_exact_attention_02_b200 as ta
+
+    rank, world, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = WORKLOADS[WORKLOAD]
+    x = make_inputs(w, seed=w.seed + rank)
+
+    def dev_bf16(bits):
+        import numpy as np
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
+
+    q, k, v, do = (dev_bf16(x[n]) for n in ("q", "k", "v", "do"))
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.Lq), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(ta.bwd_workspace_size(w.B, w.Hq, w.Hkv, w.Lq, w.Lk, w.d), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    N_EV = 5  # fwd | pre | main | post boundaries
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(N_EV)] for _ in range(args.steps)]
+
+    def step(evs=None):
+        if evs:
+            evs[0].record(stream)
+        ta.fwd(q, k, v, o, lse, w.causal, w.window, w.scale, stream)
+        ta.bwd_phases(q, k, v, o, lse, do, dq, dk, dv, ws, w.causal, w.window, w.scale, stream,
+                      between=(lambda i: evs[i + 1].record(stream)) if evs else None)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    st, site = ta.device_error()
+    if st != 0:
+        raise SystemExit(f"device error {st} at site {site}")
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(events[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    st, site = ta.device_error()
+    if st != 0:
+        raise SystemExit(f"device error {st} at site {site}")
+    ms_total = max_over_ranks(t_start.elapsed_time(t_end), world)
+    ms_step = ms_total / args.steps
+    flops_step = w.fwd_flops() + w.bwd_flops()
+    value = world * flops_step / (ms_step * 1e-3) / 1e12
+
+    names = ["attn_fwd", "attn_bwd_preprocess", "attn_bwd_main", "attn_bwd_finalize"]
+    per = {n: statistics.mean(e[j].elapsed_time(e[j + 1]) for e in events) for j, n in enumerate(names)}
+    burst, sustained, hbm, peak_src = peaks()
+    main_ms = per[DOMINANT]
+    achieved = w.bwd_flops() / (main_ms * 1e-3) / 1e12
+    fwd_tf = w.fwd_flops() / (per["attn_fwd"] * 1e-3) / 1e12
+
+    # End to end through the public API with host buffers: pinned host inputs
+    # copied in, the step run, and every output (O, LSE, dQ, dK, dV) copied out.
+    e2e = None
+    if args.e2e_steps > 0:
+        hin = [t.cpu().pin_memory() for t in (q, k, v, do)]
+        outs = (o, lse, dq, dk, dv)
+        hout = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
+        h2d = sum(t.numel() * t.element_size() for t in hin)
+        d2h = sum(t.numel() * t.element_size() for t in hout)
+        dins = (q, k, v, do)
+
+        def e2e_step():
+            for dst, src in zip(dins, hin):
+                dst.copy_(src, non_blocking=True)
+            step()
+            for dst, src in zip(hout, outs):
+                dst.copy_(src, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ms_e2e = max_over_ranks(a.elapsed_time(b), world) / args.e2e_steps
+        e2e = {"value": world * flops_step / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e}
+
+    if rank != 0:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        xs = make_inputs(w)
+        secs, fl, n = 0.0, 0.0, 0
+        units = cpu_units(w)
+        while secs < 12.0 and n < len(units):
+            s, f = oracle_sample(w, xs, [units[(n * 97) % len(units)]])
+            secs += s
+            fl += f
+            n += 1
+        cpu = {"value": fl / secs / 1e12, "unit": "TFLOP/s", "cores": host_cores(), "kind": "oracle",
+               "sample": f"{n} of {len(units)} units ({ROWS_PER_UNIT} query rows x 1 head) of {WORKLOAD}, "
+                         f"float64 numpy fwd+bwd, {secs:.1f} s"}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.Lq, "d": w.d,
+                   "causal": w.causal, "window": w.window, "global_batch": w.B * world,
+                   "flops_per_step_per_gpu": flops_step, "parallelism": f"independent batches x{world}",
+                   "l2": "inputs larger than L2 (Q,K,V,O,dO,dQ,dK,dV = 512 MB per GPU); no flush"},
+        "frac_of_peak": {"spec_2250": value / world / 2250.0, f"{peak_src}_sustained": value / world / sustained},
+        "kernels_ms": per,
+        "fwd_tflops": fwd_tf,
+        "roofline": {"kernel": DOMINANT, "bound": "tensor", "achieved": achieved, "peak": sustained,
+                     "peak_kind": f"{peak_src} bf16 sustained", "unit": "TFLOP/s", "frac": achieved / sustained,
+                     "traffic": profile_traffic()},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": 4 * args.steps,
+        "clocks": clk,
+    }
+    print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

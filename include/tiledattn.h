@@ -106,8 +106,31 @@ ATTN_API int attn_bwd(const void* q, const void* k, const void* v, const void* o
              void* dk, void* dv, int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale, int causal, int window,
              void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * The three phases attn_bwd runs, for callers that schedule or time them
+ * separately (same arguments and rules as attn_bwd; call them in this order
+ * on one stream with the same workspace):
+ *   attn_bwd_preprocess  D_i = dO_i . O_i into the workspace, zero the dQ accumulator
+ *   attn_bwd_main        recompute P tile by tile; write dK, dV; accumulate dQ
+ *   attn_bwd_finalize    dQ = scale * accumulator, rounded to bf16
+ */
+ATTN_API int attn_bwd_preprocess(const void* o, const void* dO, int B, int Hq, int Lq, int d, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+ATTN_API int attn_bwd_main(const void* q, const void* k, const void* v, const float* lse, const void* dO, void* dk,
+                           void* dv, int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale, int causal, int window,
+                           void* workspace, size_t workspace_bytes, void* stream);
+ATTN_API int attn_bwd_finalize(void* dq, int B, int Hq, int Lq, int d, float scale, void* workspace,
+                               size_t workspace_bytes, void* stream);
+
 /* Static, human-readable name of a status code. */
 ATTN_API const char* attn_status_string(int status);
+
+/*
+ * Text of the last CUDA error that made a call on this thread return
+ * ATTN_ERR_CUDA, prefixed with the failing step ("" if none).  The pointer
+ * stays valid until the next call on this thread.
+ */
+ATTN_API const char* attn_last_cuda_error(void);
 
 /*
  * Synchronises `stream`, then reads and clears the current device's error

@@ -12,4 +12,5 @@ from .attention import (  # noqa: F401
     attn_fwd,
     attn_fwd_rows,
     attn_bwd,
+    attn_row_block,
 )

@@ -164,6 +164,24 @@ def attn_fwd_rows(q, k, v, scale, causal, window, b, h, rows):
     return O, lse
 
 
+def _rows_bwd(qh, kh, vh, doh, scale, causal, window, r0, r1):
+    """Rows [r0, r1) of one head: their O and LSE, their dQ rows, and their
+    contributions to dK and dV over the visible key band [lo, hi)."""
+    Lk = kh.shape[0]
+    lo, hi = visible_band(r0, r1, Lk, causal, window)
+    vis = _band_mask(np.arange(r0, r1), lo, hi, causal, window)
+    A, lse = attention_weights(qh[r0:r1], kh[lo:hi], scale, vis)
+    O = A @ vh[lo:hi]
+    dO = doh[r0:r1]
+    dv = A.T @ dO                                # dV = A^T dO
+    dP = dO @ vh[lo:hi].T                        # dP = dO V^T
+    D = np.sum(dO * O, axis=1, keepdims=True)    # D_i = dO_i . O_i = sum_j A_ij dP_ij
+    dS = A * (dP - D)                            # softmax Jacobian applied row by row
+    dq = scale * (dS @ kh[lo:hi])                # S = scale Q K^T
+    dk = scale * (dS.T @ qh[r0:r1])
+    return lo, hi, O, lse, dq, dk, dv
+
+
 def _head_bwd(qh, kh, vh, doh, scale, causal, window):
     """dQ, dK, dV for one (query head, kv head) pair; textbook softmax gradient."""
     Lq, Lk = qh.shape[0], kh.shape[0]
@@ -173,18 +191,24 @@ def _head_bwd(qh, kh, vh, doh, scale, causal, window):
     step = max(1, _ROW_BLOCK_ELEMS // max(1, Lk))
     for r0 in range(0, Lq, step):
         r1 = min(Lq, r0 + step)
-        lo, hi = visible_band(r0, r1, Lk, causal, window)
-        vis = _band_mask(np.arange(r0, r1), lo, hi, causal, window)
-        A, _ = attention_weights(qh[r0:r1], kh[lo:hi], scale, vis)
-        O = A @ vh[lo:hi]
-        dO = doh[r0:r1]
-        dv[lo:hi] += A.T @ dO                       # dV = A^T dO
-        dP = dO @ vh[lo:hi].T                        # dP = dO V^T
-        D = np.sum(dO * O, axis=1, keepdims=True)    # D_i = dO_i . O_i = sum_j A_ij dP_ij
-        dS = A * (dP - D)                            # softmax Jacobian applied row by row
-        dq[r0:r1] = scale * (dS @ kh[lo:hi])         # S = scale Q K^T
-        dk[lo:hi] += scale * (dS.T @ qh[r0:r1])
+        lo, hi, _, _, dqb, dkb, dvb = _rows_bwd(qh, kh, vh, doh, scale, causal, window, r0, r1)
+        dq[r0:r1] = dqb
+        dk[lo:hi] += dkb
+        dv[lo:hi] += dvb
     return dq, dk, dv
+
+
+def attn_row_block(q, k, v, do, scale, causal, window, b, h, r0, r1):
+    """Query rows [r0, r1) of head (b, h): O and LSE of those rows, their dQ
+    rows, and their (partial) contributions to dK and dV of K/V head
+    h // (Hq/Hkv), returned as (O, lse, dq, lo, hi, dk_part, dv_part) with
+    dk_part/dv_part covering keys [lo, hi).  Summing the parts over all row
+    blocks of all heads of a group gives attn_bwd's dK and dV."""
+    Hq, Hkv = q.shape[1], k.shape[1]
+    g = _kv_head(h, Hq, Hkv)
+    lo, hi, O, lse, dq, dk, dv = _rows_bwd(_f64(q[b, h]), _f64(k[b, g]), _f64(v[b, g]), _f64(do[b, h]),
+                                           scale, causal, window, r0, r1)
+    return O, lse, dq, lo, hi, dk, dv
 
 
 def attn_bwd(q, k, v, do, scale: float, causal: bool = False, window: int = 0, heads=None):

@@ -1,0 +1,108 @@
+"""Backward parity: dQ, dK, dV from the CUDA path against the float64 oracle.
+
+The forward outputs O and LSE fed to the backward pass come from the CUDA
+forward (as in training); the oracle recomputes everything from Q, K, V, dO
+in float64.  Tolerance: relative Frobenius error <= 2e-2 for each gradient.
+"""
+
+import numpy as np
+import pytest
+
+import oracle
+from synth import WORKLOADS, make_inputs, make_shape_inputs
+from tests._util import check_grad, to_dev, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def ta():
+    import torch
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    import tiled_exact_attention_02_b200 as ta
+    return ta
+
+
+def run_fwd_bwd(ta, x, causal, window, scale):
+    q, k, v, do = (to_dev(x[n]) for n in ("q", "k", "v", "do"))
+    o, lse = ta.attention(q, k, v, causal, window, scale)
+    dq, dk, dv = ta.attention_backward(q, k, v, o, lse, do, causal, window, scale)
+    st, site = ta.device_error()
+    assert st == 0, f"device error {st} at site {site}"
+    return to_f64(dq), to_f64(dk), to_f64(dv)
+
+
+EDGE = [
+    (1, 1, 1, 128, 128, 128, False, 0),
+    (1, 2, 2, 7, 7, 128, True, 0),
+    (1, 2, 1, 129, 129, 128, True, 0),
+    (2, 4, 2, 200, 200, 128, True, 0),
+    (1, 2, 2, 100, 333, 128, False, 0),
+    (1, 2, 2, 333, 100, 128, False, 0),
+    (1, 4, 4, 257, 257, 128, True, 1),
+    (1, 2, 2, 384, 384, 128, True, 1000),
+    (1, 8, 1, 256, 256, 128, True, 0),
+    (1, 6, 2, 300, 300, 128, True, 64),
+    (1, 2, 2, 300, 100, 128, True, 50),
+    (1, 1, 1, 128, 128, 64, False, 0),
+    (1, 2, 1, 200, 200, 64, True, 0),
+    (2, 4, 2, 333, 333, 64, True, 77),
+    (1, 2, 2, 1000, 1000, 128, True, 0),
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Lq,Lk,d,causal,window", EDGE)
+def test_bwd_edge_shapes(ta, B, Hq, Hkv, Lq, Lk, d, causal, window):
+    x = make_shape_inputs(B, Hq, Hkv, Lq, Lk, d, seed=Lq * 3 + Lk + d + 1, with_do=True)
+    scale = d ** -0.5
+    dq, dk, dv = run_fwd_bwd(ta, x, causal, window, scale)
+    rq, rk, rv = oracle.attn_bwd(x["q"], x["k"], x["v"], x["do"], scale, causal, window)
+    check_grad(dq, rq, "dQ")
+    check_grad(dk, rk, "dK")
+    check_grad(dv, rv, "dV")
+
+
+def test_bwd_gqa_window_2048(ta):
+    x = make_shape_inputs(1, 8, 2, 2048, 2048, 128, seed=17, with_do=True)
+    dq, dk, dv = run_fwd_bwd(ta, x, True, 300, 128 ** -0.5)
+    rq, rk, rv = oracle.attn_bwd(x["q"], x["k"], x["v"], x["do"], 128 ** -0.5, True, 300)
+    check_grad(dq, rq, "dQ")
+    check_grad(dk, rk, "dK")
+    check_grad(dv, rv, "dV")
+
+
+def test_bwd_full_size_sampled_heads(ta):
+    """The fwd+bwd workload at full size (benchmark launch configuration);
+    whole K/V heads (independent units) compared against the oracle."""
+    w = WORKLOADS["mha_causal_fwdbwd"]
+    x = make_inputs(w)
+    dq, dk, dv = run_fwd_bwd(ta, x, w.causal, w.window, w.scale)
+    heads = [(0, 0), (1, 31)]
+    rq, rk, rv = oracle.attn_bwd(x["q"], x["k"], x["v"], x["do"], w.scale, w.causal, w.window, heads=heads)
+    for b, h in heads:
+        check_grad(dq[b, h], rq[b, h], f"dQ[{b},{h}]")
+        check_grad(dk[b, h], rk[b, h], f"dK[{b},{h}]")
+        check_grad(dv[b, h], rv[b, h], f"dV[{b},{h}]")
+    assert np.all(np.isfinite(dq)) and np.all(np.isfinite(dk)) and np.all(np.isfinite(dv))
+
+
+def test_autograd_wrapper(ta):
+    import torch
+    x = make_shape_inputs(1, 2, 1, 300, 300, 128, seed=3, with_do=True)
+    q, k, v, do = (to_dev(x[n]).requires_grad_(n != "do") for n in ("q", "k", "v", "do"))
+    o = ta.tiled_attention(q, k, v, True, 0, None)
+    o.backward(do)
+    rq, rk, rv = oracle.attn_bwd(x["q"], x["k"], x["v"], x["do"], 128 ** -0.5, True, 0)
+    check_grad(to_f64(q.grad), rq, "dQ")
+    check_grad(to_f64(k.grad), rk, "dK")
+    check_grad(to_f64(v.grad), rv, "dV")
+
+
+def test_bwd_repeated_calls_identical_up_to_atomics(ta):
+    """Two backward calls on the same inputs agree (dQ differs only by the
+    order of fp32 atomic adds)."""
+    x = make_shape_inputs(1, 2, 2, 512, 512, 128, seed=8, with_do=True)
+    a = run_fwd_bwd(ta, x, True, 0, 128 ** -0.5)
+    b = run_fwd_bwd(ta, x, True, 0, 128 ** -0.5)
+    assert np.array_equal(a[1], b[1]) and np.array_equal(a[2], b[2])
+    assert np.max(np.abs(a[0] - b[0])) <= 2 ** -6 * max(1.0, np.max(np.abs(a[0])))

@@ -255,6 +255,27 @@ def test_row_blocking_is_invisible(monkeypatch):
     np.testing.assert_allclose(lrow, ref[1][0, 1, rows], atol=1e-14)
 
 
+def test_row_blocks_sum_to_full_backward():
+    """Row-block contributions (the benchmark's bounded CPU sample) add up to attn_bwd."""
+    B, Hq, Hkv, L, d = 1, 4, 2, 50, 8
+    q, do = _rand(B, Hq, L, d), _rand(B, Hq, L, d)
+    k, v = _rand(B, Hkv, L, d), _rand(B, Hkv, L, d)
+    O, lse = oracle.attn_fwd(q, k, v, 0.3, True, 11)
+    dq, dk, dv = oracle.attn_bwd(q, k, v, do, 0.3, True, 11)
+    sk, sv = np.zeros_like(dk), np.zeros_like(dv)
+    for h in range(Hq):
+        for r0 in range(0, L, 16):
+            r1 = min(L, r0 + 16)
+            Ob, lb, dqb, lo, hi, dkb, dvb = oracle.attn_row_block(q, k, v, do, 0.3, True, 11, 0, h, r0, r1)
+            np.testing.assert_allclose(Ob, O[0, h, r0:r1], atol=1e-14)
+            np.testing.assert_allclose(lb, lse[0, h, r0:r1], atol=1e-14)
+            np.testing.assert_allclose(dqb, dq[0, h, r0:r1], atol=1e-14)
+            sk[0, h // 2, lo:hi] += dkb
+            sv[0, h // 2, lo:hi] += dvb
+    np.testing.assert_allclose(sk, dk, atol=1e-13)
+    np.testing.assert_allclose(sv, dv, atol=1e-13)
+
+
 # ---------------------------------------------------------------- library cross-checks
 torch = pytest.importorskip("torch")
 

@@ -26,7 +26,10 @@ ATTN_ERR_TIMEOUT = 4
 class AttnError(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
-        super().__init__(f"{what}: {status_string(status)} ({status})")
+        msg = f"{what}: {status_string(status)} ({status})"
+        if status == ATTN_ERR_CUDA:
+            msg += f" [{lib.attn_last_cuda_error().decode()}]"
+        super().__init__(msg)
 
 
 def _load() -> ctypes.CDLL:
@@ -41,6 +44,14 @@ def _load() -> ctypes.CDLL:
     lib.attn_bwd_workspace_size.restype = sz
     lib.attn_bwd.argtypes = [vp] * 9 + [i] * 6 + [f, i, i, vp, sz, vp]
     lib.attn_bwd.restype = i
+    lib.attn_bwd_preprocess.argtypes = [vp, vp, i, i, i, i, vp, sz, vp]
+    lib.attn_bwd_preprocess.restype = i
+    lib.attn_bwd_main.argtypes = [vp] * 7 + [i] * 6 + [f, i, i, vp, sz, vp]
+    lib.attn_bwd_main.restype = i
+    lib.attn_bwd_finalize.argtypes = [vp, i, i, i, i, f, vp, sz, vp]
+    lib.attn_bwd_finalize.restype = i
+    lib.attn_last_cuda_error.argtypes = []
+    lib.attn_last_cuda_error.restype = ctypes.c_char_p
     lib.attn_status_string.argtypes = [i]
     lib.attn_status_string.restype = ctypes.c_char_p
     lib.attn_get_device_error.argtypes = [vp, ctypes.POINTER(i)]
@@ -121,6 +132,25 @@ def bwd(q, k, v, o, lse, do, dq, dk, dv, workspace, causal: bool = False, window
                       int(bool(causal)), int(window), workspace.data_ptr(),
                       workspace.numel() * workspace.element_size(), _stream_ptr(stream))
     _check(st, "attn_bwd")
+
+
+def bwd_phases(q, k, v, o, lse, do, dq, dk, dv, workspace, causal: bool = False, window: int = 0,
+               scale: float | None = None, stream=None, between=None):
+    """attn_bwd as its three C-ABI phases; `between(i)` (optional) is called
+    before phase i (0..2) and after the last (i = 3), e.g. to record events."""
+    B, Hq, Hkv, Lq, Lk, d = _shapes(q, k)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    ws, wsb, sp = workspace.data_ptr(), workspace.numel() * workspace.element_size(), _stream_ptr(stream)
+    hook = between or (lambda i: None)
+    hook(0)
+    _check(lib.attn_bwd_preprocess(o.data_ptr(), do.data_ptr(), B, Hq, Lq, d, ws, wsb, sp), "attn_bwd_preprocess")
+    hook(1)
+    _check(lib.attn_bwd_main(q.data_ptr(), k.data_ptr(), v.data_ptr(), lse.data_ptr(), do.data_ptr(),
+                             dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv, Lq, Lk, d, scale, int(bool(causal)),
+                             int(window), ws, wsb, sp), "attn_bwd_main")
+    hook(2)
+    _check(lib.attn_bwd_finalize(dq.data_ptr(), B, Hq, Lq, d, scale, ws, wsb, sp), "attn_bwd_finalize")
+    hook(3)
 
 
 def device_error(stream=None) -> tuple[int, int]:

@@ -5,6 +5,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <cstdio>
 #include <mutex>
 
 #include "../../include/tiledattn.h"
@@ -25,6 +26,18 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s without progress
 std::mutex g_mu;
 int* g_err_addr[kMaxDevices];
 
+thread_local char g_last_err[256];
+
+// Record a failed CUDA call for attn_last_cuda_error and map it to ATTN_ERR_CUDA.
+int cuda_fail(const char* step, cudaError_t e) {
+  snprintf(g_last_err, sizeof(g_last_err), "%s: %s (%d)", step, cudaGetErrorString(e), (int)e);
+  return ATTN_ERR_CUDA;
+}
+int cu_fail(const char* step, CUresult r) {
+  snprintf(g_last_err, sizeof(g_last_err), "%s: CUresult %d", step, (int)r);
+  return ATTN_ERR_CUDA;
+}
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -36,9 +49,9 @@ int get_encoder(EncodeTiledFn* fn) {
   if (!g_encode) {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess || !p)
-      return ATTN_ERR_CUDA;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+    if (e != cudaSuccess) return cuda_fail("cudaGetDriverEntryPoint", e);
+    if (q != cudaDriverEntryPointSuccess || !p) return cu_fail("cuTensorMapEncodeTiled lookup", CUDA_ERROR_NOT_FOUND);
     g_encode = reinterpret_cast<EncodeTiledFn>(p);
   }
   *fn = g_encode;
@@ -48,11 +61,14 @@ int get_encoder(EncodeTiledFn* fn) {
 // Device address of the current device's error word (looked up once per device).
 int get_err_word(int** out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
+  if (dev < 0 || dev >= kMaxDevices) return cuda_fail("cudaGetDevice", cudaErrorInvalidDevice);
   std::lock_guard<std::mutex> lk(g_mu);
   if (!g_err_addr[dev]) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_dev_err) != cudaSuccess) return ATTN_ERR_CUDA;
+    e = cudaGetSymbolAddress(&p, g_dev_err);
+    if (e != cudaSuccess) return cuda_fail("cudaGetSymbolAddress", e);
     g_err_addr[dev] = static_cast<int*>(p);
   }
   *out = g_err_addr[dev];
@@ -76,20 +92,21 @@ int check_shape(int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale, int 
   if ((int64_t)B * Hq > (1 << 24) || (int64_t)B * Hkv > (1 << 24)) return ATTN_ERR_UNSUPPORTED;
   if (Lq > (1 << 28) || Lk > (1 << 28)) return ATTN_ERR_UNSUPPORTED;
   if ((int64_t)B * Hq * ((Lq + 127) / 128) >= (int64_t)1 << 31) return ATTN_ERR_UNSUPPORTED;
+  if ((int64_t)B * Hkv * ((Lk + 127) / 128) >= (int64_t)1 << 31) return ATTN_ERR_UNSUPPORTED;
   return ATTN_OK;
 }
 
-// 3-D map over a [BH, L, d] bf16 tensor, box 64 x 128 x 1, 128-byte swizzle.
-// Rows past L inside a box read as zero.
-int make_map(EncodeTiledFn enc, CUtensorMap* m, const void* ptr, int BH, int L, int d) {
+// 3-D map over a [BH, L, d] bf16 tensor, box 64 x box_rows x 1, 128-byte
+// swizzle.  Rows past L inside a box read as zero.
+int make_map(EncodeTiledFn enc, CUtensorMap* m, const void* ptr, int BH, int L, int d, int box_rows = 128) {
   cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)(L > 0 ? L : 1), (cuuint64_t)(BH > 0 ? BH : 1)};
   cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)d * 2 * (cuuint64_t)(L > 0 ? L : 1)};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
   cuuint32_t es[3] = {1, 1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+  return r == CUDA_SUCCESS ? ATTN_OK : cu_fail("cuTensorMapEncodeTiled", r);
 }
 
 __global__ void selftest_wait_kernel(int* err, uint64_t limit_ns) {
@@ -149,7 +166,8 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   fwd_plan(P.prob, &P.n_units, &P.pair_heads);
   if ((st = get_err_word(&P.err)) != ATTN_OK) return st;
   P.limit_ns = kWaitLimitNs;
-  return launch_fwd(P, static_cast<cudaStream_t>(stream)) == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  const cudaError_t e = launch_fwd(P, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ATTN_OK : cuda_fail("attn_fwd launch", e);
 }
 
 size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int Lq, int Lk, int d) {
@@ -161,16 +179,128 @@ size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int Lq, int Lk, int d) {
   return dsz + dq;
 }
 
+// Workspace layout: D (fp32 [rows], padded to 256 bytes), then the fp32 dQ accumulator.
+static int split_workspace(int B, int Hq, int Lq, int d, void* workspace, size_t workspace_bytes, float** dvec,
+                           float** dq_acc) {
+  const size_t need = attn_bwd_workspace_size(B, Hq, 1, Lq, 1, d);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need)
+    return ATTN_ERR_INVALID_ARG;
+  const size_t rows = (size_t)B * Hq * Lq;
+  *dvec = static_cast<float*>(workspace);
+  *dq_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + (rows * 4 + 255) / 256 * 256);
+  return ATTN_OK;
+}
+
+int attn_bwd_preprocess(const void* o, const void* dO, int B, int Hq, int Lq, int d, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+  int st = check_shape(B, Hq, Hq > 0 ? 1 : 0, Lq, 1, d, 1.f, 0, 0);
+  if (st != ATTN_OK) return st;
+  if (B == 0 || Hq == 0 || Lq == 0) return ATTN_OK;
+  if (!o || !dO || !aligned16(o) || !aligned16(dO)) return ATTN_ERR_INVALID_ARG;
+  float *dvec, *dq_acc;
+  if ((st = split_workspace(B, Hq, Lq, d, workspace, workspace_bytes, &dvec, &dq_acc)) != ATTN_OK) return st;
+  const cudaError_t e =
+      launch_bwd_pre(o, dO, dvec, dq_acc, (int64_t)B * Hq * Lq, d, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ATTN_OK : cuda_fail("attn_bwd_preprocess launch", e);
+}
+
+int attn_bwd_main(const void* q, const void* k, const void* v, const float* lse, const void* dO, void* dk, void* dv,
+                  int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale, int causal, int window, void* workspace,
+                  size_t workspace_bytes, void* stream) {
+  int st = check_shape(B, Hq, Hkv, Lq, Lk, d, scale, causal, window);
+  if (st != ATTN_OK) return st;
+  if (B == 0 || Hq == 0 || Lk == 0) return ATTN_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (!k || !v || !dk || !dv || !aligned16(k) || !aligned16(v) || !aligned16(dk) || !aligned16(dv))
+    return ATTN_ERR_INVALID_ARG;
+  if (Lq == 0) {  // no query: dK = dV = 0
+    const size_t kv_bytes = (size_t)B * Hkv * Lk * d * 2;
+    cudaError_t e = cudaMemsetAsync(dk, 0, kv_bytes, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dv, 0, kv_bytes, s);
+    return e == cudaSuccess ? ATTN_OK : cuda_fail("cudaMemsetAsync dK/dV", e);
+  }
+  if (!q || !lse || !dO || !aligned16(q) || !aligned16(lse) || !aligned16(dO)) return ATTN_ERR_INVALID_ARG;
+  float *dvec, *dq_acc;
+  if ((st = split_workspace(B, Hq, Lq, d, workspace, workspace_bytes, &dvec, &dq_acc)) != ATTN_OK) return st;
+  EncodeTiledFn enc;
+  if ((st = get_encoder(&enc)) != ATTN_OK) return st;
+  BwdParams P;
+  memset(&P, 0, sizeof(P));
+  P.prob = Problem{B, Hq, Hkv, Lq, Lk, d, causal, window, scale};
+  const int bm = bwd_block_m(d);
+  if ((st = make_map(enc, &P.tm_q, q, B * Hq, Lq, d, bm)) != ATTN_OK) return st;
+  if ((st = make_map(enc, &P.tm_do, dO, B * Hq, Lq, d, bm)) != ATTN_OK) return st;
+  if ((st = make_map(enc, &P.tm_k, k, B * Hkv, Lk, d, 128)) != ATTN_OK) return st;
+  if ((st = make_map(enc, &P.tm_v, v, B * Hkv, Lk, d, 128)) != ATTN_OK) return st;
+  P.lse = lse;
+  P.dvec = dvec;
+  P.dq_acc = dq_acc;
+  P.dk = dk;
+  P.dv = dv;
+  P.scale = scale;
+  P.scale_log2 = scale * 1.4426950408889634f;
+  P.n_units = B * Hkv * ((Lk + 127) / 128);
+  if ((st = get_err_word(&P.err)) != ATTN_OK) return st;
+  P.limit_ns = kWaitLimitNs;
+  const cudaError_t e = launch_bwd(P, s);
+  return e == cudaSuccess ? ATTN_OK : cuda_fail("attn_bwd_main launch", e);
+}
+
+int attn_bwd_finalize(void* dq, int B, int Hq, int Lq, int d, float scale, void* workspace, size_t workspace_bytes,
+                      void* stream) {
+  int st = check_shape(B, Hq, Hq > 0 ? 1 : 0, Lq, 1, d, scale, 0, 0);
+  if (st != ATTN_OK) return st;
+  if (B == 0 || Hq == 0 || Lq == 0) return ATTN_OK;
+  if (!dq || !aligned16(dq)) return ATTN_ERR_INVALID_ARG;
+  float *dvec, *dq_acc;
+  if ((st = split_workspace(B, Hq, Lq, d, workspace, workspace_bytes, &dvec, &dq_acc)) != ATTN_OK) return st;
+  const cudaError_t e = launch_bwd_post(dq_acc, dq, (int64_t)B * Hq * Lq * d, scale, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ATTN_OK : cuda_fail("attn_bwd_finalize launch", e);
+}
+
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO, void* dq,
+             void* dk, void* dv, int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale, int causal, int window,
+             void* workspace, size_t workspace_bytes, void* stream) {
+  int st = check_shape(B, Hq, Hkv, Lq, Lk, d, scale, causal, window);
+  if (st != ATTN_OK) return st;
+  if (B == 0 || Hq == 0) return ATTN_OK;
+  if (Lq == 0 || Lk == 0) {
+    if (Lq == 0)  // dK = dV = 0
+      return attn_bwd_main(q, k, v, lse, dO, dk, dv, B, Hq, Hkv, Lq, Lk, d, scale, causal, window, workspace,
+                           workspace_bytes, stream);
+    // No key: every row is fully masked, dQ = 0.
+    if (!dq || !aligned16(dq)) return ATTN_ERR_INVALID_ARG;
+    const cudaError_t e = cudaMemsetAsync(dq, 0, (size_t)B * Hq * Lq * d * 2, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? ATTN_OK : cuda_fail("cudaMemsetAsync dQ", e);
+  }
+  // Validate every pointer before the first launch.
+  if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv || !aligned16(q) || !aligned16(k) || !aligned16(v) ||
+      !aligned16(o) || !aligned16(lse) || !aligned16(dO) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return ATTN_ERR_INVALID_ARG;
+  float *dvec, *dq_acc;
+  if ((st = split_workspace(B, Hq, Lq, d, workspace, workspace_bytes, &dvec, &dq_acc)) != ATTN_OK) return st;
+  if ((st = attn_bwd_preprocess(o, dO, B, Hq, Lq, d, workspace, workspace_bytes, stream)) != ATTN_OK) return st;
+  if ((st = attn_bwd_main(q, k, v, lse, dO, dk, dv, B, Hq, Hkv, Lq, Lk, d, scale, causal, window, workspace,
+                          workspace_bytes, stream)) != ATTN_OK)
+    return st;
+  return attn_bwd_finalize(dq, B, Hq, Lq, d, scale, workspace, workspace_bytes, stream);
+}
+
+const char* attn_last_cuda_error(void) { return g_last_err; }
+
 int attn_get_device_error(void* stream, int* site) {
   int* addr = nullptr;
   int st = get_err_word(&addr);
   if (st != ATTN_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaStreamSynchronize(s) != cudaSuccess) return ATTN_ERR_CUDA;
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail("cudaStreamSynchronize", e);
   int word = 0;
-  if (cudaMemcpyFromSymbol(&word, g_dev_err, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+  e = cudaMemcpyFromSymbol(&word, g_dev_err, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail("read error word", e);
   const int zero = 0;
-  if (cudaMemcpyToSymbol(g_dev_err, &zero, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+  e = cudaMemcpyToSymbol(g_dev_err, &zero, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail("clear error word", e);
   if (site) *site = word >> 8;
   return (word & 0xFF) == DEV_TIMEOUT ? ATTN_ERR_TIMEOUT : ATTN_OK;
 }
@@ -181,7 +311,8 @@ int attn_selftest_wait_timeout(int64_t limit_ns, void* stream) {
   int st = get_err_word(&err);
   if (st != ATTN_OK) return st;
   selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(err, (uint64_t)limit_ns);
-  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? ATTN_OK : cuda_fail("selftest launch", e);
 }
 
 }  // extern "C"

@@ -1,8 +1,609 @@
-// attn_bwd.cu - backward attention kernels for sm_100a (being written).
+// attn_bwd.cu - backward attention kernels for sm_100a.
+//
+// Recompute backward ("缩放定律与高效注意力" §3.3: only O and the per-row
+// logsumexp are kept from the forward pass; Q, K, V are read again and the
+// scores rebuilt tile by tile).  The gradient itself is the textbook softmax
+// gradient, which the pages do not print:
+//   D_i = dO_i . O_i,  P = exp(scale*S - LSE),  dV = P^T dO,  dP = dO V^T,
+//   dS = P * (dP - D),  dQ = scale * dS K,  dK = scale * dS^T Q.
+//
+// Three launches:
+//   bwd_pre   D_i for every query row, and zero the fp32 dQ accumulator
+//   bwd_main  one CTA per (batch, K/V head, tile of 128 keys); it loops over
+//             the query heads of the GQA group and the query tiles that see
+//             its keys, accumulating dK and dV in tensor memory for the whole
+//             loop and sending each step's dQ contribution to the fp32
+//             accumulator with a bulk reduce-add
+//   bwd_post  dQ = scale * accumulator, rounded to bf16
+//
+// bwd_main works in the transposed orientation, keys on the 128 TMEM lanes:
+//   S^T = K Q^T and dP^T = V dO^T     (M = 128 keys, N = BM query rows)
+//   dV += P^T dO and dK += dS^T Q     (M = 128 keys, N = d)
+//   dQ^T = K^T dS^T  (d = 128)  or  dQ = dS K  (d = 64)   (M = 128, N = 64)
+// so that one thread per key turns a row of S^T into P^T and dS^T, and the
+// bf16 P^T and dS^T, written once to shared memory, serve both as the K-major
+// A operand of dV/dK and as the MN-major operand of dQ.
+// Warp roles (384 threads): warp 0 TMA, warp 1 MMA issuer, warps 4-7 the
+// per-key softmax gradient, warps 8-11 the dQ drain.  Tensor memory: S^T |
+// dP^T | dV | dK | dQ, 448 of 512 columns.
+#include <cuda.h>
 #include <cuda_runtime.h>
-#include "../../include/tiledattn.h"
+#include <cstdint>
+#include <cmath>
 
-extern "C" int attn_bwd(const void*, const void*, const void*, const void*, const float*, const void*, void*, void*,
-                        void*, int, int, int, int, int, int, float, int, int, void*, size_t, void*) {
-  return ATTN_ERR_UNSUPPORTED;
+#include "sm100.cuh"
+#include "attn_common.cuh"
+#include "attn_kernels.h"
+
+namespace tea {
+namespace bwd {
+
+constexpr int BN = 128;  // keys per CTA
+constexpr int THREADS = 384;
+constexpr int KPANEL = 16384;  // 128 rows x 128 bytes
+constexpr float LOG2E = 1.4426950408889634f;
+
+template <int D>
+struct Cfg {
+  static constexpr int BM = D == 128 ? 64 : 128;  // query rows per step
+  static constexpr int NBUF = D == 128 ? 2 : 1;   // P^T / dS^T buffers
+  static constexpr int KV_TILE = BN * D * 2;
+  static constexpr int Q_TILE = BM * D * 2;
+  static constexpr int Q_PANEL = BM * 128;
+  static constexpr int PS_TILE = BN * BM * 2;
+  static constexpr int STAGE_BYTES = BM * D * 4;
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + KV_TILE;
+  static constexpr int OFF_Q = OFF_V + KV_TILE;
+  static constexpr int OFF_DO = OFF_Q + 2 * Q_TILE;
+  static constexpr int OFF_PT = OFF_DO + 2 * Q_TILE;
+  static constexpr int OFF_DST = OFF_PT + NBUF * PS_TILE;
+  static constexpr int OFF_STG = OFF_DST + NBUF * PS_TILE;
+  static constexpr int OFF_VEC = OFF_STG + STAGE_BYTES;  // [2 bufs][lse2 | D][BM] fp32
+  static constexpr int OFF_BAR = OFF_VEC + 2 * 2 * BM * 4;
+  static constexpr int SMEM = OFF_BAR + 256 + 1024;
+  static constexpr uint32_t T_S = 0, T_DP = BM, T_DV = 2 * BM, T_DK = 2 * BM + D, T_DQ = 2 * BM + 2 * D;
+  static_assert(T_DQ + 64 <= 512, "tensor memory budget");
+};
+
+struct Bars {
+  uint64_t kv_full;
+  uint64_t q_full[2], q_empty[2];
+  uint64_t sdp_full, s_consumed;
+  uint64_t ds_full[2], ds_empty[2];
+  uint64_t dq_full, dq_empty;
+  uint64_t vec_full[2];
+  uint64_t stg_full, stg_free;
+  uint64_t dkv_full;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+struct Unit {
+  int b, kvh, k0;
+  int G, nq, qt_lo, n_steps;
+};
+
+template <int D>
+__device__ __forceinline__ Unit decode_unit(const BwdParams& P, int idx) {
+  const Problem& p = P.prob;
+  Unit u;
+  const int per = p.B * p.Hkv;
+  const int n = idx / per;  // key tile; early keys see the most queries: heavy first
+  const int rem = idx % per;
+  u.b = rem / p.Hkv;
+  u.kvh = rem % p.Hkv;
+  u.k0 = n * BN;
+  u.G = p.Hq / p.Hkv;
+  int q_lo, q_hi;
+  q_row_range(p, u.k0, u.k0 + BN, q_lo, q_hi);
+  constexpr int BM = Cfg<D>::BM;
+  u.qt_lo = q_lo / BM;
+  u.nq = q_hi > q_lo ? cdiv(q_hi, BM) - u.qt_lo : 0;
+  u.n_steps = u.G * u.nq;
+  return u;
 }
+
+// Step i of a unit: query head h (global head index) and first query row q0.
+template <int D>
+__device__ __forceinline__ void step_of(const Unit& u, int i, int& h, int& q0) {
+  const int g = i / u.nq;
+  h = u.kvh * u.G + g;
+  q0 = (u.qt_lo + i % u.nq) * Cfg<D>::BM;
+}
+
+// ------------------------------------------------------------------ producer
+template <int D>
+__device__ void producer(const BwdParams& P, const Unit& u, uint8_t* smem, Bars& bars, const WaitGuard& g) {
+  using C = Cfg<D>;
+  const Problem& p = P.prob;
+  tma_prefetch_desc(&P.tm_q);
+  tma_prefetch_desc(&P.tm_do);
+  tma_prefetch_desc(&P.tm_k);
+  tma_prefetch_desc(&P.tm_v);
+  mbar_arrive_expect_tx(&bars.kv_full, 2 * C::KV_TILE);
+  for (int pnl = 0; pnl < D / 64; pnl++) {
+    tma_load_3d(smem + C::OFF_K + pnl * KPANEL, &P.tm_k, &bars.kv_full, pnl * 64, u.k0, u.b * p.Hkv + u.kvh);
+    tma_load_3d(smem + C::OFF_V + pnl * KPANEL, &P.tm_v, &bars.kv_full, pnl * 64, u.k0, u.b * p.Hkv + u.kvh);
+  }
+  int issued = 0;
+  for (int i = 0; i < u.n_steps; i++) {
+    const int st = i & 1;
+    if (!mbar_wait(&bars.q_empty[st], ((i >> 1) & 1) ^ 1, g, 1)) break;
+    int h, q0;
+    step_of<D>(u, i, h, q0);
+    mbar_arrive_expect_tx(&bars.q_full[st], 2 * C::Q_TILE);
+    for (int pnl = 0; pnl < D / 64; pnl++) {
+      tma_load_3d(smem + C::OFF_Q + st * C::Q_TILE + pnl * C::Q_PANEL, &P.tm_q, &bars.q_full[st], pnl * 64, q0,
+                  u.b * p.Hq + h);
+      tma_load_3d(smem + C::OFF_DO + st * C::Q_TILE + pnl * C::Q_PANEL, &P.tm_do, &bars.q_full[st], pnl * 64, q0,
+                  u.b * p.Hq + h);
+    }
+    issued = i + 1;
+  }
+  // Let every copy this warp started land before the CTA may exit (bounded).
+  mbar_wait_ignore_abort(&bars.kv_full, 0, g);
+  for (int i = imax(0, issued - 2); i < issued; i++) mbar_wait_ignore_abort(&bars.q_full[i & 1], (i >> 1) & 1, g);
+}
+
+// ------------------------------------------------------------------ MMA issuer
+template <int D>
+__device__ void mma_issuer(const BwdParams& P, const Unit& u, uint8_t* smem, Bars& bars, uint32_t tmem,
+                           const WaitGuard& g) {
+  using C = Cfg<D>;
+  constexpr int BM = C::BM;
+  const uint32_t idesc_s = idesc_bf16_f32(128, BM, 0, 0);
+  const uint32_t idesc_dkv = idesc_bf16_f32(128, D, 0, 1);
+  const uint32_t idesc_dq = idesc_bf16_f32(128, 64, 1, 1);
+  const uint32_t k_addr = smem_u32(smem + C::OFF_K);
+  const uint32_t v_addr = smem_u32(smem + C::OFF_V);
+  const uint32_t q_addr = smem_u32(smem + C::OFF_Q);
+  const uint32_t do_addr = smem_u32(smem + C::OFF_DO);
+  const uint32_t pt_addr = smem_u32(smem + C::OFF_PT);
+  const uint32_t dst_addr = smem_u32(smem + C::OFF_DST);
+
+  // S^T = K Q^T and dP^T = V dO^T for step i (contraction over d).
+  auto issue_sdp = [&](int i) {
+    const uint32_t qa = q_addr + (i & 1) * C::Q_TILE;
+    const uint32_t da = do_addr + (i & 1) * C::Q_TILE;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; kk++) {
+      const uint32_t oa = (kk / 4) * KPANEL + (kk % 4) * 32;
+      const uint32_t ob = (kk / 4) * C::Q_PANEL + (kk % 4) * 32;
+      mma_ss(tmem + C::T_S, sw128_desc(k_addr + oa, 16, 1024), sw128_desc(qa + ob, 16, 1024), idesc_s, kk > 0);
+    }
+#pragma unroll
+    for (int kk = 0; kk < D / 16; kk++) {
+      const uint32_t oa = (kk / 4) * KPANEL + (kk % 4) * 32;
+      const uint32_t ob = (kk / 4) * C::Q_PANEL + (kk % 4) * 32;
+      mma_ss(tmem + C::T_DP, sw128_desc(v_addr + oa, 16, 1024), sw128_desc(da + ob, 16, 1024), idesc_s, kk > 0);
+    }
+    mma_commit(&bars.sdp_full);
+  };
+
+  if (u.n_steps == 0) goto done;
+  if (!mbar_wait(&bars.kv_full, 0, g, 10)) goto done;
+  if (!mbar_wait(&bars.q_full[0], 0, g, 11)) goto done;
+  tc_fence_after();
+  issue_sdp(0);
+
+  for (int i = 0; i < u.n_steps; i++) {
+    if (i + 1 < u.n_steps) {
+      if (!mbar_wait(&bars.q_full[(i + 1) & 1], ((i + 1) >> 1) & 1, g, 12)) goto done;
+      if (!mbar_wait(&bars.s_consumed, i & 1, g, 13)) goto done;
+      tc_fence_after();
+      issue_sdp(i + 1);
+    }
+    const int buf = i % C::NBUF;
+    if (!mbar_wait(&bars.ds_full[buf], (i / C::NBUF) & 1, g, 14)) goto done;
+    tc_fence_after();
+    const uint32_t qa = q_addr + (i & 1) * C::Q_TILE;
+    const uint32_t da = do_addr + (i & 1) * C::Q_TILE;
+    const uint32_t pa = pt_addr + buf * C::PS_TILE;
+    const uint32_t sa = dst_addr + buf * C::PS_TILE;
+    // dV += P^T dO and dK += dS^T Q (contraction over the BM query rows).
+#pragma unroll
+    for (int kk = 0; kk < BM / 16; kk++) {
+      const uint32_t oa = (kk / 4) * KPANEL + (kk % 4) * 32;
+      mma_ss(tmem + C::T_DV, sw128_desc(pa + oa, 16, 1024), sw128_desc(da + kk * 2048, C::Q_PANEL, 1024),
+             idesc_dkv, (i > 0) || (kk > 0));
+    }
+#pragma unroll
+    for (int kk = 0; kk < BM / 16; kk++) {
+      const uint32_t oa = (kk / 4) * KPANEL + (kk % 4) * 32;
+      mma_ss(tmem + C::T_DK, sw128_desc(sa + oa, 16, 1024), sw128_desc(qa + kk * 2048, C::Q_PANEL, 1024),
+             idesc_dkv, (i > 0) || (kk > 0));
+    }
+    // dQ contribution of this key tile (contraction over the 128 keys).
+    if (!mbar_wait(&bars.dq_empty, (i & 1) ^ 1, g, 15)) goto done;
+    tc_fence_after();
+#pragma unroll
+    for (int kk = 0; kk < BN / 16; kk++) {
+      if (D == 128)  // dQ^T = K^T dS^T: A = K (M = d), B = dS^T (N = query rows)
+        mma_ss(tmem + C::T_DQ, sw128_desc(k_addr + kk * 2048, KPANEL, 1024), sw128_desc(sa + kk * 2048, KPANEL, 1024),
+               idesc_dq, kk > 0);
+      else  // dQ = dS K: A = dS^T viewed MN-major (M = query rows), B = K (N = d)
+        mma_ss(tmem + C::T_DQ, sw128_desc(sa + kk * 2048, KPANEL, 1024), sw128_desc(k_addr + kk * 2048, KPANEL, 1024),
+               idesc_dq, kk > 0);
+    }
+    mma_commit(&bars.dq_full);
+    mma_commit(&bars.ds_empty[buf]);
+    mma_commit(&bars.q_empty[i & 1]);
+  }
+done:
+  mma_commit(&bars.dkv_full);
+  mma_commit(&bars.drain);
+  mbar_wait_ignore_abort(&bars.drain, 0, g);
+}
+
+// ------------------------------------------------------------------ softmax gradient
+// Thread `row` owns key k0 + row (TMEM lane row) and turns its row of S^T and
+// dP^T into P^T = exp2(c*S - LSE*log2e) and dS^T = P^T * (dP^T - D), written
+// as bf16 rows of the 128-byte-swizzled shared tiles.
+template <int D>
+__device__ void grad_rows(const BwdParams& P, const Unit& u, uint8_t* smem, Bars& bars, uint32_t tmem,
+                          const WaitGuard& g) {
+  using C = Cfg<D>;
+  constexpr int BM = C::BM;
+  const Problem& p = P.prob;
+  const int t = threadIdx.x - 128;  // 0..127
+  const int wl = (threadIdx.x / 32) % 4;
+  const int lane = threadIdx.x % 32;
+  const int row = t;
+  const int key = u.k0 + row;
+  const uint32_t lane_base = (uint32_t)(wl * 32) << 16;
+  // Queries [vis_lo, vis_hi) see this key.
+  int vis_lo = 0, vis_hi = 0;
+  if (key < p.Lk) {
+    vis_lo = p.causal ? key : 0;
+    vis_hi = p.window > 0 ? imin(p.Lq, key + p.window) : p.Lq;
+  }
+  const float c = P.scale_log2;
+  float* vec = reinterpret_cast<float*>(smem + C::OFF_VEC);
+  uint8_t* pt_base = smem + C::OFF_PT;
+  uint8_t* dst_base = smem + C::OFF_DST;
+  const uint32_t sw = (uint32_t)(row & 7);
+
+  for (int i = 0; i < u.n_steps; i++) {
+    int h, q0;
+    step_of<D>(u, i, h, q0);
+    // Per-query LSE (log2 units) and D for this step, shared by the group.
+    const int vb = i & 1;
+    if (t < BM) {
+      const int q = q0 + t;
+      const size_t r = (size_t)(u.b * p.Hq + h) * p.Lq + q;
+      vec[(vb * 2 + 0) * BM + t] = q < p.Lq ? P.lse[r] * LOG2E : INFINITY;  // +inf: row past Lq gives p = 0
+      vec[(vb * 2 + 1) * BM + t] = q < p.Lq ? P.dvec[r] : 0.f;
+    }
+    mbar_arrive(&bars.vec_full[vb]);
+    if (!mbar_wait(&bars.vec_full[vb], (i >> 1) & 1, g, 20)) return;
+    const float* lse2 = vec + (vb * 2 + 0) * BM;
+    const float* dd = vec + (vb * 2 + 1) * BM;
+    const bool full = vis_lo <= q0 && q0 + BM <= vis_hi;
+
+    if (!mbar_wait(&bars.sdp_full, i & 1, g, 21)) return;
+    tc_fence_after();
+    const int buf = i % C::NBUF;
+    uint8_t* pt_row = pt_base + buf * C::PS_TILE + row * 128;
+    uint8_t* ds_row = dst_base + buf * C::PS_TILE + row * 128;
+
+    // The BM columns go in chunks of 32 (one 32-column TMEM load each of S^T
+    // and dP^T); a chunk's four 16-byte pieces go to shared memory.
+    constexpr int NCH = BM / 32;
+    auto emit_chunk = [&](int ch, const uint32_t* sv, const uint32_t* dpv) {
+#pragma unroll
+      for (int piece = 0; piece < 4; piece++) {
+        uint32_t pw[4], dw[4];
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+          float pr[2], dr[2];
+#pragma unroll
+          for (int z = 0; z < 2; z++) {
+            const int col = piece * 8 + e * 2 + z;  // column within the chunk
+            const int qq = ch * 32 + col;           // query within the step
+            float pv = ex2_approx(fmaf(__uint_as_float(sv[col]), c, -lse2[qq]));
+            if (!full) {
+              const int q = q0 + qq;
+              if (q < vis_lo || q >= vis_hi) pv = 0.f;
+            }
+            pr[z] = pv;
+            dr[z] = pv * (__uint_as_float(dpv[col]) - dd[qq]);
+          }
+          pw[e] = pack_bf16x2(pr[0], pr[1]);
+          dw[e] = pack_bf16x2(dr[0], dr[1]);
+        }
+        // 16-byte piece j of the row lives in panel j / 8, at chunk (j % 8) ^ (row % 8).
+        const int j = ch * 4 + piece;
+        const uint32_t off = (uint32_t)(j / 8) * KPANEL + (((uint32_t)(j % 8) ^ sw) << 4);
+        *reinterpret_cast<uint4*>(pt_row + off) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
+        *reinterpret_cast<uint4*>(ds_row + off) = make_uint4(dw[0], dw[1], dw[2], dw[3]);
+      }
+    };
+    if constexpr (NCH <= 2) {
+      // Small step: read all of S^T / dP^T first so the next step's MMAs can
+      // start while this one is being turned into P^T / dS^T.
+      uint32_t sv[NCH][32], dpv[NCH][32];
+#pragma unroll
+      for (int ch = 0; ch < NCH; ch++) {
+        tmem_ld32p(tmem + lane_base + C::T_S + 32 * ch, sv[ch]);
+        tmem_ld32p(tmem + lane_base + C::T_DP + 32 * ch, dpv[ch]);
+      }
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.s_consumed);  // S^T / dP^T may be overwritten
+      if (!mbar_wait(&bars.ds_empty[buf], ((i / C::NBUF) & 1) ^ 1, g, 22)) return;
+#pragma unroll
+      for (int ch = 0; ch < NCH; ch++) emit_chunk(ch, sv[ch], dpv[ch]);
+    } else {
+      if (!mbar_wait(&bars.ds_empty[buf], ((i / C::NBUF) & 1) ^ 1, g, 22)) return;
+#pragma unroll
+      for (int ch = 0; ch < NCH; ch++) {
+        uint32_t sv[32], dpv[32];
+        tmem_ld32p(tmem + lane_base + C::T_S + 32 * ch, sv);
+        tmem_ld32p(tmem + lane_base + C::T_DP + 32 * ch, dpv);
+        tmem_wait_ld();
+        if (ch == NCH - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars.s_consumed);
+        }
+        emit_chunk(ch, sv, dpv);
+      }
+    }
+    fence_proxy_async_smem();  // generic-proxy stores -> tensor-core reads
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bars.ds_full[buf]);
+  }
+
+  // Epilogue: dV and scale * dK for this thread's key.
+  const bool has = u.n_steps > 0;
+  if (has) {
+    if (!mbar_wait(&bars.dkv_full, 0, g, 23)) return;
+    tc_fence_after();
+  }
+  const bool write = key < p.Lk;
+  const size_t off = ((size_t)(u.b * p.Hkv + u.kvh) * p.Lk + key) * D;
+#pragma unroll
+  for (int which = 0; which < 2; which++) {
+    uint4* out = reinterpret_cast<uint4*>(static_cast<uint16_t*>(which ? P.dk : P.dv) + off);
+    const float f = which ? P.scale : 1.f;
+    const uint32_t col0 = which ? C::T_DK : C::T_DV;
+#pragma unroll
+    for (int q = 0; q < D / 32; q++) {
+      uint32_t o[32];
+      if (has) {
+        tmem_ld32p(tmem + lane_base + col0 + 32 * q, o);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; e++) o[e] = 0u;
+      }
+      uint32_t w[16];
+#pragma unroll
+      for (int e = 0; e < 16; e++) w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * f, __uint_as_float(o[2 * e + 1]) * f);
+      if (write) {
+#pragma unroll
+        for (int v = 0; v < 4; v++) out[q * 4 + v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ dQ drain
+// Moves each step's 128 x 64 fp32 dQ tile from tensor memory to a linear
+// shared-memory staging tile [query][d] and adds it into the fp32
+// accumulator with one bulk reduce-add (element-wise atomic in L2).
+template <int D>
+__device__ void dq_drain(const BwdParams& P, const Unit& u, uint8_t* smem, Bars& bars, uint32_t tmem,
+                         const WaitGuard& g) {
+  using C = Cfg<D>;
+  constexpr int BM = C::BM;
+  const Problem& p = P.prob;
+  const int t = threadIdx.x - 256;  // 0..127 = TMEM lane
+  const int wl = (threadIdx.x / 32) % 4;
+  const int lane = threadIdx.x % 32;
+  const uint32_t lane_base = (uint32_t)(wl * 32) << 16;
+  float* stg = reinterpret_cast<float*>(smem + C::OFF_STG);
+
+  for (int i = 0; i < u.n_steps; i++) {
+    int h, q0;
+    step_of<D>(u, i, h, q0);
+    if (!mbar_wait(&bars.dq_full, i & 1, g, 30)) break;
+    tc_fence_after();
+    uint32_t r[64];
+    tmem_ld32p(tmem + lane_base + C::T_DQ, r);
+    tmem_ld32p(tmem + lane_base + C::T_DQ + 32, r + 32);
+    tmem_wait_ld();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bars.dq_empty);
+    // The previous step's bulk reduce must have finished reading the staging tile.
+    if (!mbar_wait(&bars.stg_free, (i & 1) ^ 1, g, 31)) break;
+    if (D == 128) {
+      // Lane t holds dQ^T row t (= column d of dQ) for the BM = 64 queries.
+#pragma unroll
+      for (int qq = 0; qq < 64; qq++) stg[qq * D + t] = __uint_as_float(r[qq]);
+    } else {
+      // Lane t holds dQ row t (query q0 + t), 64 values of d.
+      float4* dst = reinterpret_cast<float4*>(stg + t * D);
+#pragma unroll
+      for (int v = 0; v < 16; v++)
+        dst[v] = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]), __uint_as_float(r[4 * v + 2]),
+                             __uint_as_float(r[4 * v + 3]));
+    }
+    fence_proxy_async_smem();
+    mbar_arrive(&bars.stg_full);
+    if (t == 0) {
+      if (!mbar_wait(&bars.stg_full, i & 1, g, 32)) break;
+      const int rows = imin(BM, p.Lq - q0);
+      float* dst = P.dq_acc + ((size_t)(u.b * p.Hq + h) * p.Lq + q0) * D;
+      bulk_reduce_add_f32(dst, stg, (uint32_t)(rows * D * 4));
+      bulk_commit();
+      bulk_wait_read_all();
+      mbar_arrive(&bars.stg_free);
+    }
+  }
+  if (t == 0) bulk_wait_all();
+}
+
+// ------------------------------------------------------------------ kernel
+template <int D>
+__global__ void __launch_bounds__(THREADS, 1) attn_bwd_kernel(const __grid_constant__ BwdParams P) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  Bars& bars = *reinterpret_cast<Bars*>(smem + C::OFF_BAR);
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const Unit u = decode_unit<D>(P, blockIdx.x);
+  const WaitGuard g{P.err, &bars.abort_flag, P.limit_ns, 100};
+
+  if (threadIdx.x == 0) {
+    bars.abort_flag = 0;
+    mbar_init(&bars.kv_full, 1);
+    for (int s = 0; s < 2; s++) {
+      mbar_init(&bars.q_full[s], 1);
+      mbar_init(&bars.q_empty[s], 1);
+      mbar_init(&bars.ds_full[s], 4);
+      mbar_init(&bars.ds_empty[s], 1);
+      mbar_init(&bars.vec_full[s], 128);
+    }
+    mbar_init(&bars.sdp_full, 1);
+    mbar_init(&bars.s_consumed, 4);
+    mbar_init(&bars.dq_full, 1);
+    mbar_init(&bars.dq_empty, 4);
+    mbar_init(&bars.stg_full, 128);
+    mbar_init(&bars.stg_free, 1);
+    mbar_init(&bars.dkv_full, 1);
+    mbar_init(&bars.drain, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars.tmem_base;
+
+  // Registers: 384 x 168 at launch; load/MMA group 80, the two others 208.
+  if (warp < 4) {
+    regs_dec<80>();
+    if (warp == 0) {
+      if (lane == 0) producer<D>(P, u, smem, bars, g);
+    } else if (warp == 1) {
+      if (lane == 0) mma_issuer<D>(P, u, smem, bars, tmem, g);
+    }
+  } else if (warp < 8) {
+    regs_inc<208>();
+    grad_rows<D>(P, u, smem, bars, tmem, g);
+  } else {
+    regs_inc<208>();
+    dq_drain<D>(P, u, smem, bars, tmem, g);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------ pre / post
+// D_i = sum_c dO_ic * O_ic for every row (fp32), and zero the dQ accumulator.
+// Threads in groups of d/8, each reading 8 bf16 of O and dO (16 bytes each).
+template <int D>
+__global__ void __launch_bounds__(256) bwd_pre_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dO,
+                                                      float* __restrict__ dvec, float* __restrict__ dq_acc,
+                                                      int64_t rows) {
+  constexpr int TPR = D / 8;  // threads per row
+  const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  const int64_t n = ((rows * TPR + 255) / 256) * 256;  // keep whole warps in the loop
+  for (int64_t x = tid; x < n; x += stride) {
+    const int64_t r = x / TPR;
+    const int part = (int)(x % TPR);
+    float acc = 0.f;
+    if (r < rows) {
+      const uint4 a = *reinterpret_cast<const uint4*>(o + r * D + part * 8);
+      const uint4 b = *reinterpret_cast<const uint4*>(dO + r * D + part * 8);
+      const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int e = 0; e < 4; e++) {
+        acc = fmaf(__uint_as_float(aw[e] << 16), __uint_as_float(bw[e] << 16), acc);
+        acc = fmaf(__uint_as_float(aw[e] & 0xFFFF0000u), __uint_as_float(bw[e] & 0xFFFF0000u), acc);
+      }
+      float4* z = reinterpret_cast<float4*>(dq_acc + r * D + part * 8);
+      z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+      z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int sh = TPR / 2; sh > 0; sh >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, sh);
+    if (r < rows && part == 0) dvec[r] = acc;
+  }
+}
+
+// dQ = scale * accumulator, rounded to bf16; 8 elements per thread.
+__global__ void __launch_bounds__(256) bwd_post_kernel(const float* __restrict__ acc, uint16_t* __restrict__ dq,
+                                                       int64_t n8, float scale) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; x < n8; x += stride) {
+    const float4 a = reinterpret_cast<const float4*>(acc)[2 * x];
+    const float4 b = reinterpret_cast<const float4*>(acc)[2 * x + 1];
+    uint4 w;
+    w.x = pack_bf16x2(a.x * scale, a.y * scale);
+    w.y = pack_bf16x2(a.z * scale, a.w * scale);
+    w.z = pack_bf16x2(b.x * scale, b.y * scale);
+    w.w = pack_bf16x2(b.z * scale, b.w * scale);
+    reinterpret_cast<uint4*>(dq)[x] = w;
+  }
+}
+
+}  // namespace bwd
+
+static int elementwise_grid(int64_t work_threads) {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t want = (work_threads + 255) / 256;
+  const int64_t cap = (int64_t)sms * 8;
+  return (int)(want < cap ? (want > 0 ? want : 1) : cap);
+}
+
+cudaError_t launch_bwd_pre(const void* o, const void* dO, float* dvec, float* dq_acc, int64_t rows, int d,
+                           cudaStream_t stream) {
+  if (rows <= 0) return cudaSuccess;
+  const int grid = elementwise_grid(rows * (d / 8));
+  if (d == 128)
+    bwd::bwd_pre_kernel<128><<<grid, 256, 0, stream>>>(static_cast<const uint16_t*>(o),
+                                                        static_cast<const uint16_t*>(dO), dvec, dq_acc, rows);
+  else
+    bwd::bwd_pre_kernel<64><<<grid, 256, 0, stream>>>(static_cast<const uint16_t*>(o),
+                                                       static_cast<const uint16_t*>(dO), dvec, dq_acc, rows);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_post(const float* dq_acc, void* dq, int64_t n, float scale, cudaStream_t stream) {
+  if (n <= 0) return cudaSuccess;
+  const int64_t n8 = n / 8;
+  bwd::bwd_post_kernel<<<elementwise_grid(n8), 256, 0, stream>>>(dq_acc, static_cast<uint16_t*>(dq), n8, scale);
+  return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t launch_bwd_d(const BwdParams& P, cudaStream_t stream) {
+  constexpr int smem = bwd::Cfg<D>::SMEM;
+  cudaError_t e = cudaFuncSetAttribute(bwd::attn_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  bwd::attn_bwd_kernel<D><<<P.n_units, bwd::THREADS, smem, stream>>>(P);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd(const BwdParams& P, cudaStream_t stream) {
+  if (P.n_units <= 0) return cudaSuccess;
+  return P.prob.d == 128 ? launch_bwd_d<128>(P, stream) : launch_bwd_d<64>(P, stream);
+}
+
+}  // namespace tea

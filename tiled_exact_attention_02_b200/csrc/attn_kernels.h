@@ -21,6 +21,32 @@ struct FwdParams {
   uint64_t limit_ns; // bounded-wait limit
 };
 
+struct BwdParams {
+  CUtensorMap tm_q;   // [B*Hq, Lq, d], box 64 x BM x 1 (BM = query rows per step)
+  CUtensorMap tm_do;  // [B*Hq, Lq, d], same box
+  CUtensorMap tm_k;   // [B*Hkv, Lk, d], box 64 x 128 x 1
+  CUtensorMap tm_v;   // [B*Hkv, Lk, d], same box
+  Problem prob;
+  const float* lse;   // fp32 [B, Hq, Lq], natural log (forward output)
+  const float* dvec;  // fp32 [B, Hq, Lq], D_i = dO_i . O_i (workspace)
+  float* dq_acc;      // fp32 [B, Hq, Lq, d], sum over key tiles of dS K (workspace)
+  void* dk;           // bf16 [B, Hkv, Lk, d]
+  void* dv;           // bf16 [B, Hkv, Lk, d]
+  float scale;
+  float scale_log2;
+  int n_units;        // CTAs: B * Hkv * key tiles
+  int* err;
+  uint64_t limit_ns;
+};
+
+// Query rows per backward step for head dimension d.
+inline int bwd_block_m(int d) { return d == 128 ? 64 : 128; }
+
+cudaError_t launch_bwd_pre(const void* o, const void* dO, float* dvec, float* dq_acc, int64_t rows, int d,
+                           cudaStream_t stream);
+cudaError_t launch_bwd(const BwdParams& P, cudaStream_t stream);
+cudaError_t launch_bwd_post(const float* dq_acc, void* dq, int64_t n, float scale, cudaStream_t stream);
+
 // Number of CTAs of the forward grid and whether heads are paired.
 void fwd_plan(const Problem& p, int* n_units, int* pair_heads);
 cudaError_t launch_fwd(const FwdParams& P, cudaStream_t stream);
