@@ -122,6 +122,30 @@ ATTN_API int attn_bwd_main(const void* q, const void* k, const void* v, const fl
 ATTN_API int attn_bwd_finalize(void* dq, int B, int Hq, int Lq, int d, float scale, void* workspace,
                                size_t workspace_bytes, void* stream);
 
+/*
+ * attn_bwd without a workspace argument, for callers that cannot allocate
+ * device memory (for example a plugin inside a framework that owns every
+ * device allocation, or a latency-critical path that must not call
+ * cudaMalloc).  It allocates nothing: the workspace lives in a fixed 32 MiB
+ * array of the library's own device memory, which every GPU that loads the
+ * library holds until the process exits.  The pages have no counterpart;
+ * this is a deployment convenience.
+ *
+ *  - Arguments, layouts and results are those of attn_bwd.
+ *  - Problems whose attn_bwd_workspace_size exceeds 32 MiB (33554432 bytes)
+ *    return ATTN_ERR_UNSUPPORTED before anything runs; at d = 128 that is
+ *    about 65,000 query rows (B * Hq * Lq).
+ *  - The first call on a device looks up the array's device address (with
+ *    that device current); make that first call before any stream capture.
+ *  - Every call on a device shares the one array.  Each call rewrites all of
+ *    it that it reads (D and the zeroed dQ accumulator), but calls whose work
+ *    overlaps on the GPU (different streams, or different host threads
+ *    without ordering) race on it and give wrong results.
+ */
+ATTN_API int attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                              const void* dO, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Lq, int Lk,
+                              int d, float scale, int causal, int window, void* stream);
+
 /* Static, human-readable name of a status code. */
 ATTN_API const char* attn_status_string(int status);
 
