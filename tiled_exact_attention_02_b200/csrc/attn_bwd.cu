@@ -12,8 +12,8 @@
 //   bwd_main  one CTA per (batch, K/V head, tile of 128 keys); it loops over
 //             the query heads of the GQA group and the query tiles that see
 //             its keys, accumulating dK and dV in tensor memory for the whole
-//             loop and sending each step's dQ contribution to the fp32
-//             accumulator with a bulk reduce-add
+//             loop and adding each step's dQ contribution into the fp32
+//             accumulator with coalesced atomic adds (red.global)
 //   bwd_post  dQ = scale * accumulator, rounded to bf16
 //
 // bwd_main works in the transposed orientation, keys on the 128 TMEM lanes:
@@ -23,9 +23,10 @@
 // so that one thread per key turns a row of S^T into P^T and dS^T, and the
 // bf16 P^T and dS^T, written once to shared memory, serve both as the K-major
 // A operand of dV/dK and as the MN-major operand of dQ.
-// Warp roles (384 threads): warp 0 TMA, warp 1 MMA issuer, warps 4-7 the
-// per-key softmax gradient, warps 8-11 the dQ drain.  Tensor memory: S^T |
-// dP^T | dV | dK | dQ, 448 of 512 columns.
+// Warp roles (512 threads): warp 0 TMA, warp 1 MMA issuer, warps 4-7 and
+// 8-11 the per-key softmax gradient (each group takes half of a step's query
+// columns), warps 12-15 the dQ drain.  Tensor memory: S^T | dP^T | dV | dK |
+// dQ, 448 of 512 columns.  Q/dO tiles stream through a 3-stage ring.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cstdint>
@@ -39,41 +40,46 @@ namespace tea {
 namespace bwd {
 
 constexpr int BN = 128;  // keys per CTA
-constexpr int THREADS = 384;
+constexpr int THREADS = 512;
 constexpr int KPANEL = 16384;  // 128 rows x 128 bytes
 constexpr float LOG2E = 1.4426950408889634f;
 
 template <int D>
 struct Cfg {
   static constexpr int BM = D == 128 ? 64 : 128;  // query rows per step
-  static constexpr int NBUF = D == 128 ? 2 : 1;   // P^T / dS^T buffers
+  static constexpr int NBUF = D == 128 ? 2 : 1;   // dS^T (and P^T) shared-memory buffers
+  // d = 128: P^T and dS^T also go to tensor memory and feed dV/dK as the A
+  // operand from TMEM (no P^T tile in shared memory).  d = 64 has no TMEM
+  // room for them and reads both from shared memory.
+  static constexpr bool TS = D == 128;
+  static constexpr int NQS = D == 128 ? 4 : 3;       // Q/dO ring stages
   static constexpr int KV_TILE = BN * D * 2;
   static constexpr int Q_TILE = BM * D * 2;
   static constexpr int Q_PANEL = BM * 128;
   static constexpr int PS_TILE = BN * BM * 2;
-  static constexpr int STAGE_BYTES = BM * D * 4;
+  static constexpr int CW = BM / 2;               // query columns per gradient warpgroup
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + KV_TILE;
   static constexpr int OFF_Q = OFF_V + KV_TILE;
-  static constexpr int OFF_DO = OFF_Q + 2 * Q_TILE;
-  static constexpr int OFF_PT = OFF_DO + 2 * Q_TILE;
-  static constexpr int OFF_DST = OFF_PT + NBUF * PS_TILE;
-  static constexpr int OFF_STG = OFF_DST + NBUF * PS_TILE;
-  static constexpr int OFF_VEC = OFF_STG + STAGE_BYTES;  // [2 bufs][lse2 | D][BM] fp32
-  static constexpr int OFF_BAR = OFF_VEC + 2 * 2 * BM * 4;
+  static constexpr int OFF_DO = OFF_Q + NQS * Q_TILE;
+  static constexpr int OFF_PT = OFF_DO + NQS * Q_TILE;
+  static constexpr int OFF_DST = OFF_PT + (TS ? 0 : NBUF * PS_TILE);
+  static constexpr int OFF_VEC = OFF_DST + NBUF * PS_TILE;  // [group][2 bufs][lse2 | D][CW] fp32
+  static constexpr int OFF_BAR = OFF_VEC + 2 * 2 * 2 * CW * 4;
   static constexpr int SMEM = OFF_BAR + 256 + 1024;
   static constexpr uint32_t T_S = 0, T_DP = BM, T_DV = 2 * BM, T_DK = 2 * BM + D, T_DQ = 2 * BM + 2 * D;
-  static_assert(T_DQ + 64 <= 512, "tensor memory budget");
+  static constexpr uint32_t T_PT = T_DQ + 64, T_DST = T_PT + BM / 2;  // bf16 pairs (TS only)
+  static_assert(T_DQ + 64 <= 512 && (!TS || T_DST + BM / 2 <= 512), "tensor memory budget");
 };
 
 struct Bars {
   uint64_t kv_full;
-  uint64_t q_full[2], q_empty[2];
+  uint64_t q_full[4], q_empty[4];  // Q/dO ring (up to 4 stages)
+  uint64_t pt_free;  // dV/dK MMAs done reading P^T / dS^T in tensor memory
   uint64_t sdp_full, s_consumed;
   uint64_t ds_full[2], ds_empty[2];
   uint64_t dq_full, dq_empty;
-  uint64_t vec_full[2];
-  uint64_t stg_full, stg_free;
+  uint64_t vec_full[2][2];  // [group][buffer]
   uint64_t dkv_full;
   uint64_t drain;
   uint32_t tmem_base;
@@ -89,11 +95,19 @@ template <int D>
 __device__ __forceinline__ Unit decode_unit(const BwdParams& P, int idx) {
   const Problem& p = P.prob;
   Unit u;
-  const int per = p.B * p.Hkv;
-  const int n = idx / per;  // key tile; early keys see the most queries: heavy first
-  const int rem = idx % per;
-  u.b = rem / p.Hkv;
-  u.kvh = rem % p.Hkv;
+  // Heads in groups of up to 8: the CTAs running at one time share the
+  // Q/dO/K/V of a few heads in L2.  Inside a group, key tiles ascend (early
+  // keys see the most queries under a causal mask: heavy first).
+  const int nkt = cdiv(p.Lk, BN);
+  const int heads = p.B * p.Hkv;
+  constexpr int HG = 8;
+  const int grp = idx / (HG * nkt);
+  const int hg = imin(HG, heads - grp * HG);
+  const int rem = idx - grp * HG * nkt;
+  const int n = rem / hg;
+  const int head = grp * HG + rem % hg;
+  u.b = head / p.Hkv;
+  u.kvh = head % p.Hkv;
   u.k0 = n * BN;
   u.G = p.Hq / p.Hkv;
   int q_lo, q_hi;
@@ -129,8 +143,8 @@ __device__ void producer(const BwdParams& P, const Unit& u, uint8_t* smem, Bars&
   }
   int issued = 0;
   for (int i = 0; i < u.n_steps; i++) {
-    const int st = i & 1;
-    if (!mbar_wait(&bars.q_empty[st], ((i >> 1) & 1) ^ 1, g, 1)) break;
+    const int st = i % C::NQS;
+    if (!mbar_wait(&bars.q_empty[st], ((i / C::NQS) & 1) ^ 1, g, 1)) break;
     int h, q0;
     step_of<D>(u, i, h, q0);
     mbar_arrive_expect_tx(&bars.q_full[st], 2 * C::Q_TILE);
@@ -144,7 +158,7 @@ __device__ void producer(const BwdParams& P, const Unit& u, uint8_t* smem, Bars&
   }
   // Let every copy this warp started land before the CTA may exit (bounded).
   mbar_wait_ignore_abort(&bars.kv_full, 0, g);
-  for (int i = imax(0, issued - 2); i < issued; i++) mbar_wait_ignore_abort(&bars.q_full[i & 1], (i >> 1) & 1, g);
+  for (int i = imax(0, issued - C::NQS); i < issued; i++) mbar_wait_ignore_abort(&bars.q_full[i % C::NQS], (i / C::NQS) & 1, g);
 }
 
 // ------------------------------------------------------------------ MMA issuer
@@ -165,8 +179,8 @@ __device__ void mma_issuer(const BwdParams& P, const Unit& u, uint8_t* smem, Bar
 
   // S^T = K Q^T and dP^T = V dO^T for step i (contraction over d).
   auto issue_sdp = [&](int i) {
-    const uint32_t qa = q_addr + (i & 1) * C::Q_TILE;
-    const uint32_t da = do_addr + (i & 1) * C::Q_TILE;
+    const uint32_t qa = q_addr + (i % C::NQS) * C::Q_TILE;
+    const uint32_t da = do_addr + (i % C::NQS) * C::Q_TILE;
 #pragma unroll
     for (int kk = 0; kk < D / 16; kk++) {
       const uint32_t oa = (kk / 4) * KPANEL + (kk % 4) * 32;
@@ -190,7 +204,7 @@ __device__ void mma_issuer(const BwdParams& P, const Unit& u, uint8_t* smem, Bar
 
   for (int i = 0; i < u.n_steps; i++) {
     if (i + 1 < u.n_steps) {
-      if (!mbar_wait(&bars.q_full[(i + 1) & 1], ((i + 1) >> 1) & 1, g, 12)) goto done;
+      if (!mbar_wait(&bars.q_full[(i + 1) % C::NQS], ((i + 1) / C::NQS) & 1, g, 12)) goto done;
       if (!mbar_wait(&bars.s_consumed, i & 1, g, 13)) goto done;
       tc_fence_after();
       issue_sdp(i + 1);
@@ -198,22 +212,35 @@ __device__ void mma_issuer(const BwdParams& P, const Unit& u, uint8_t* smem, Bar
     const int buf = i % C::NBUF;
     if (!mbar_wait(&bars.ds_full[buf], (i / C::NBUF) & 1, g, 14)) goto done;
     tc_fence_after();
-    const uint32_t qa = q_addr + (i & 1) * C::Q_TILE;
-    const uint32_t da = do_addr + (i & 1) * C::Q_TILE;
+    const uint32_t qa = q_addr + (i % C::NQS) * C::Q_TILE;
+    const uint32_t da = do_addr + (i % C::NQS) * C::Q_TILE;
     const uint32_t pa = pt_addr + buf * C::PS_TILE;
     const uint32_t sa = dst_addr + buf * C::PS_TILE;
     // dV += P^T dO and dK += dS^T Q (contraction over the BM query rows).
+    if constexpr (C::TS) {
+      // A operand from tensor memory: 16 query rows = 8 columns of bf16 pairs.
 #pragma unroll
-    for (int kk = 0; kk < BM / 16; kk++) {
-      const uint32_t oa = (kk / 4) * KPANEL + (kk % 4) * 32;
-      mma_ss(tmem + C::T_DV, sw128_desc(pa + oa, 16, 1024), sw128_desc(da + kk * 2048, C::Q_PANEL, 1024),
-             idesc_dkv, (i > 0) || (kk > 0));
-    }
+      for (int kk = 0; kk < BM / 16; kk++)
+        mma_ts(tmem + C::T_DV, tmem + C::T_PT + kk * 8, sw128_desc(da + kk * 2048, C::Q_PANEL, 1024), idesc_dkv,
+               (i > 0) || (kk > 0));
 #pragma unroll
-    for (int kk = 0; kk < BM / 16; kk++) {
-      const uint32_t oa = (kk / 4) * KPANEL + (kk % 4) * 32;
-      mma_ss(tmem + C::T_DK, sw128_desc(sa + oa, 16, 1024), sw128_desc(qa + kk * 2048, C::Q_PANEL, 1024),
-             idesc_dkv, (i > 0) || (kk > 0));
+      for (int kk = 0; kk < BM / 16; kk++)
+        mma_ts(tmem + C::T_DK, tmem + C::T_DST + kk * 8, sw128_desc(qa + kk * 2048, C::Q_PANEL, 1024), idesc_dkv,
+               (i > 0) || (kk > 0));
+      mma_commit(&bars.pt_free);
+    } else {
+#pragma unroll
+      for (int kk = 0; kk < BM / 16; kk++) {
+        const uint32_t oa = (kk / 4) * KPANEL + (kk % 4) * 32;
+        mma_ss(tmem + C::T_DV, sw128_desc(pa + oa, 16, 1024), sw128_desc(da + kk * 2048, C::Q_PANEL, 1024),
+               idesc_dkv, (i > 0) || (kk > 0));
+      }
+#pragma unroll
+      for (int kk = 0; kk < BM / 16; kk++) {
+        const uint32_t oa = (kk / 4) * KPANEL + (kk % 4) * 32;
+        mma_ss(tmem + C::T_DK, sw128_desc(sa + oa, 16, 1024), sw128_desc(qa + kk * 2048, C::Q_PANEL, 1024),
+               idesc_dkv, (i > 0) || (kk > 0));
+      }
     }
     // dQ contribution of this key tile (contraction over the 128 keys).
     if (!mbar_wait(&bars.dq_empty, (i & 1) ^ 1, g, 15)) goto done;
@@ -229,7 +256,7 @@ __device__ void mma_issuer(const BwdParams& P, const Unit& u, uint8_t* smem, Bar
     }
     mma_commit(&bars.dq_full);
     mma_commit(&bars.ds_empty[buf]);
-    mma_commit(&bars.q_empty[i & 1]);
+    mma_commit(&bars.q_empty[i % C::NQS]);
   }
 done:
   mma_commit(&bars.dkv_full);
@@ -238,20 +265,22 @@ done:
 }
 
 // ------------------------------------------------------------------ softmax gradient
-// Thread `row` owns key k0 + row (TMEM lane row) and turns its row of S^T and
-// dP^T into P^T = exp2(c*S - LSE*log2e) and dS^T = P^T * (dP^T - D), written
-// as bf16 rows of the 128-byte-swizzled shared tiles.
+// Two warpgroups share a step: group w takes query columns [w*CW, w*CW + CW).
+// Thread `row` of a group owns key k0 + row (TMEM lane row) and turns its part
+// of the S^T and dP^T rows into P^T = exp2(c*S - LSE*log2e) and
+// dS^T = P^T * (dP^T - D), written as bf16 into the 128-byte-swizzled tiles.
 template <int D>
-__device__ void grad_rows(const BwdParams& P, const Unit& u, uint8_t* smem, Bars& bars, uint32_t tmem,
+__device__ void grad_rows(const BwdParams& P, const Unit& u, uint8_t* smem, Bars& bars, uint32_t tmem, int grp,
                           const WaitGuard& g) {
   using C = Cfg<D>;
   constexpr int BM = C::BM;
+  constexpr int CW = C::CW;
   const Problem& p = P.prob;
-  const int t = threadIdx.x - 128;  // 0..127
+  const int row = threadIdx.x % 128;  // key row = TMEM lane
   const int wl = (threadIdx.x / 32) % 4;
   const int lane = threadIdx.x % 32;
-  const int row = t;
   const int key = u.k0 + row;
+  const int col0 = grp * CW;  // first query column of this group
   const uint32_t lane_base = (uint32_t)(wl * 32) << 16;
   // Queries [vis_lo, vis_hi) see this key.
   int vis_lo = 0, vis_hi = 0;
@@ -260,27 +289,46 @@ __device__ void grad_rows(const BwdParams& P, const Unit& u, uint8_t* smem, Bars
     vis_hi = p.window > 0 ? imin(p.Lq, key + p.window) : p.Lq;
   }
   const float c = P.scale_log2;
-  float* vec = reinterpret_cast<float*>(smem + C::OFF_VEC);
+  float* vec = reinterpret_cast<float*>(smem + C::OFF_VEC) + grp * (2 * 2 * CW);
   uint8_t* pt_base = smem + C::OFF_PT;
   uint8_t* dst_base = smem + C::OFF_DST;
   const uint32_t sw = (uint32_t)(row & 7);
 
+  // LSE and D of the group's queries in step i: thread row < CW fetches query
+  // q0 + col0 + row one step ahead (raw values; the load stays in flight
+  // during the previous step) and publishes them to shared memory at the
+  // step's start.  Rows past Lq: LSE = +inf (so p = 0) and D = 0.
+  auto fetch = [&](int i, float& l, float& dv) {
+    int h, q0;
+    step_of<D>(u, i, h, q0);
+    const int q = q0 + col0 + row;
+    l = INFINITY;
+    dv = 0.f;
+    if (row < CW && q < p.Lq) {
+      const size_t r = (size_t)(u.b * p.Hq + h) * p.Lq + q;
+      l = P.lse[r];
+      dv = P.dvec[r];
+    }
+  };
+  float next_l = INFINITY, next_d = 0.f;
+  if (u.n_steps > 0) fetch(0, next_l, next_d);
+
   for (int i = 0; i < u.n_steps; i++) {
     int h, q0;
     step_of<D>(u, i, h, q0);
-    // Per-query LSE (log2 units) and D for this step, shared by the group.
     const int vb = i & 1;
-    if (t < BM) {
-      const int q = q0 + t;
-      const size_t r = (size_t)(u.b * p.Hq + h) * p.Lq + q;
-      vec[(vb * 2 + 0) * BM + t] = q < p.Lq ? P.lse[r] * LOG2E : INFINITY;  // +inf: row past Lq gives p = 0
-      vec[(vb * 2 + 1) * BM + t] = q < p.Lq ? P.dvec[r] : 0.f;
+    if (row < CW) {
+      vec[(vb * 2 + 0) * CW + row] = next_l * LOG2E;
+      vec[(vb * 2 + 1) * CW + row] = next_d;
     }
-    mbar_arrive(&bars.vec_full[vb]);
-    if (!mbar_wait(&bars.vec_full[vb], (i >> 1) & 1, g, 20)) return;
-    const float* lse2 = vec + (vb * 2 + 0) * BM;
-    const float* dd = vec + (vb * 2 + 1) * BM;
-    const bool full = vis_lo <= q0 && q0 + BM <= vis_hi;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bars.vec_full[grp][vb]);
+    if (i + 1 < u.n_steps) fetch(i + 1, next_l, next_d);
+    if (!mbar_wait(&bars.vec_full[grp][vb], (i >> 1) & 1, g, 20)) return;
+    const float* lse2 = vec + (vb * 2 + 0) * CW;
+    const float* dd = vec + (vb * 2 + 1) * CW;
+    const int qc0 = q0 + col0;  // first query of this group's columns
+    const bool full = vis_lo <= qc0 && qc0 + CW <= vis_hi;
 
     if (!mbar_wait(&bars.sdp_full, i & 1, g, 21)) return;
     tc_fence_after();
@@ -288,9 +336,14 @@ __device__ void grad_rows(const BwdParams& P, const Unit& u, uint8_t* smem, Bars
     uint8_t* pt_row = pt_base + buf * C::PS_TILE + row * 128;
     uint8_t* ds_row = dst_base + buf * C::PS_TILE + row * 128;
 
-    // The BM columns go in chunks of 32 (one 32-column TMEM load each of S^T
-    // and dP^T); a chunk's four 16-byte pieces go to shared memory.
-    constexpr int NCH = BM / 32;
+    // 32 columns per chunk (one 32-column TMEM load each of S^T and dP^T);
+    // a chunk's four 16-byte pieces go to shared memory.
+    constexpr int NCH = CW / 32;
+    // Computes P^T and dS^T for 32 columns; dS^T always goes to the swizzled
+    // shared tile (operand of the dQ MMA); P^T goes there too unless the dV/dK
+    // MMAs read both from tensor memory, in which case the packed words are
+    // left in pw_all / dw_all for a TMEM store.
+    uint32_t pw_all[16], dw_all[16];
     auto emit_chunk = [&](int ch, const uint32_t* sv, const uint32_t* dpv) {
 #pragma unroll
       for (int piece = 0; piece < 4; piece++) {
@@ -301,10 +354,10 @@ __device__ void grad_rows(const BwdParams& P, const Unit& u, uint8_t* smem, Bars
 #pragma unroll
           for (int z = 0; z < 2; z++) {
             const int col = piece * 8 + e * 2 + z;  // column within the chunk
-            const int qq = ch * 32 + col;           // query within the step
+            const int qq = ch * 32 + col;           // column within the group
             float pv = ex2_approx(fmaf(__uint_as_float(sv[col]), c, -lse2[qq]));
             if (!full) {
-              const int q = q0 + qq;
+              const int q = qc0 + qq;
               if (q < vis_lo || q >= vis_hi) pv = 0.f;
             }
             pr[z] = pv;
@@ -312,37 +365,46 @@ __device__ void grad_rows(const BwdParams& P, const Unit& u, uint8_t* smem, Bars
           }
           pw[e] = pack_bf16x2(pr[0], pr[1]);
           dw[e] = pack_bf16x2(dr[0], dr[1]);
+          if constexpr (C::TS) {
+            pw_all[piece * 4 + e] = pw[e];
+            dw_all[piece * 4 + e] = dw[e];
+          }
         }
         // 16-byte piece j of the row lives in panel j / 8, at chunk (j % 8) ^ (row % 8).
-        const int j = ch * 4 + piece;
+        const int j = (col0 + ch * 32) / 8 + piece;
         const uint32_t off = (uint32_t)(j / 8) * KPANEL + (((uint32_t)(j % 8) ^ sw) << 4);
-        *reinterpret_cast<uint4*>(pt_row + off) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
+        if constexpr (!C::TS) *reinterpret_cast<uint4*>(pt_row + off) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
         *reinterpret_cast<uint4*>(ds_row + off) = make_uint4(dw[0], dw[1], dw[2], dw[3]);
       }
     };
-    if constexpr (NCH <= 2) {
-      // Small step: read all of S^T / dP^T first so the next step's MMAs can
-      // start while this one is being turned into P^T / dS^T.
-      uint32_t sv[NCH][32], dpv[NCH][32];
-#pragma unroll
-      for (int ch = 0; ch < NCH; ch++) {
-        tmem_ld32p(tmem + lane_base + C::T_S + 32 * ch, sv[ch]);
-        tmem_ld32p(tmem + lane_base + C::T_DP + 32 * ch, dpv[ch]);
-      }
+    if constexpr (NCH == 1) {
+      // Read this group's S^T / dP^T columns first so the next step's MMAs
+      // can start while they are turned into P^T / dS^T.
+      uint32_t sv[32], dpv[32];
+      tmem_ld32p(tmem + lane_base + C::T_S + col0, sv);
+      tmem_ld32p(tmem + lane_base + C::T_DP + col0, dpv);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.s_consumed);  // S^T / dP^T may be overwritten
       if (!mbar_wait(&bars.ds_empty[buf], ((i / C::NBUF) & 1) ^ 1, g, 22)) return;
-#pragma unroll
-      for (int ch = 0; ch < NCH; ch++) emit_chunk(ch, sv[ch], dpv[ch]);
+      emit_chunk(0, sv, dpv);
+      if constexpr (C::TS) {
+        // The previous step's dV/dK MMAs must be done with the TMEM copies.
+        if (!mbar_wait(&bars.pt_free, (i & 1) ^ 1, g, 24)) return;
+        tc_fence_after();
+        tmem_st16(tmem + lane_base + C::T_PT + grp * 16, pw_all);
+        tmem_st16(tmem + lane_base + C::T_DST + grp * 16, dw_all);
+        tmem_wait_st();
+        tc_fence_before();
+      }
     } else {
       if (!mbar_wait(&bars.ds_empty[buf], ((i / C::NBUF) & 1) ^ 1, g, 22)) return;
 #pragma unroll
       for (int ch = 0; ch < NCH; ch++) {
         uint32_t sv[32], dpv[32];
-        tmem_ld32p(tmem + lane_base + C::T_S + 32 * ch, sv);
-        tmem_ld32p(tmem + lane_base + C::T_DP + 32 * ch, dpv);
+        tmem_ld32p(tmem + lane_base + C::T_S + col0 + 32 * ch, sv);
+        tmem_ld32p(tmem + lane_base + C::T_DP + col0 + 32 * ch, dpv);
         tmem_wait_ld();
         if (ch == NCH - 1) {
           tc_fence_before();
@@ -357,7 +419,7 @@ __device__ void grad_rows(const BwdParams& P, const Unit& u, uint8_t* smem, Bars
     if (lane == 0) mbar_arrive(&bars.ds_full[buf]);
   }
 
-  // Epilogue: dV and scale * dK for this thread's key.
+  // Epilogue: group 0 writes dV, group 1 writes scale * dK for its key.
   const bool has = u.n_steps > 0;
   if (has) {
     if (!mbar_wait(&bars.dkv_full, 0, g, 23)) return;
@@ -365,47 +427,50 @@ __device__ void grad_rows(const BwdParams& P, const Unit& u, uint8_t* smem, Bars
   }
   const bool write = key < p.Lk;
   const size_t off = ((size_t)(u.b * p.Hkv + u.kvh) * p.Lk + key) * D;
+  uint4* out = reinterpret_cast<uint4*>(static_cast<uint16_t*>(grp ? P.dk : P.dv) + off);
+  const float f = grp ? P.scale : 1.f;
+  const uint32_t colx = grp ? C::T_DK : C::T_DV;
 #pragma unroll
-  for (int which = 0; which < 2; which++) {
-    uint4* out = reinterpret_cast<uint4*>(static_cast<uint16_t*>(which ? P.dk : P.dv) + off);
-    const float f = which ? P.scale : 1.f;
-    const uint32_t col0 = which ? C::T_DK : C::T_DV;
+  for (int q = 0; q < D / 32; q++) {
+    uint32_t o[32];
+    if (has) {
+      tmem_ld32p(tmem + lane_base + colx + 32 * q, o);
+      tmem_wait_ld();
+    } else {
 #pragma unroll
-    for (int q = 0; q < D / 32; q++) {
-      uint32_t o[32];
-      if (has) {
-        tmem_ld32p(tmem + lane_base + col0 + 32 * q, o);
-        tmem_wait_ld();
-      } else {
+      for (int e = 0; e < 32; e++) o[e] = 0u;
+    }
+    uint32_t w[16];
 #pragma unroll
-        for (int e = 0; e < 32; e++) o[e] = 0u;
-      }
-      uint32_t w[16];
+    for (int e = 0; e < 16; e++) w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * f, __uint_as_float(o[2 * e + 1]) * f);
+    if (write) {
 #pragma unroll
-      for (int e = 0; e < 16; e++) w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * f, __uint_as_float(o[2 * e + 1]) * f);
-      if (write) {
-#pragma unroll
-        for (int v = 0; v < 4; v++) out[q * 4 + v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
-      }
+      for (int v = 0; v < 4; v++) out[q * 4 + v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
     }
   }
 }
 
 // ------------------------------------------------------------------ dQ drain
-// Moves each step's 128 x 64 fp32 dQ tile from tensor memory to a linear
-// shared-memory staging tile [query][d] and adds it into the fp32
-// accumulator with one bulk reduce-add (element-wise atomic in L2).
+// Moves each step's 128 x 64 fp32 dQ tile out of tensor memory and adds it
+// into the fp32 accumulator with atomic adds (red.global: no return value;
+// element-wise atomic in L2).  At d = 128 lane t holds column t of dQ for the
+// step's 64 queries, so each warp instruction covers 32 consecutive floats.
+__device__ __forceinline__ void red_add_f32(float* p, float v) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
+}
+__device__ __forceinline__ void red_add_v4_f32(float* p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+
 template <int D>
-__device__ void dq_drain(const BwdParams& P, const Unit& u, uint8_t* smem, Bars& bars, uint32_t tmem,
-                         const WaitGuard& g) {
+__device__ void dq_drain(const BwdParams& P, const Unit& u, Bars& bars, uint32_t tmem, const WaitGuard& g) {
   using C = Cfg<D>;
-  constexpr int BM = C::BM;
   const Problem& p = P.prob;
-  const int t = threadIdx.x - 256;  // 0..127 = TMEM lane
+  const int t = threadIdx.x % 128;  // TMEM lane
   const int wl = (threadIdx.x / 32) % 4;
   const int lane = threadIdx.x % 32;
   const uint32_t lane_base = (uint32_t)(wl * 32) << 16;
-  float* stg = reinterpret_cast<float*>(smem + C::OFF_STG);
 
   for (int i = 0; i < u.n_steps; i++) {
     int h, q0;
@@ -419,33 +484,23 @@ __device__ void dq_drain(const BwdParams& P, const Unit& u, uint8_t* smem, Bars&
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(&bars.dq_empty);
-    // The previous step's bulk reduce must have finished reading the staging tile.
-    if (!mbar_wait(&bars.stg_free, (i & 1) ^ 1, g, 31)) break;
+    float* base = P.dq_acc + (size_t)(u.b * p.Hq + h) * p.Lq * D;
     if (D == 128) {
-      // Lane t holds dQ^T row t (= column d of dQ) for the BM = 64 queries.
+      // Lane t holds dQ^T row t (= column t of dQ) for the BM = 64 queries.
 #pragma unroll
-      for (int qq = 0; qq < 64; qq++) stg[qq * D + t] = __uint_as_float(r[qq]);
+      for (int qq = 0; qq < 64; qq++)
+        if (q0 + qq < p.Lq) red_add_f32(base + (size_t)(q0 + qq) * D + t, __uint_as_float(r[qq]));
     } else {
-      // Lane t holds dQ row t (query q0 + t), 64 values of d.
-      float4* dst = reinterpret_cast<float4*>(stg + t * D);
+      // Lane t holds dQ row q0 + t (64 values of d).
+      if (q0 + t < p.Lq) {
+        float* rowp = base + (size_t)(q0 + t) * D;
 #pragma unroll
-      for (int v = 0; v < 16; v++)
-        dst[v] = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]), __uint_as_float(r[4 * v + 2]),
-                             __uint_as_float(r[4 * v + 3]));
-    }
-    fence_proxy_async_smem();
-    mbar_arrive(&bars.stg_full);
-    if (t == 0) {
-      if (!mbar_wait(&bars.stg_full, i & 1, g, 32)) break;
-      const int rows = imin(BM, p.Lq - q0);
-      float* dst = P.dq_acc + ((size_t)(u.b * p.Hq + h) * p.Lq + q0) * D;
-      bulk_reduce_add_f32(dst, stg, (uint32_t)(rows * D * 4));
-      bulk_commit();
-      bulk_wait_read_all();
-      mbar_arrive(&bars.stg_free);
+        for (int v = 0; v < 16; v++)
+          red_add_v4_f32(rowp + 4 * v, __uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                         __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+      }
     }
   }
-  if (t == 0) bulk_wait_all();
 }
 
 // ------------------------------------------------------------------ kernel
@@ -463,20 +518,22 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kernel(const __grid_const
   if (threadIdx.x == 0) {
     bars.abort_flag = 0;
     mbar_init(&bars.kv_full, 1);
-    for (int s = 0; s < 2; s++) {
+    for (int s = 0; s < C::NQS; s++) {
       mbar_init(&bars.q_full[s], 1);
       mbar_init(&bars.q_empty[s], 1);
-      mbar_init(&bars.ds_full[s], 4);
+    }
+    for (int s = 0; s < 2; s++) {
+      mbar_init(&bars.ds_full[s], 8);
       mbar_init(&bars.ds_empty[s], 1);
-      mbar_init(&bars.vec_full[s], 128);
+      mbar_init(&bars.vec_full[0][s], 4);
+      mbar_init(&bars.vec_full[1][s], 4);
     }
     mbar_init(&bars.sdp_full, 1);
-    mbar_init(&bars.s_consumed, 4);
+    mbar_init(&bars.s_consumed, 8);
     mbar_init(&bars.dq_full, 1);
     mbar_init(&bars.dq_empty, 4);
-    mbar_init(&bars.stg_full, 128);
-    mbar_init(&bars.stg_free, 1);
     mbar_init(&bars.dkv_full, 1);
+    mbar_init(&bars.pt_free, 1);
     mbar_init(&bars.drain, 1);
     fence_barrier_init();
   }
@@ -489,7 +546,9 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kernel(const __grid_const
   tc_fence_after();
   const uint32_t tmem = bars.tmem_base;
 
-  // Registers: 384 x 168 at launch; load/MMA group 80, the two others 208.
+  // Registers: 512 x 128 at launch; the load/MMA group drops to 80 (enough
+  // for the issue loop without spilling), the other three take 144 each
+  // (128*80 + 384*144 = 512*128).
   if (warp < 4) {
     regs_dec<80>();
     if (warp == 0) {
@@ -497,12 +556,12 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kernel(const __grid_const
     } else if (warp == 1) {
       if (lane == 0) mma_issuer<D>(P, u, smem, bars, tmem, g);
     }
-  } else if (warp < 8) {
-    regs_inc<208>();
-    grad_rows<D>(P, u, smem, bars, tmem, g);
+  } else if (warp < 12) {
+    regs_inc<144>();
+    grad_rows<D>(P, u, smem, bars, tmem, (warp - 4) / 4, g);
   } else {
-    regs_inc<208>();
-    dq_drain<D>(P, u, smem, bars, tmem, g);
+    regs_inc<144>();
+    dq_drain<D>(P, u, bars, tmem, g);
   }
   tc_fence_before();
   __syncthreads();

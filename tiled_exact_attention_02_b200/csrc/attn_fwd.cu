@@ -84,25 +84,31 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& P, int idx) {
   Unit u;
   const int G = p.Hq / p.Hkv;
   const int nqt = cdiv(p.Lq, BM);
+  // Work is grouped by heads (up to 8 head units per group, so the CTAs
+  // running at one time share the K/V of a few heads in L2); inside a group
+  // the query tiles go from last to first (late rows see the most keys under
+  // a causal mask: heavy first).
+  const int nh = P.pair_heads ? p.B * (p.Hq / 2) : p.B * p.Hq;  // head units
+  const int nq = P.pair_heads ? nqt : cdiv(nqt, 2);              // query units per head unit
+  constexpr int HG = 8;
+  const int grp = idx / (HG * nq);
+  const int hg = imin(HG, nh - grp * HG);
+  const int rem = idx - grp * HG * nq;
+  const int qi = nq - 1 - rem / hg;
+  const int hu = grp * HG + rem % hg;
   if (P.pair_heads) {
-    // Two heads of one GQA group, same query rows.  Heavy (late) rows first.
-    const int per_q = p.B * (p.Hq / 2);
-    const int qi = nqt - 1 - idx / per_q;
-    const int rem = idx % per_q;
-    u.b = rem / (p.Hq / 2);
-    const int hp = rem % (p.Hq / 2);
+    // Two heads of one GQA group, same query rows.
+    u.b = hu / (p.Hq / 2);
+    const int hp = hu % (p.Hq / 2);
     u.head[0] = 2 * hp;
     u.head[1] = 2 * hp + 1;
     u.q0[0] = u.q0[1] = qi * BM;
   } else {
-    const int nqp = cdiv(nqt, 2);
-    const int per_q = p.B * p.Hq;
-    const int qp = nqp - 1 - idx / per_q;
-    const int rem = idx % per_q;
-    u.b = rem / p.Hq;
-    u.head[0] = u.head[1] = rem % p.Hq;
-    u.q0[0] = qp * 2 * BM;
-    u.q0[1] = qp * 2 * BM + BM;
+    // Two consecutive row tiles of one head.
+    u.b = hu / p.Hq;
+    u.head[0] = u.head[1] = hu % p.Hq;
+    u.q0[0] = qi * 2 * BM;
+    u.q0[1] = qi * 2 * BM + BM;
   }
   u.kvh = u.head[0] / G;
   u.ulo = 1 << 30;
@@ -395,16 +401,16 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_kernel(const __grid_const
   const uint32_t tmem = bars.tmem_base;
 
   // Registers: launched at 168 per thread (384 x 168); the load/MMA group
-  // gives up to 80, each softmax group takes 208 (128*80 + 256*208 <= 384*168).
+  // drops to 112, each softmax group takes 192 (128*112 + 256*192 <= 384*168).
   if (warp < 4) {
-    regs_dec<80>();
+    regs_dec<112>();
     if (warp == 0) {
       if (lane == 0) producer<D>(P, u, smem, bars, g);
     } else if (warp == 1) {
       if (lane == 0) mma_issuer<D>(P, u, smem, bars, tmem, g);
     }
   } else {
-    regs_inc<208>();
+    regs_inc<192>();
     softmax_slot<D>(P, u, (warp - 4) / 4, bars, tmem, g);
   }
   tc_fence_before();
