@@ -23,7 +23,7 @@
 // so that one thread per key turns a row of S^T into P^T and dS^T, and the
 // bf16 P^T and dS^T, written once to shared memory, serve both as the K-major
 // A operand of dV/dK and as the MN-major operand of dQ.
-// Warp roles (512 threads): warp 0 TMA, warp 1 MMA issuer, warps 4-7 and
+// Warp roles (512 threads): warp 0 TMA, warps 1 and 2 MMA issuers, warps 4-7 and
 // 8-11 the per-key softmax gradient (each group takes half of a step's query
 // columns), warps 12-15 the dQ drain.  Tensor memory: S^T | dP^T | dV | dK |
 // dQ, 448 of 512 columns.  Q/dO tiles stream through a 3-stage ring.
@@ -72,16 +72,25 @@ struct Cfg {
   static_assert(T_DQ + 64 <= 512 && (!TS || T_DST + BM / 2 <= 512), "tensor memory budget");
 };
 
+// Barriers.  The MMA issuer pays for every wait and commit with tensor-core
+// idle time (its issue queue is shallow), so each of its waits covers
+// everything the next MMA group needs:
+//   sq_ready[stage]  Q/dO of a step landed (TMA, 1 arrival + bytes) and the
+//                    previous step's S^T/dP^T were read out (8 gradient warps)
+//   grad_ready[2]    P^T/dS^T of a step written (8 gradient warps) and the
+//                    previous step's dQ read out of TMEM (4 drain warps)
+//   sdp_full         S^T/dP^T of a step complete
+//   step_done        all MMAs of a step complete (dQ readable; P^T/dS^T and
+//                    the dS^T tile may be overwritten)
+//   q_empty[stage]   the step's Q/dO stage may be reloaded
 struct Bars {
   uint64_t kv_full;
-  uint64_t q_full[4], q_empty[4];  // Q/dO ring (up to 4 stages)
-  uint64_t pt_free;  // dV/dK MMAs done reading P^T / dS^T in tensor memory
-  uint64_t sdp_full, s_consumed;
-  uint64_t ds_full[2], ds_empty[2];
-  uint64_t dq_full, dq_empty;
+  uint64_t sq_ready[4], q_empty[4];  // Q/dO ring (up to 4 stages)
+  uint64_t grad_ready[2];
+  uint64_t sdp_full, step_done;
   uint64_t vec_full[2][2];  // [group][buffer]
   uint64_t dkv_full;
-  uint64_t drain;
+  uint64_t drain[2];
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -147,22 +156,31 @@ __device__ void producer(const BwdParams& P, const Unit& u, uint8_t* smem, Bars&
     if (!mbar_wait(&bars.q_empty[st], ((i / C::NQS) & 1) ^ 1, g, 1)) break;
     int h, q0;
     step_of<D>(u, i, h, q0);
-    mbar_arrive_expect_tx(&bars.q_full[st], 2 * C::Q_TILE);
+    mbar_arrive_expect_tx(&bars.sq_ready[st], 2 * C::Q_TILE);
     for (int pnl = 0; pnl < D / 64; pnl++) {
-      tma_load_3d(smem + C::OFF_Q + st * C::Q_TILE + pnl * C::Q_PANEL, &P.tm_q, &bars.q_full[st], pnl * 64, q0,
+      tma_load_3d(smem + C::OFF_Q + st * C::Q_TILE + pnl * C::Q_PANEL, &P.tm_q, &bars.sq_ready[st], pnl * 64, q0,
                   u.b * p.Hq + h);
-      tma_load_3d(smem + C::OFF_DO + st * C::Q_TILE + pnl * C::Q_PANEL, &P.tm_do, &bars.q_full[st], pnl * 64, q0,
+      tma_load_3d(smem + C::OFF_DO + st * C::Q_TILE + pnl * C::Q_PANEL, &P.tm_do, &bars.sq_ready[st], pnl * 64, q0,
                   u.b * p.Hq + h);
     }
     issued = i + 1;
   }
-  // Let every copy this warp started land before the CTA may exit (bounded).
+  // Let every copy this warp started land before the CTA may exit.  K/V have
+  // their own barrier; the Q/dO copies share sq_ready with the gradient
+  // warps' arrivals, so after an abort give them a fixed 50 us to land.
   mbar_wait_ignore_abort(&bars.kv_full, 0, g);
-  for (int i = imax(0, issued - C::NQS); i < issued; i++) mbar_wait_ignore_abort(&bars.q_full[i % C::NQS], (i / C::NQS) & 1, g);
+  if (*g.abort_flag && issued > 0) {
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 50000) {
+    }
+  }
 }
 
 // ------------------------------------------------------------------ MMA issuer
-template <int D>
+// Two issuing threads keep the tensor core fed: each mbarrier wait costs the
+// issuing thread about as long as an MMA, and the tensor core's issue queue is
+// shallow, so while one issuer waits the other one issues.
+template <int D, int ROLE>
 __device__ void mma_issuer(const BwdParams& P, const Unit& u, uint8_t* smem, Bars& bars, uint32_t tmem,
                            const WaitGuard& g) {
   using C = Cfg<D>;
@@ -170,98 +188,107 @@ __device__ void mma_issuer(const BwdParams& P, const Unit& u, uint8_t* smem, Bar
   const uint32_t idesc_s = idesc_bf16_f32(128, BM, 0, 0);
   const uint32_t idesc_dkv = idesc_bf16_f32(128, D, 0, 1);
   const uint32_t idesc_dq = idesc_bf16_f32(128, 64, 1, 1);
+  // Shared-memory descriptors are built once; an operand slice at byte offset
+  // `off` from a tile's start is that tile's descriptor plus off / 16 (the
+  // start-address field; no carry since shared addresses are < 256 KB).
   const uint32_t k_addr = smem_u32(smem + C::OFF_K);
-  const uint32_t v_addr = smem_u32(smem + C::OFF_V);
-  const uint32_t q_addr = smem_u32(smem + C::OFF_Q);
-  const uint32_t do_addr = smem_u32(smem + C::OFF_DO);
-  const uint32_t pt_addr = smem_u32(smem + C::OFF_PT);
-  const uint32_t dst_addr = smem_u32(smem + C::OFF_DST);
+  const uint64_t k_kmaj = sw128_desc(k_addr, 16, 1024);                    // K as K-major A (S^T)
+  const uint64_t v_kmaj = sw128_desc(smem_u32(smem + C::OFF_V), 16, 1024); // V as K-major A (dP^T)
+  const uint64_t k_mn = sw128_desc(k_addr, KPANEL, 1024);                  // K as MN-major operand (dQ)
+  const uint64_t q_kmaj = sw128_desc(smem_u32(smem + C::OFF_Q), 16, 1024);
+  const uint64_t do_kmaj = sw128_desc(smem_u32(smem + C::OFF_DO), 16, 1024);
+  const uint64_t q_mn = sw128_desc(smem_u32(smem + C::OFF_Q), C::Q_PANEL, 1024);
+  const uint64_t do_mn = sw128_desc(smem_u32(smem + C::OFF_DO), C::Q_PANEL, 1024);
+  const uint64_t pt_kmaj = sw128_desc(smem_u32(smem + C::OFF_PT), 16, 1024);
+  const uint64_t ds_kmaj = sw128_desc(smem_u32(smem + C::OFF_DST), 16, 1024);
+  const uint64_t ds_mn = sw128_desc(smem_u32(smem + C::OFF_DST), KPANEL, 1024);
+  auto adv = [](uint64_t d, uint32_t bytes) { return d + (uint64_t)(bytes >> 4); };
 
   // S^T = K Q^T and dP^T = V dO^T for step i (contraction over d).
   auto issue_sdp = [&](int i) {
-    const uint32_t qa = q_addr + (i % C::NQS) * C::Q_TILE;
-    const uint32_t da = do_addr + (i % C::NQS) * C::Q_TILE;
+    const uint32_t st_off = (uint32_t)(i % C::NQS) * C::Q_TILE;
+    const uint64_t qd = adv(q_kmaj, st_off), dd = adv(do_kmaj, st_off);
 #pragma unroll
     for (int kk = 0; kk < D / 16; kk++) {
       const uint32_t oa = (kk / 4) * KPANEL + (kk % 4) * 32;
       const uint32_t ob = (kk / 4) * C::Q_PANEL + (kk % 4) * 32;
-      mma_ss(tmem + C::T_S, sw128_desc(k_addr + oa, 16, 1024), sw128_desc(qa + ob, 16, 1024), idesc_s, kk > 0);
+      mma_ss(tmem + C::T_S, adv(k_kmaj, oa), adv(qd, ob), idesc_s, kk > 0);
     }
 #pragma unroll
     for (int kk = 0; kk < D / 16; kk++) {
       const uint32_t oa = (kk / 4) * KPANEL + (kk % 4) * 32;
       const uint32_t ob = (kk / 4) * C::Q_PANEL + (kk % 4) * 32;
-      mma_ss(tmem + C::T_DP, sw128_desc(v_addr + oa, 16, 1024), sw128_desc(da + ob, 16, 1024), idesc_s, kk > 0);
+      mma_ss(tmem + C::T_DP, adv(v_kmaj, oa), adv(dd, ob), idesc_s, kk > 0);
     }
     mma_commit(&bars.sdp_full);
   };
 
-  if (u.n_steps == 0) goto done;
-  if (!mbar_wait(&bars.kv_full, 0, g, 10)) goto done;
-  if (!mbar_wait(&bars.q_full[0], 0, g, 11)) goto done;
-  tc_fence_after();
-  issue_sdp(0);
-
-  for (int i = 0; i < u.n_steps; i++) {
-    if (i + 1 < u.n_steps) {
-      if (!mbar_wait(&bars.q_full[(i + 1) % C::NQS], ((i + 1) / C::NQS) & 1, g, 12)) goto done;
-      if (!mbar_wait(&bars.s_consumed, i & 1, g, 13)) goto done;
+  if (ROLE == 0) {
+    // Issuer A: S^T and dP^T of every step.
+    if (u.n_steps == 0) goto done;
+    if (!mbar_wait(&bars.kv_full, 0, g, 10)) goto done;
+    for (int i = 0; i < u.n_steps; i++) {
+      // Q/dO of step i landed and S^T/dP^T of step i-1 read out.
+      if (!mbar_wait(&bars.sq_ready[i % C::NQS], (i / C::NQS) & 1, g, 12)) goto done;
       tc_fence_after();
-      issue_sdp(i + 1);
+      issue_sdp(i);
     }
-    const int buf = i % C::NBUF;
-    if (!mbar_wait(&bars.ds_full[buf], (i / C::NBUF) & 1, g, 14)) goto done;
-    tc_fence_after();
-    const uint32_t qa = q_addr + (i % C::NQS) * C::Q_TILE;
-    const uint32_t da = do_addr + (i % C::NQS) * C::Q_TILE;
-    const uint32_t pa = pt_addr + buf * C::PS_TILE;
-    const uint32_t sa = dst_addr + buf * C::PS_TILE;
-    // dV += P^T dO and dK += dS^T Q (contraction over the BM query rows).
-    if constexpr (C::TS) {
-      // A operand from tensor memory: 16 query rows = 8 columns of bf16 pairs.
+  } else {
+    // Issuer B: dV, dK and dQ of every step.
+    if (u.n_steps == 0) goto done;
+    if (!mbar_wait(&bars.kv_full, 0, g, 10)) goto done;
+    for (int i = 0; i < u.n_steps; i++) {
+      // P^T/dS^T of step i written and dQ of step i-1 read out of TMEM.
+      if (!mbar_wait(&bars.grad_ready[i & 1], (i >> 1) & 1, g, 14)) goto done;
+      tc_fence_after();
+      const int buf = i % C::NBUF;
+      const uint32_t st_off = (uint32_t)(i % C::NQS) * C::Q_TILE;
+      const uint32_t ps_off = (uint32_t)buf * C::PS_TILE;
+      const uint64_t qmn = adv(q_mn, st_off), domn = adv(do_mn, st_off);
+      const uint32_t acc0 = i > 0;
+      // dV += P^T dO and dK += dS^T Q (contraction over the BM query rows).
+      if constexpr (C::TS) {
+        // A operand from tensor memory: 16 query rows = 8 columns of bf16 pairs.
 #pragma unroll
-      for (int kk = 0; kk < BM / 16; kk++)
-        mma_ts(tmem + C::T_DV, tmem + C::T_PT + kk * 8, sw128_desc(da + kk * 2048, C::Q_PANEL, 1024), idesc_dkv,
-               (i > 0) || (kk > 0));
+        for (int kk = 0; kk < BM / 16; kk++)
+          mma_ts(tmem + C::T_DV, tmem + C::T_PT + kk * 8, adv(domn, kk * 2048), idesc_dkv, kk > 0 ? 1u : acc0);
 #pragma unroll
-      for (int kk = 0; kk < BM / 16; kk++)
-        mma_ts(tmem + C::T_DK, tmem + C::T_DST + kk * 8, sw128_desc(qa + kk * 2048, C::Q_PANEL, 1024), idesc_dkv,
-               (i > 0) || (kk > 0));
-      mma_commit(&bars.pt_free);
-    } else {
+        for (int kk = 0; kk < BM / 16; kk++)
+          mma_ts(tmem + C::T_DK, tmem + C::T_DST + kk * 8, adv(qmn, kk * 2048), idesc_dkv, kk > 0 ? 1u : acc0);
+      } else {
+        const uint64_t pd = adv(pt_kmaj, ps_off), sd = adv(ds_kmaj, ps_off);
 #pragma unroll
-      for (int kk = 0; kk < BM / 16; kk++) {
-        const uint32_t oa = (kk / 4) * KPANEL + (kk % 4) * 32;
-        mma_ss(tmem + C::T_DV, sw128_desc(pa + oa, 16, 1024), sw128_desc(da + kk * 2048, C::Q_PANEL, 1024),
-               idesc_dkv, (i > 0) || (kk > 0));
+        for (int kk = 0; kk < BM / 16; kk++) {
+          const uint32_t oa = (kk / 4) * KPANEL + (kk % 4) * 32;
+          mma_ss(tmem + C::T_DV, adv(pd, oa), adv(domn, kk * 2048), idesc_dkv, kk > 0 ? 1u : acc0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < BM / 16; kk++) {
+          const uint32_t oa = (kk / 4) * KPANEL + (kk % 4) * 32;
+          mma_ss(tmem + C::T_DK, adv(sd, oa), adv(qmn, kk * 2048), idesc_dkv, kk > 0 ? 1u : acc0);
+        }
       }
+      // dQ contribution of this key tile (contraction over the 128 keys).
+      const uint64_t dsmn = adv(ds_mn, ps_off);
 #pragma unroll
-      for (int kk = 0; kk < BM / 16; kk++) {
-        const uint32_t oa = (kk / 4) * KPANEL + (kk % 4) * 32;
-        mma_ss(tmem + C::T_DK, sw128_desc(sa + oa, 16, 1024), sw128_desc(qa + kk * 2048, C::Q_PANEL, 1024),
-               idesc_dkv, (i > 0) || (kk > 0));
+      for (int kk = 0; kk < BN / 16; kk++) {
+        if (D == 128)  // dQ^T = K^T dS^T: A = K (M = d), B = dS^T (N = query rows)
+          mma_ss(tmem + C::T_DQ, adv(k_mn, kk * 2048), adv(dsmn, kk * 2048), idesc_dq, kk > 0);
+        else  // dQ = dS K: A = dS^T viewed MN-major (M = query rows), B = K (N = d)
+          mma_ss(tmem + C::T_DQ, adv(dsmn, kk * 2048), adv(k_mn, kk * 2048), idesc_dq, kk > 0);
       }
+      // Everything of step i issued by B (and, causally, S^T/dP^T of step i
+      // by A, which the gradient warps had to read first) is done when these
+      // fire.
+      mma_commit(&bars.step_done);
+      mma_commit(&bars.q_empty[i % C::NQS]);
     }
-    // dQ contribution of this key tile (contraction over the 128 keys).
-    if (!mbar_wait(&bars.dq_empty, (i & 1) ^ 1, g, 15)) goto done;
-    tc_fence_after();
-#pragma unroll
-    for (int kk = 0; kk < BN / 16; kk++) {
-      if (D == 128)  // dQ^T = K^T dS^T: A = K (M = d), B = dS^T (N = query rows)
-        mma_ss(tmem + C::T_DQ, sw128_desc(k_addr + kk * 2048, KPANEL, 1024), sw128_desc(sa + kk * 2048, KPANEL, 1024),
-               idesc_dq, kk > 0);
-      else  // dQ = dS K: A = dS^T viewed MN-major (M = query rows), B = K (N = d)
-        mma_ss(tmem + C::T_DQ, sw128_desc(sa + kk * 2048, KPANEL, 1024), sw128_desc(k_addr + kk * 2048, KPANEL, 1024),
-               idesc_dq, kk > 0);
-    }
-    mma_commit(&bars.dq_full);
-    mma_commit(&bars.ds_empty[buf]);
-    mma_commit(&bars.q_empty[i % C::NQS]);
   }
 done:
-  mma_commit(&bars.dkv_full);
-  mma_commit(&bars.drain);
-  mbar_wait_ignore_abort(&bars.drain, 0, g);
+  if (ROLE == 1) mma_commit(&bars.dkv_full);
+  // Drain: every MMA this thread issued has completed (each issuer has its own barrier).
+  mma_commit(&bars.drain[ROLE]);
+  mbar_wait_ignore_abort(&bars.drain[ROLE], 0, g);
 }
 
 // ------------------------------------------------------------------ softmax gradient
@@ -312,6 +339,9 @@ __device__ void grad_rows(const BwdParams& P, const Unit& u, uint8_t* smem, Bars
   };
   float next_l = INFINITY, next_d = 0.f;
   if (u.n_steps > 0) fetch(0, next_l, next_d);
+  // Step 0 has no earlier S^T/dP^T to read out.
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&bars.sq_ready[0]);
 
   for (int i = 0; i < u.n_steps; i++) {
     int h, q0;
@@ -336,87 +366,71 @@ __device__ void grad_rows(const BwdParams& P, const Unit& u, uint8_t* smem, Bars
     uint8_t* pt_row = pt_base + buf * C::PS_TILE + row * 128;
     uint8_t* ds_row = dst_base + buf * C::PS_TILE + row * 128;
 
-    // 32 columns per chunk (one 32-column TMEM load each of S^T and dP^T);
-    // a chunk's four 16-byte pieces go to shared memory.
+    // The group's CW columns are read from TMEM 32 at a time (S^T and dP^T);
+    // P^T and dS^T are kept as packed bf16 pairs until the previous step's
+    // MMAs have released their destinations.
     constexpr int NCH = CW / 32;
-    // Computes P^T and dS^T for 32 columns; dS^T always goes to the swizzled
-    // shared tile (operand of the dQ MMA); P^T goes there too unless the dV/dK
-    // MMAs read both from tensor memory, in which case the packed words are
-    // left in pw_all / dw_all for a TMEM store.
-    uint32_t pw_all[16], dw_all[16];
-    auto emit_chunk = [&](int ch, const uint32_t* sv, const uint32_t* dpv) {
+    uint32_t pw_all[CW / 2], dw_all[CW / 2];
+    auto calc_chunk = [&](int ch, const uint32_t* sv, const uint32_t* dpv) {
 #pragma unroll
-      for (int piece = 0; piece < 4; piece++) {
-        uint32_t pw[4], dw[4];
+      for (int e = 0; e < 16; e++) {
+        float pr[2], dr[2];
 #pragma unroll
-        for (int e = 0; e < 4; e++) {
-          float pr[2], dr[2];
-#pragma unroll
-          for (int z = 0; z < 2; z++) {
-            const int col = piece * 8 + e * 2 + z;  // column within the chunk
-            const int qq = ch * 32 + col;           // column within the group
-            float pv = ex2_approx(fmaf(__uint_as_float(sv[col]), c, -lse2[qq]));
-            if (!full) {
-              const int q = qc0 + qq;
-              if (q < vis_lo || q >= vis_hi) pv = 0.f;
-            }
-            pr[z] = pv;
-            dr[z] = pv * (__uint_as_float(dpv[col]) - dd[qq]);
+        for (int z = 0; z < 2; z++) {
+          const int col = e * 2 + z;     // column within the chunk
+          const int qq = ch * 32 + col;  // column within the group
+          float pv = ex2_approx(fmaf(__uint_as_float(sv[col]), c, -lse2[qq]));
+          if (!full) {
+            const int q = qc0 + qq;
+            if (q < vis_lo || q >= vis_hi) pv = 0.f;
           }
-          pw[e] = pack_bf16x2(pr[0], pr[1]);
-          dw[e] = pack_bf16x2(dr[0], dr[1]);
-          if constexpr (C::TS) {
-            pw_all[piece * 4 + e] = pw[e];
-            dw_all[piece * 4 + e] = dw[e];
-          }
+          pr[z] = pv;
+          dr[z] = pv * (__uint_as_float(dpv[col]) - dd[qq]);
         }
-        // 16-byte piece j of the row lives in panel j / 8, at chunk (j % 8) ^ (row % 8).
-        const int j = (col0 + ch * 32) / 8 + piece;
-        const uint32_t off = (uint32_t)(j / 8) * KPANEL + (((uint32_t)(j % 8) ^ sw) << 4);
-        if constexpr (!C::TS) *reinterpret_cast<uint4*>(pt_row + off) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
-        *reinterpret_cast<uint4*>(ds_row + off) = make_uint4(dw[0], dw[1], dw[2], dw[3]);
+        pw_all[ch * 16 + e] = pack_bf16x2(pr[0], pr[1]);
+        dw_all[ch * 16 + e] = pack_bf16x2(dr[0], dr[1]);
       }
     };
-    if constexpr (NCH == 1) {
-      // Read this group's S^T / dP^T columns first so the next step's MMAs
-      // can start while they are turned into P^T / dS^T.
-      uint32_t sv[32], dpv[32];
-      tmem_ld32p(tmem + lane_base + C::T_S + col0, sv);
-      tmem_ld32p(tmem + lane_base + C::T_DP + col0, dpv);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.s_consumed);  // S^T / dP^T may be overwritten
-      if (!mbar_wait(&bars.ds_empty[buf], ((i / C::NBUF) & 1) ^ 1, g, 22)) return;
-      emit_chunk(0, sv, dpv);
-      if constexpr (C::TS) {
-        // The previous step's dV/dK MMAs must be done with the TMEM copies.
-        if (!mbar_wait(&bars.pt_free, (i & 1) ^ 1, g, 24)) return;
-        tc_fence_after();
-        tmem_st16(tmem + lane_base + C::T_PT + grp * 16, pw_all);
-        tmem_st16(tmem + lane_base + C::T_DST + grp * 16, dw_all);
-        tmem_wait_st();
-        tc_fence_before();
-      }
-    } else {
-      if (!mbar_wait(&bars.ds_empty[buf], ((i / C::NBUF) & 1) ^ 1, g, 22)) return;
 #pragma unroll
-      for (int ch = 0; ch < NCH; ch++) {
-        uint32_t sv[32], dpv[32];
-        tmem_ld32p(tmem + lane_base + C::T_S + col0 + 32 * ch, sv);
-        tmem_ld32p(tmem + lane_base + C::T_DP + col0 + 32 * ch, dpv);
-        tmem_wait_ld();
-        if (ch == NCH - 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bars.s_consumed);
-        }
-        emit_chunk(ch, sv, dpv);
+    for (int ch = 0; ch < NCH; ch++) {
+      uint32_t sv[32], dpv[32];
+      tmem_ld32p(tmem + lane_base + C::T_S + col0 + 32 * ch, sv);
+      tmem_ld32p(tmem + lane_base + C::T_DP + col0 + 32 * ch, dpv);
+      tmem_wait_ld();
+      if (ch == NCH - 1) {
+        // S^T / dP^T of this step are read: the next step's MMAs may overwrite them.
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.sq_ready[(i + 1) % C::NQS]);
       }
+      calc_chunk(ch, sv, dpv);
+    }
+    // The previous step's MMAs must be done with the TMEM P^T/dS^T and with
+    // this dS^T (and P^T) shared-memory buffer.
+    if (i > 0) {
+      if (!mbar_wait(&bars.step_done, (i - 1) & 1, g, 22)) return;
+      tc_fence_after();
+    }
+#pragma unroll
+    for (int j4 = 0; j4 < CW / 8; j4++) {
+      // 16-byte piece j of the row lives in panel j / 8, at chunk (j % 8) ^ (row % 8).
+      const int j = col0 / 8 + j4;
+      const uint32_t off = (uint32_t)(j / 8) * KPANEL + (((uint32_t)(j % 8) ^ sw) << 4);
+      if constexpr (!C::TS)
+        *reinterpret_cast<uint4*>(pt_row + off) =
+            make_uint4(pw_all[4 * j4], pw_all[4 * j4 + 1], pw_all[4 * j4 + 2], pw_all[4 * j4 + 3]);
+      *reinterpret_cast<uint4*>(ds_row + off) =
+          make_uint4(dw_all[4 * j4], dw_all[4 * j4 + 1], dw_all[4 * j4 + 2], dw_all[4 * j4 + 3]);
+    }
+    if constexpr (C::TS) {
+      tmem_st16(tmem + lane_base + C::T_PT + grp * 16, *reinterpret_cast<const uint32_t(*)[16]>(pw_all));
+      tmem_st16(tmem + lane_base + C::T_DST + grp * 16, *reinterpret_cast<const uint32_t(*)[16]>(dw_all));
+      tmem_wait_st();
     }
     fence_proxy_async_smem();  // generic-proxy stores -> tensor-core reads
+    tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive(&bars.ds_full[buf]);
+    if (lane == 0) mbar_arrive(&bars.grad_ready[i & 1]);
   }
 
   // Epilogue: group 0 writes dV, group 1 writes scale * dK for its key.
@@ -472,10 +486,12 @@ __device__ void dq_drain(const BwdParams& P, const Unit& u, Bars& bars, uint32_t
   const int lane = threadIdx.x % 32;
   const uint32_t lane_base = (uint32_t)(wl * 32) << 16;
 
+  // Step 0 has no earlier dQ to read out.
+  if (lane == 0) mbar_arrive(&bars.grad_ready[0]);
   for (int i = 0; i < u.n_steps; i++) {
     int h, q0;
     step_of<D>(u, i, h, q0);
-    if (!mbar_wait(&bars.dq_full, i & 1, g, 30)) break;
+    if (!mbar_wait(&bars.step_done, i & 1, g, 30)) break;
     tc_fence_after();
     uint32_t r[64];
     tmem_ld32p(tmem + lane_base + C::T_DQ, r);
@@ -483,7 +499,7 @@ __device__ void dq_drain(const BwdParams& P, const Unit& u, Bars& bars, uint32_t
     tmem_wait_ld();
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive(&bars.dq_empty);
+    if (lane == 0) mbar_arrive(&bars.grad_ready[(i + 1) & 1]);  // dQ TMEM free for step i+1
     float* base = P.dq_acc + (size_t)(u.b * p.Hq + h) * p.Lq * D;
     if (D == 128) {
       // Lane t holds dQ^T row t (= column t of dQ) for the BM = 64 queries.
@@ -504,6 +520,11 @@ __device__ void dq_drain(const BwdParams& P, const Unit& u, Bars& bars, uint32_t
 }
 
 // ------------------------------------------------------------------ kernel
+// Per-thread register budgets after setmaxnreg (launch: 512 x 128):
+// load/MMA group, gradient groups, dQ drain; 128*RM + 256*RG + 128*RQ <= 65536.
+constexpr int RM = 104, RG = 152, RQ = 104;
+static_assert(128 * RM + 256 * RG + 128 * RQ <= 512 * 128, "register budget");
+
 template <int D>
 __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kernel(const __grid_constant__ BwdParams P) {
   using C = Cfg<D>;
@@ -519,22 +540,19 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kernel(const __grid_const
     bars.abort_flag = 0;
     mbar_init(&bars.kv_full, 1);
     for (int s = 0; s < C::NQS; s++) {
-      mbar_init(&bars.q_full[s], 1);
+      mbar_init(&bars.sq_ready[s], 1 + 8);  // producer + 8 gradient warps
       mbar_init(&bars.q_empty[s], 1);
     }
     for (int s = 0; s < 2; s++) {
-      mbar_init(&bars.ds_full[s], 8);
-      mbar_init(&bars.ds_empty[s], 1);
+      mbar_init(&bars.grad_ready[s], 8 + 4);  // 8 gradient warps + 4 drain warps
       mbar_init(&bars.vec_full[0][s], 4);
       mbar_init(&bars.vec_full[1][s], 4);
     }
     mbar_init(&bars.sdp_full, 1);
-    mbar_init(&bars.s_consumed, 8);
-    mbar_init(&bars.dq_full, 1);
-    mbar_init(&bars.dq_empty, 4);
+    mbar_init(&bars.step_done, 1);
     mbar_init(&bars.dkv_full, 1);
-    mbar_init(&bars.pt_free, 1);
-    mbar_init(&bars.drain, 1);
+    mbar_init(&bars.drain[0], 1);
+    mbar_init(&bars.drain[1], 1);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -546,21 +564,23 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kernel(const __grid_const
   tc_fence_after();
   const uint32_t tmem = bars.tmem_base;
 
-  // Registers: 512 x 128 at launch; the load/MMA group drops to 80 (enough
-  // for the issue loop without spilling), the other three take 144 each
-  // (128*80 + 384*144 = 512*128).
+  // Registers: 512 x 128 at launch; the load/MMA group keeps 120 (the issue
+  // loop holds a dozen 64-bit descriptors), the other three keep 128
+  // (128*120 + 384*128 <= 512*128).
   if (warp < 4) {
-    regs_dec<80>();
+    regs_set<RM, 128>();
     if (warp == 0) {
       if (lane == 0) producer<D>(P, u, smem, bars, g);
     } else if (warp == 1) {
-      if (lane == 0) mma_issuer<D>(P, u, smem, bars, tmem, g);
+      if (lane == 0) mma_issuer<D, 0>(P, u, smem, bars, tmem, g);
+    } else if (warp == 2) {
+      if (lane == 0) mma_issuer<D, 1>(P, u, smem, bars, tmem, g);
     }
   } else if (warp < 12) {
-    regs_inc<144>();
+    regs_set<RG, 128>();
     grad_rows<D>(P, u, smem, bars, tmem, (warp - 4) / 4, g);
   } else {
-    regs_inc<144>();
+    regs_set<RQ, 128>();
     dq_drain<D>(P, u, bars, tmem, g);
   }
   tc_fence_before();

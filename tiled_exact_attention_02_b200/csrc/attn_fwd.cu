@@ -176,25 +176,28 @@ __device__ void mma_issuer(const FwdParams& P, const Unit& u, uint8_t* smem, Bar
   using C = Cfg<D>;
   const uint32_t idesc_qk = idesc_bf16_f32(BM, BN, 0, 0);
   const uint32_t idesc_pv = idesc_bf16_f32(BM, D, 0, 1);
-  const uint32_t q_addr = smem_u32(smem + C::OFF_Q);
-  const uint32_t kv_addr = smem_u32(smem + C::OFF_KV);
+  // Descriptors are built once; a slice at byte offset `off` inside a tile is
+  // the tile's descriptor plus off / 16 (start-address field, no carry).
+  const uint64_t q_kmaj = sw128_desc(smem_u32(smem + C::OFF_Q), 16, 1024);
+  const uint64_t kv_kmaj = sw128_desc(smem_u32(smem + C::OFF_KV), 16, 1024);
+  const uint64_t kv_mn = sw128_desc(smem_u32(smem + C::OFF_KV), PANEL, 1024);
+  auto adv = [](uint64_t d, uint32_t bytes) { return d + (uint64_t)(bytes >> 4); };
   if (u.uhi <= u.ulo) return;
 
   auto stage_of = [&](int j, int which) { return (2 * (j - u.ulo) + which) % C::NST; };
   auto phase_of = [&](int j, int which) { return (uint32_t)(((2 * (j - u.ulo) + which) / C::NST) & 1); };
 
   auto issue_s = [&](int s, int j) {
-    const uint32_t qa = q_addr + s * C::TILE;
-    const uint32_t ka = kv_addr + stage_of(j, 0) * C::TILE;
+    const uint64_t qd = adv(q_kmaj, s * C::TILE);
+    const uint64_t kd = adv(kv_kmaj, stage_of(j, 0) * C::TILE);
 #pragma unroll
     for (int kk = 0; kk < D / 16; kk++) {
       const uint32_t off = (kk / 4) * PANEL + (kk % 4) * 32;
-      mma_ss(tmem + s_col(s), sw128_desc(qa + off, 16, 1024), sw128_desc(ka + off, 16, 1024), idesc_qk, kk > 0);
+      mma_ss(tmem + s_col(s), adv(qd, off), adv(kd, off), idesc_qk, kk > 0);
     }
     mma_commit(&bars.s_full[s]);
   };
 
-#pragma unroll
   for (int s = 0; s < 2; s++)
     if (u.lo[s] < u.hi[s] && !mbar_wait(&bars.q_full[s], 0, g, 10)) goto out;
 
@@ -212,16 +215,16 @@ __device__ void mma_issuer(const FwdParams& P, const Unit& u, uint8_t* smem, Bar
     if (next) {
       if (!mbar_wait(&bars.kv_full[stage_of(j + 1, 0)], phase_of(j + 1, 0), g, 13)) goto out;
     }
-    const uint32_t va = kv_addr + stage_of(j, 1) * C::TILE;
+    const uint64_t vd = adv(kv_mn, stage_of(j, 1) * C::TILE);
 #pragma unroll
     for (int s = 0; s < 2; s++) {
       if (active(u, s, j)) {
         if (!mbar_wait(&bars.p_full[s], (j - u.lo[s]) & 1, g, 14 + s)) goto out;
         tc_fence_after();
+        const uint32_t acc0 = j > u.lo[s];
 #pragma unroll
         for (int kk = 0; kk < BN / 16; kk++)
-          mma_ts(tmem + o_col(s), tmem + s_col(s) + kk * 8, sw128_desc(va + kk * 2048, PANEL, 1024), idesc_pv,
-                 (j > u.lo[s]) || kk > 0);
+          mma_ts(tmem + o_col(s), tmem + s_col(s) + kk * 8, adv(vd, kk * 2048), idesc_pv, kk > 0 ? 1u : acc0);
         if (j == u.hi[s] - 1) mma_commit(&bars.o_full[s]);
       }
       if (next && active(u, s, j + 1)) issue_s(s, j + 1);

@@ -127,6 +127,16 @@ __device__ __forceinline__ void regs_inc() {
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
+// Move this warpgroup's budget from the launch count LAUNCH to N: setmaxnreg.inc
+// only raises and setmaxnreg.dec only lowers (the other direction is
+// undefined), so pick the instruction at compile time.
+template <int N, int LAUNCH>
+__device__ __forceinline__ void regs_set() {
+  static_assert(N % 8 == 0 && N >= 24 && N <= 256, "setmaxnreg range");
+  if constexpr (N > LAUNCH) regs_inc<N>();
+  else if constexpr (N < LAUNCH) regs_dec<N>();
+}
+
 // ------------------------------------------------------------------ proxies
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
