@@ -52,7 +52,10 @@ struct Cfg {
   // operand from TMEM (no P^T tile in shared memory).  d = 64 has no TMEM
   // room for them and reads both from shared memory.
   static constexpr bool TS = D == 128;
-  static constexpr int NQS = D == 128 ? 4 : 3;       // Q/dO ring stages
+  static constexpr int NQS = 3;                   // Q/dO ring stages
+  // d = 128: the dQ^T tile of a step leaves through two 16 KB halves of a
+  // 128-byte-swizzled staging area and a TMA tensor reduce-add.
+  static constexpr int STG_BYTES = D == 128 ? 2 * 16384 : 0;
   static constexpr int KV_TILE = BN * D * 2;
   static constexpr int Q_TILE = BM * D * 2;
   static constexpr int Q_PANEL = BM * 128;
@@ -64,12 +67,15 @@ struct Cfg {
   static constexpr int OFF_DO = OFF_Q + NQS * Q_TILE;
   static constexpr int OFF_PT = OFF_DO + NQS * Q_TILE;
   static constexpr int OFF_DST = OFF_PT + (TS ? 0 : NBUF * PS_TILE);
-  static constexpr int OFF_VEC = OFF_DST + NBUF * PS_TILE;  // [group][2 bufs][lse2 | D][CW] fp32
+  static constexpr int OFF_STG = OFF_DST + NBUF * PS_TILE;
+  static constexpr int OFF_VEC = OFF_STG + STG_BYTES;  // [group][2 bufs][lse2 | D][CW] fp32
   static constexpr int OFF_BAR = OFF_VEC + 2 * 2 * 2 * CW * 4;
   static constexpr int SMEM = OFF_BAR + 256 + 1024;
   static constexpr uint32_t T_S = 0, T_DP = BM, T_DV = 2 * BM, T_DK = 2 * BM + D, T_DQ = 2 * BM + 2 * D;
   static constexpr uint32_t T_PT = T_DQ + 64, T_DST = T_PT + BM / 2;  // bf16 pairs (TS only)
   static_assert(T_DQ + 64 <= 512 && (!TS || T_DST + BM / 2 <= 512), "tensor memory budget");
+  static_assert(SMEM <= 232448, "shared memory budget");
+  static_assert(OFF_STG % 1024 == 0, "staging must be 1024-byte aligned for the 128-byte swizzle");
 };
 
 // Barriers.  The MMA issuer pays for every wait and commit with tensor-core
@@ -89,6 +95,7 @@ struct Bars {
   uint64_t grad_ready[2];
   uint64_t sdp_full, step_done;
   uint64_t vec_full[2][2];  // [group][buffer]
+  uint64_t stg_full[2], stg_free[2];  // dQ staging halves (d = 128)
   uint64_t dkv_full;
   uint64_t drain[2];
   uint32_t tmem_base;
@@ -465,26 +472,41 @@ __device__ void grad_rows(const BwdParams& P, const Unit& u, uint8_t* smem, Bars
 }
 
 // ------------------------------------------------------------------ dQ drain
-// Moves each step's 128 x 64 fp32 dQ tile out of tensor memory and adds it
-// into the fp32 accumulator with atomic adds (red.global: no return value;
-// element-wise atomic in L2).  At d = 128 lane t holds column t of dQ for the
-// step's 64 queries, so each warp instruction covers 32 consecutive floats.
+// Moves each step's fp32 dQ tile out of tensor memory into the accumulator,
+// which is stored transposed, [head][d][q] (row pitch lq_pad), so that the
+// values a lane holds are contiguous in it:
+//   d = 128 (dQ^T in TMEM, lane = d, 64 query columns): the lane writes its
+//     row as 16-byte pieces into a 128-byte-swizzled staging half (32
+//     queries x 128 rows = 16 KB, conflict-free), and one thread adds the
+//     half into the accumulator with a TMA tensor reduce-add (element-wise
+//     atomic in L2); two halves alternate so staging overlaps the reduce.
+//   d = 64 (dQ in TMEM, lane = query, 64 d columns): per column, the lanes
+//     hold 32 consecutive queries, so red.global covers 128 bytes per warp.
 __device__ __forceinline__ void red_add_f32(float* p, float v) {
   asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
 }
-__device__ __forceinline__ void red_add_v4_f32(float* p, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
-               : "memory");
+
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* map, const void* src, int c0, int c1) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(smem_u32(src)), "r"(c0), "r"(c1)
+      : "memory");
 }
+// Wait until at most one committed bulk group still reads shared memory.
+__device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 
 template <int D>
-__device__ void dq_drain(const BwdParams& P, const Unit& u, Bars& bars, uint32_t tmem, const WaitGuard& g) {
+__device__ void dq_drain(const BwdParams& P, const Unit& u, uint8_t* smem, Bars& bars, uint32_t tmem,
+                         const WaitGuard& g) {
   using C = Cfg<D>;
   const Problem& p = P.prob;
   const int t = threadIdx.x % 128;  // TMEM lane
   const int wl = (threadIdx.x / 32) % 4;
   const int lane = threadIdx.x % 32;
   const uint32_t lane_base = (uint32_t)(wl * 32) << 16;
+  uint8_t* stg = smem + C::OFF_STG;
+  int half = 0;  // staging halves used so far
 
   // Step 0 has no earlier dQ to read out.
   if (lane == 0) mbar_arrive(&bars.grad_ready[0]);
@@ -500,23 +522,40 @@ __device__ void dq_drain(const BwdParams& P, const Unit& u, Bars& bars, uint32_t
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(&bars.grad_ready[(i + 1) & 1]);  // dQ TMEM free for step i+1
-    float* base = P.dq_acc + (size_t)(u.b * p.Hq + h) * p.Lq * D;
-    if (D == 128) {
-      // Lane t holds dQ^T row t (= column t of dQ) for the BM = 64 queries.
+    const int bh = u.b * p.Hq + h;
+    if constexpr (D == 128) {
 #pragma unroll
-      for (int qq = 0; qq < 64; qq++)
-        if (q0 + qq < p.Lq) red_add_f32(base + (size_t)(q0 + qq) * D + t, __uint_as_float(r[qq]));
+      for (int hh = 0; hh < 2; hh++, half++) {
+        const int b = half & 1, use = half >> 1;
+        // The reduce of this buffer's previous use must have read it.
+        if (use > 0 && !mbar_wait(&bars.stg_free[b], (use - 1) & 1, g, 31)) return;
+        uint8_t* row = stg + b * 16384 + t * 128;
+#pragma unroll
+        for (int c = 0; c < 8; c++)
+          *reinterpret_cast<uint4*>(row + (((uint32_t)c ^ (uint32_t)(t & 7)) << 4)) =
+              make_uint4(r[32 * hh + 4 * c], r[32 * hh + 4 * c + 1], r[32 * hh + 4 * c + 2], r[32 * hh + 4 * c + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.stg_full[b]);
+        if (t == 0) {
+          if (!mbar_wait(&bars.stg_full[b], use & 1, g, 32)) return;
+          // Columns past Lq are clipped by the tensor bounds.
+          tma_reduce_add_2d(&P.tm_dq, stg + b * 16384, q0 + 32 * hh, bh * D);
+          bulk_commit();
+          bulk_wait_read_1();  // the previous half has been read
+          if (half > 0) mbar_arrive(&bars.stg_free[(half - 1) & 1]);
+        }
+      }
     } else {
-      // Lane t holds dQ row q0 + t (64 values of d).
+      // Lane t holds dQ row q0 + t: column c goes to accumulator row (bh, c).
       if (q0 + t < p.Lq) {
-        float* rowp = base + (size_t)(q0 + t) * D;
+        float* colp = P.dq_acc + (size_t)bh * D * P.lq_pad + q0 + t;
 #pragma unroll
-        for (int v = 0; v < 16; v++)
-          red_add_v4_f32(rowp + 4 * v, __uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
-                         __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+        for (int c = 0; c < 64; c++) red_add_f32(colp + (size_t)c * P.lq_pad, __uint_as_float(r[c]));
       }
     }
   }
+  if (D == 128 && t == 0) bulk_wait_all();  // every reduce complete before the CTA exits
 }
 
 // ------------------------------------------------------------------ kernel
@@ -550,6 +589,10 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kernel(const __grid_const
     }
     mbar_init(&bars.sdp_full, 1);
     mbar_init(&bars.step_done, 1);
+    for (int b = 0; b < 2; b++) {
+      mbar_init(&bars.stg_full[b], 4);  // 4 drain warps wrote their rows
+      mbar_init(&bars.stg_free[b], 1);  // the reduce finished reading the half
+    }
     mbar_init(&bars.dkv_full, 1);
     mbar_init(&bars.drain[0], 1);
     mbar_init(&bars.drain[1], 1);
@@ -581,7 +624,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kernel(const __grid_const
     grad_rows<D>(P, u, smem, bars, tmem, (warp - 4) / 4, g);
   } else {
     regs_set<RQ, 128>();
-    dq_drain<D>(P, u, bars, tmem, g);
+    dq_drain<D>(P, u, smem, bars, tmem, g);
   }
   tc_fence_before();
   __syncthreads();
@@ -597,7 +640,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kernel(const __grid_const
 template <int D>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dO,
                                                       float* __restrict__ dvec, float* __restrict__ dq_acc,
-                                                      int64_t rows) {
+                                                      int64_t rows, int64_t acc_floats) {
   constexpr int TPR = D / 8;  // threads per row
   const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -615,29 +658,42 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const uint16_t* __restrict
         acc = fmaf(__uint_as_float(aw[e] << 16), __uint_as_float(bw[e] << 16), acc);
         acc = fmaf(__uint_as_float(aw[e] & 0xFFFF0000u), __uint_as_float(bw[e] & 0xFFFF0000u), acc);
       }
-      float4* z = reinterpret_cast<float4*>(dq_acc + r * D + part * 8);
-      z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-      z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
     for (int sh = TPR / 2; sh > 0; sh >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, sh);
     if (r < rows && part == 0) dvec[r] = acc;
   }
+  // The accumulator (a multiple of 4 floats) is zeroed with 16-byte stores.
+  float4* z = reinterpret_cast<float4*>(dq_acc);
+  for (int64_t x = tid; x < acc_floats / 4; x += stride) z[x] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
-// dQ = scale * accumulator, rounded to bf16; 8 elements per thread.
-__global__ void __launch_bounds__(256) bwd_post_kernel(const float* __restrict__ acc, uint16_t* __restrict__ dq,
-                                                       int64_t n8, float scale) {
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; x < n8; x += stride) {
-    const float4 a = reinterpret_cast<const float4*>(acc)[2 * x];
-    const float4 b = reinterpret_cast<const float4*>(acc)[2 * x + 1];
-    uint4 w;
-    w.x = pack_bf16x2(a.x * scale, a.y * scale);
-    w.y = pack_bf16x2(a.z * scale, a.w * scale);
-    w.z = pack_bf16x2(b.x * scale, b.y * scale);
-    w.w = pack_bf16x2(b.z * scale, b.w * scale);
-    reinterpret_cast<uint4*>(dq)[x] = w;
+// dQ[bh, q, :] = scale * acc[bh, :, q], rounded to bf16.  One CTA transposes a
+// 64-query x d tile through shared memory: reads run along q, writes along d.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_post_kernel(const float* __restrict__ acc, uint16_t* __restrict__ dq, int Lq,
+                                                       int lq_pad, float scale) {
+  __shared__ float tile[D][65];
+  const int bh = blockIdx.y;
+  const int q0 = blockIdx.x * 64;
+  const float* src = acc + (size_t)bh * D * lq_pad;
+  for (int idx = threadIdx.x; idx < D * 64; idx += 256) {
+    const int dd = idx / 64, qq = idx % 64;
+    tile[dd][qq] = q0 + qq < Lq ? src[(size_t)dd * lq_pad + q0 + qq] : 0.f;
+  }
+  __syncthreads();
+  constexpr int CH = D / 8;  // 16-byte output chunks per row
+  for (int idx = threadIdx.x; idx < 64 * CH; idx += 256) {
+    const int qq = idx / CH, c = idx % CH;
+    const int q = q0 + qq;
+    if (q < Lq) {
+      uint4 w;
+      w.x = pack_bf16x2(tile[c * 8 + 0][qq] * scale, tile[c * 8 + 1][qq] * scale);
+      w.y = pack_bf16x2(tile[c * 8 + 2][qq] * scale, tile[c * 8 + 3][qq] * scale);
+      w.z = pack_bf16x2(tile[c * 8 + 4][qq] * scale, tile[c * 8 + 5][qq] * scale);
+      w.w = pack_bf16x2(tile[c * 8 + 6][qq] * scale, tile[c * 8 + 7][qq] * scale);
+      *reinterpret_cast<uint4*>(dq + ((size_t)bh * Lq + q) * D + c * 8) = w;
+    }
   }
 }
 
@@ -652,22 +708,29 @@ static int elementwise_grid(int64_t work_threads) {
 }
 
 cudaError_t launch_bwd_pre(const void* o, const void* dO, float* dvec, float* dq_acc, int64_t rows, int d,
-                           cudaStream_t stream) {
+                           int64_t acc_floats, cudaStream_t stream) {
   if (rows <= 0) return cudaSuccess;
-  const int grid = elementwise_grid(rows * (d / 8));
+  const int64_t work = rows * (d / 8) > acc_floats / 4 ? rows * (d / 8) : acc_floats / 4;
+  const int grid = elementwise_grid(work);
   if (d == 128)
     bwd::bwd_pre_kernel<128><<<grid, 256, 0, stream>>>(static_cast<const uint16_t*>(o),
-                                                        static_cast<const uint16_t*>(dO), dvec, dq_acc, rows);
+                                                        static_cast<const uint16_t*>(dO), dvec, dq_acc, rows,
+                                                        acc_floats);
   else
     bwd::bwd_pre_kernel<64><<<grid, 256, 0, stream>>>(static_cast<const uint16_t*>(o),
-                                                       static_cast<const uint16_t*>(dO), dvec, dq_acc, rows);
+                                                       static_cast<const uint16_t*>(dO), dvec, dq_acc, rows,
+                                                       acc_floats);
   return cudaGetLastError();
 }
 
-cudaError_t launch_bwd_post(const float* dq_acc, void* dq, int64_t n, float scale, cudaStream_t stream) {
-  if (n <= 0) return cudaSuccess;
-  const int64_t n8 = n / 8;
-  bwd::bwd_post_kernel<<<elementwise_grid(n8), 256, 0, stream>>>(dq_acc, static_cast<uint16_t*>(dq), n8, scale);
+cudaError_t launch_bwd_post(const float* dq_acc, void* dq, int BH, int Lq, int lq_pad, int d, float scale,
+                            cudaStream_t stream) {
+  if (BH <= 0 || Lq <= 0) return cudaSuccess;
+  const dim3 grid((Lq + 63) / 64, BH);
+  if (d == 128)
+    bwd::bwd_post_kernel<128><<<grid, 256, 0, stream>>>(dq_acc, static_cast<uint16_t*>(dq), Lq, lq_pad, scale);
+  else
+    bwd::bwd_post_kernel<64><<<grid, 256, 0, stream>>>(dq_acc, static_cast<uint16_t*>(dq), Lq, lq_pad, scale);
   return cudaGetLastError();
 }
 
