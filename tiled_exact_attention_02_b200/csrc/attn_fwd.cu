@@ -43,15 +43,50 @@ constexpr int THREADS = 384;
 constexpr int PANEL = 16384;   // one 128-row x 128-byte swizzled panel
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
 
+// Part of the exponentials run on the FMA pipe instead of the special-function
+// unit, which is otherwise the busiest pipe of the softmax: 2^x = 2^n * p(f)
+// with n = round(x) (Cody-Waite reduction: adding 1.5 * 2^23 rounds to an
+// integer and leaves n in the low mantissa bits), f = x - n in [-1/2, 1/2], p
+// the degree-4 polynomial minimising the relative error of 2^f there (Remez
+// exchange; coefficients from gen_exp2_poly.py, error < 3e-6), and 2^n
+// applied by adding n to the exponent field.  Arguments are clamped at -126
+// (p(f) may sit just below 1, exponent field 126, so n >= -126 keeps the sum
+// from wrapping into the sign bit);
+// only tiles without masked entries use it, so a masked -inf never gets here.
+constexpr float EXP2_C0 = 0.9999992847442627f;  // 0x3f7ffff4
+constexpr float EXP2_C1 = 0.6931217908859253f;  // 0x3f31706e
+constexpr float EXP2_C2 = 0.240247443318367f;  // 0x3e76036d
+constexpr float EXP2_C3 = 0.05591785907745361f;  // 0x3d650a20
+constexpr float EXP2_C4 = 0.009570102207362652f;  // 0x3c1ccbeb
+constexpr int POLY_EVERY = 4;  // one pair of columns in POLY_EVERY uses the polynomial
+
+__device__ __forceinline__ void exp2_poly2(float& r0, float& r1, float x0, float x1) {
+  constexpr float MAGIC = 12582912.0f;  // 1.5 * 2^23
+  x0 = fmaxf(x0, -126.f);
+  x1 = fmaxf(x1, -126.f);
+  float t0, t1, n0, n1, f0, f1, p0, p1;
+  add2(t0, t1, x0, x1, MAGIC, MAGIC);
+  add2(n0, n1, t0, t1, -MAGIC, -MAGIC);
+  fma2(f0, f1, n0, n1, -1.f, -1.f, x0, x1);
+  fma2(p0, p1, EXP2_C4, EXP2_C4, f0, f1, EXP2_C3, EXP2_C3);
+  fma2(p0, p1, p0, p1, f0, f1, EXP2_C2, EXP2_C2);
+  fma2(p0, p1, p0, p1, f0, f1, EXP2_C1, EXP2_C1);
+  fma2(p0, p1, p0, p1, f0, f1, EXP2_C0, EXP2_C0);
+  r0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  r1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
 template <int D>
 struct Cfg {
   static constexpr int PANELS = D / 64;
   static constexpr int TILE = BM * D * 2;         // bytes of one Q, K or V tile
-  static constexpr int NST = D == 128 ? 4 : 8;    // K/V ring stages
+  static constexpr int NST = D == 128 ? 5 : 8;    // K/V ring stages (2.5 key tiles ahead at d = 128)
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = 2 * TILE;
   static constexpr int OFF_BAR = OFF_KV + NST * TILE;
   static constexpr int SMEM = OFF_BAR + 512 + 1024;  // barriers + alignment slack
+  static_assert(SMEM <= 232448, "shared memory budget");
+  static_assert(NST <= 8, "barrier arrays");
 };
 
 struct Bars {
@@ -273,7 +308,8 @@ __device__ void softmax_slot(const FwdParams& P, const Unit& u, int s, Bars& bar
 
     // Element-wise mask only on tiles that straddle this row's visible range.
     const int key0 = j * BN;
-    if (key0 < key_lo || key0 + BN > key_hi) {
+    const bool masked = key0 < key_lo || key0 + BN > key_hi;
+    if (masked) {
 #pragma unroll
       for (int cc = 0; cc < BN; cc++) {
         const int key = key0 + cc;
@@ -282,11 +318,11 @@ __device__ void softmax_slot(const FwdParams& P, const Unit& u, int s, Bars& bar
     }
     float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-    for (int cc = 0; cc < BN; cc += 4) {
-      mx0 = fmaxf(mx0, __uint_as_float(x[cc]));
-      mx1 = fmaxf(mx1, __uint_as_float(x[cc + 1]));
-      mx2 = fmaxf(mx2, __uint_as_float(x[cc + 2]));
-      mx3 = fmaxf(mx3, __uint_as_float(x[cc + 3]));
+    for (int cc = 0; cc < BN; cc += 8) {
+      mx0 = max3(mx0, __uint_as_float(x[cc]), __uint_as_float(x[cc + 1]));
+      mx1 = max3(mx1, __uint_as_float(x[cc + 2]), __uint_as_float(x[cc + 3]));
+      mx2 = max3(mx2, __uint_as_float(x[cc + 4]), __uint_as_float(x[cc + 5]));
+      mx3 = max3(mx3, __uint_as_float(x[cc + 6]), __uint_as_float(x[cc + 7]));
     }
     const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
     const float m_cand = mx == -INFINITY ? -INFINITY : mx * c;
@@ -300,14 +336,32 @@ __device__ void softmax_slot(const FwdParams& P, const Unit& u, int s, Bars& bar
     const float m_sub = m == -INFINITY ? 0.f : m;
     float s0 = 0.f, s1 = 0.f;
     // P packed two per 32-bit word, written over x[0 .. BN/2) as it goes
-    // (x[2cc], x[2cc+1] are dead once read).
+    // (x[2cc], x[2cc+1] are dead once read).  Tiles this warp sees without
+    // masking send one pair in POLY_EVERY to the FMA-pipe exponential.
+    const bool poly = __all_sync(0xffffffffu, !masked);
+    if (poly) {
 #pragma unroll
-    for (int cc = 0; cc < BN / 2; cc++) {
-      const float p0 = ex2_approx(fmaf(__uint_as_float(x[2 * cc]), c, -m_sub));
-      const float p1 = ex2_approx(fmaf(__uint_as_float(x[2 * cc + 1]), c, -m_sub));
-      s0 += p0;
-      s1 += p1;
-      x[cc] = pack_bf16x2(p0, p1);
+      for (int cc = 0; cc < BN / 2; cc++) {
+        float a0, a1, p0, p1;
+        fma2(a0, a1, __uint_as_float(x[2 * cc]), __uint_as_float(x[2 * cc + 1]), c, c, -m_sub, -m_sub);
+        if (cc % POLY_EVERY == POLY_EVERY - 1) {
+          exp2_poly2(p0, p1, a0, a1);
+        } else {
+          p0 = ex2_approx(a0);
+          p1 = ex2_approx(a1);
+        }
+        add2(s0, s1, s0, s1, p0, p1);
+        x[cc] = pack_bf16x2(p0, p1);
+      }
+    } else {
+#pragma unroll
+      for (int cc = 0; cc < BN / 2; cc++) {
+        float a0, a1;
+        fma2(a0, a1, __uint_as_float(x[2 * cc]), __uint_as_float(x[2 * cc + 1]), c, c, -m_sub, -m_sub);
+        const float p0 = ex2_approx(a0), p1 = ex2_approx(a1);
+        add2(s0, s1, s0, s1, p0, p1);
+        x[cc] = pack_bf16x2(p0, p1);
+      }
     }
     l += s0 + s1;
     // P (bf16, two per column) replaces the first BN/2 columns of S.
