@@ -109,27 +109,42 @@ class ClockSampler:
                 "samples": len(sm), "reasons": sorted(reasons)}
 
 
-def dist_setup(n_gpus):
+def dist_setup(n_gpus, backend="nccl"):
+    """Join the torchrun job (one process per GPU); returns (rank, world, local rank)."""
     import torch
     import torch.distributed as dist
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
-        torch.cuda.set_device(local)
         from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=timedelta(seconds=120))
     return rank, world, local
 
 
-def max_over_ranks(x, world):
+def rank_seed(w, rank):
+    """Each rank draws its own batch of the workload (independent units)."""
+    return w.seed + 1000 * rank
+
+
+def max_over_ranks(x, world, device="cuda"):
+    """The job's time is the slowest rank's."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(world, flops_per_rank_step, ms_per_step_max):
+    """Whole-job TFLOP/s under weak scaling: every rank does one step's work."""
+    return world * flops_per_rank_step / (ms_per_step_max * 1e-3) / 1e12
 
 
 def barrier(world):
@@ -220,7 +235,7 @@ def main():
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     w = WORKLOADS[WORKLOAD]
-    x = make_inputs(w, seed=w.seed + rank)
+    x = make_inputs(w, seed=rank_seed(w, rank))
 
     def dev_bf16(bits):
         import numpy as np
@@ -265,7 +280,7 @@ def main():
     ms_total = max_over_ranks(t_start.elapsed_time(t_end), world)
     ms_step = ms_total / args.steps
     flops_step = w.fwd_flops() + w.bwd_flops()
-    value = world * flops_step / (ms_step * 1e-3) / 1e12
+    value = job_throughput(world, flops_step, ms_step)
 
     names = ["attn_fwd", "attn_bwd_preprocess", "attn_bwd_main", "attn_bwd_finalize"]
     per = {n: statistics.mean(e[j].elapsed_time(e[j + 1]) for e in events) for j, n in enumerate(names)}
@@ -303,7 +318,7 @@ def main():
         b.record(stream)
         torch.cuda.synchronize()
         ms_e2e = max_over_ranks(a.elapsed_time(b), world) / args.e2e_steps
-        e2e = {"value": world * flops_step / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e2e = {"value": job_throughput(world, flops_step, ms_e2e), "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e}
 
     if rank != 0:
