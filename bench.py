@@ -34,7 +34,7 @@ from synth import WORKLOADS, make_inputs  # noqa: E402
 WORKLOAD = "mha_causal_fwdbwd"
 METRIC = "attention TFLOP/s (bf16, mask-adjusted) fwd+bwd and % of B200 dense BF16 peak"
 DOMINANT = "attn_bwd_main"
-PROFILE = os.path.join(ROOT, "profiles", "attn_bwd_main_mha_causal_4096.md")
+PROFILE = os.path.join(ROOT, "profiles", "attn_bwd_main_mha_causal_fwdbwd.md")
 KERNEL_SRC = os.path.join(ROOT, "tiled_exact_attention_02_b200", "csrc", "attn_bwd.cu")
 
 
