@@ -13,7 +13,8 @@
 //             the query heads of the GQA group and the query tiles that see
 //             its keys, accumulating dK and dV in tensor memory for the whole
 //             loop and adding each step's dQ contribution into the fp32
-//             accumulator with coalesced atomic adds (red.global)
+//             accumulator (d = 128: TMA tensor reduce-add from a swizzled
+//             staging tile; d = 64: coalesced red.global)
 //   bwd_post  dQ = scale * accumulator, rounded to bf16
 //
 // bwd_main works in the transposed orientation, keys on the 128 TMEM lanes:
@@ -25,8 +26,9 @@
 // A operand of dV/dK and as the MN-major operand of dQ.
 // Warp roles (512 threads): warp 0 TMA, warps 1 and 2 MMA issuers, warps 4-7 and
 // 8-11 the per-key softmax gradient (each group takes half of a step's query
-// columns), warps 12-15 the dQ drain.  Tensor memory: S^T | dP^T | dV | dK |
-// dQ, 448 of 512 columns.  Q/dO tiles stream through a 3-stage ring.
+// columns), warps 12-15 the dQ drain.  Tensor memory at d = 128:
+// S^T | dP^T | dV | dK | dQ^T | P^T | dS^T = 512 columns.  Q/dO tiles stream
+// through a 3-stage ring.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cstdint>
@@ -562,7 +564,8 @@ __device__ void dq_drain(const BwdParams& P, const Unit& u, uint8_t* smem, Bars&
 // Per-thread register budgets after setmaxnreg (launch: 512 x 128):
 // load/MMA group, gradient groups, dQ drain; 128*RM + 256*RG + 128*RQ <= 65536.
 constexpr int RM = 104, RG = 152, RQ = 104;
-static_assert(128 * RM + 256 * RG + 128 * RQ <= 512 * 128, "register budget");
+constexpr int LAUNCH_REGS = 128;  // 65536 / 512
+static_assert(128 * RM + 256 * RG + 128 * RQ <= THREADS * LAUNCH_REGS, "register budget");
 
 template <int D>
 __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kernel(const __grid_constant__ BwdParams P) {
@@ -607,11 +610,10 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kernel(const __grid_const
   tc_fence_after();
   const uint32_t tmem = bars.tmem_base;
 
-  // Registers: 512 x 128 at launch; the load/MMA group keeps 120 (the issue
-  // loop holds a dozen 64-bit descriptors), the other three keep 128
-  // (128*120 + 384*128 <= 512*128).
+  // Registers: 512 x 128 at launch, redistributed per warpgroup (RM, RG, RQ
+  // above); the host refuses the launch at any other compiled count.
   if (warp < 4) {
-    regs_set<RM, 128>();
+    regs_set<RM, LAUNCH_REGS>();
     if (warp == 0) {
       if (lane == 0) producer<D>(P, u, smem, bars, g);
     } else if (warp == 1) {
@@ -620,10 +622,10 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kernel(const __grid_const
       if (lane == 0) mma_issuer<D, 1>(P, u, smem, bars, tmem, g);
     }
   } else if (warp < 12) {
-    regs_set<RG, 128>();
+    regs_set<RG, LAUNCH_REGS>();
     grad_rows<D>(P, u, smem, bars, tmem, (warp - 4) / 4, g);
   } else {
-    regs_set<RQ, 128>();
+    regs_set<RQ, LAUNCH_REGS>();
     dq_drain<D>(P, u, smem, bars, tmem, g);
   }
   tc_fence_before();
@@ -738,6 +740,10 @@ template <int D>
 static cudaError_t launch_bwd_d(const BwdParams& P, cudaStream_t stream) {
   constexpr int smem = bwd::Cfg<D>::SMEM;
   cudaError_t e = cudaFuncSetAttribute(bwd::attn_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  // setmaxnreg redistributes the registers the block was launched with: the
+  // split above is only valid at exactly LAUNCH_REGS per thread.
+  e = check_launch_regs(reinterpret_cast<const void*>(bwd::attn_bwd_kernel<D>), bwd::LAUNCH_REGS);
   if (e != cudaSuccess) return e;
   bwd::attn_bwd_kernel<D><<<P.n_units, bwd::THREADS, smem, stream>>>(P);
   return cudaGetLastError();

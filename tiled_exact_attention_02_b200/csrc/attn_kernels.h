@@ -41,6 +41,16 @@ struct BwdParams {
   uint64_t limit_ns;
 };
 
+// Kernels that move registers between warp roles with setmaxnreg are only
+// correct at the register count their split was written for: a launch at any
+// other count is refused before it starts.
+inline cudaError_t check_launch_regs(const void* kernel, int expected) {
+  cudaFuncAttributes a;
+  cudaError_t e = cudaFuncGetAttributes(&a, kernel);
+  if (e != cudaSuccess) return e;
+  return a.numRegs == expected ? cudaSuccess : cudaErrorInvalidConfiguration;
+}
+
 // Query rows per backward step for head dimension d.
 inline int bwd_block_m(int d) { return d == 128 ? 64 : 128; }
 
