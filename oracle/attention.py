@@ -11,7 +11,9 @@ Sources (page title and section):
   * "高效注意力" §3 (MQA/GQA): several query heads share one K/V head.
   * "高效注意力" §4 and "大模型高效注意力机制全解析" §3.2.1 (sliding_window):
       each token attends to a window of nearby tokens.  Read here as the
-      causal band  i - w < j <= i  (w keys, the query itself included).
+      causal band  i - w < j <= i  (w keys, the query itself included), and,
+      without a causal mask, as the two-sided band  i - w < j < i + w  (the
+      "前后" (before and after) wording of the same section).
   * "缩放定律与高效注意力" §3.3: the backward pass needs only O and the per-row
       logsumexp; the gradient formulas themselves are the textbook softmax
       gradient (the pages do not print them).
@@ -33,21 +35,37 @@ import numpy as np
 _ROW_BLOCK_ELEMS = 1 << 24
 
 
-def visible_mask(Lq: int, Lk: int, causal: bool, window: int) -> np.ndarray:
-    """Boolean [Lq, Lk]: True where key j is visible to query i."""
-    i = np.arange(Lq)[:, None]
-    j = np.arange(Lk)[None, :]
-    vis = np.ones((Lq, Lk), dtype=bool)
+def _visible(i, j, causal: bool, window: int) -> np.ndarray:
+    """Elementwise visibility of key j to query i (broadcasting arrays)."""
+    vis = np.ones(np.broadcast(i, j).shape, dtype=bool)
     if causal:
         vis &= j <= i
     if window > 0:
         vis &= j > i - window
+        if not causal:
+            vis &= j < i + window
     return vis
+
+
+def visible_mask(Lq: int, Lk: int, causal: bool, window: int) -> np.ndarray:
+    """Boolean [Lq, Lk]: True where key j is visible to query i.
+
+    Causal: j <= i.  Window w > 0: the w keys ending at i when causal
+    (i - w < j <= i, "高效注意力" §4 sliding window); without causal the band
+    reaches w - 1 keys to either side, i - w < j < i + w (the two-sided
+    "前后" reading of the same section).
+    """
+    return _visible(np.arange(Lq)[:, None], np.arange(Lk)[None, :], causal, window)
 
 
 def visible_band(r0: int, r1: int, Lk: int, causal: bool, window: int) -> tuple[int, int]:
     """Columns [lo, hi) that can be visible to any row in [r0, r1)."""
-    hi = min(Lk, r1) if causal else Lk
+    if causal:
+        hi = min(Lk, r1)
+    elif window > 0:
+        hi = min(Lk, r1 - 1 + window)
+    else:
+        hi = Lk
     lo = max(0, r0 - window + 1) if window > 0 else 0
     return lo, max(lo, hi)
 
@@ -102,14 +120,7 @@ def _head_fwd(qh, kh, vh, scale, causal, window, rows=None):
 
 
 def _band_mask(rows, lo, hi, causal, window):
-    i = np.asarray(rows)[:, None]
-    j = np.arange(lo, hi)[None, :]
-    vis = np.ones((i.shape[0], hi - lo), dtype=bool)
-    if causal:
-        vis &= j <= i
-    if window > 0:
-        vis &= j > i - window
-    return vis
+    return _visible(np.asarray(rows)[:, None], np.arange(lo, hi)[None, :], causal, window)
 
 
 def _group(Hq: int, Hkv: int) -> int:

@@ -45,7 +45,7 @@ def test_golden_hand_worked_example():
 
 
 # ---------------------------------------------------------------- invariants
-MASKS = [(False, 0), (True, 0), (True, 5), (True, 1), (True, 64)]
+MASKS = [(False, 0), (True, 0), (True, 5), (True, 1), (True, 64), (False, 5), (False, 1)]
 
 
 @pytest.mark.parametrize("causal,window", MASKS)
@@ -107,6 +107,30 @@ def test_single_visible_key_returns_that_row():
     O, lse = oracle.attn_fwd(q, k, v, 0.3, True, 1)
     assert np.array_equal(O[0, 0], v[0, 0])
     np.testing.assert_allclose(lse[0, 0], 0.3 * np.sum(q[0, 0] * k[0, 0], 1), atol=1e-14)
+
+
+def test_two_sided_window_w1_is_the_diagonal():
+    """Without causal, window 1 leaves each row its own key only: O = V, LSE = S_ii."""
+    L, d = 9, 5
+    q, k, v = _rand(1, 1, L, d), _rand(1, 1, L, d), _rand(1, 1, L, d)
+    O, lse = oracle.attn_fwd(q, k, v, 0.7, False, 1)
+    assert np.array_equal(O[0, 0], v[0, 0])
+    np.testing.assert_allclose(lse[0, 0], 0.7 * np.sum(q[0, 0] * k[0, 0], 1), atol=1e-14)
+
+
+def test_two_sided_window_counts_and_band():
+    """Two-sided window w: row i sees min(i, w-1) keys before it, itself, and
+    min(L-1-i, w-1) after it; the row-block band covers every visible column."""
+    L, w = 23, 4
+    vis = oracle.visible_mask(L, L, False, w)
+    for i in range(L):
+        assert vis[i].sum() == min(i, w - 1) + 1 + min(L - 1 - i, w - 1)
+        assert vis[i, i] and not vis[i, max(0, i - w)] or i - w < 0
+    for r0 in range(0, L, 5):
+        r1 = min(L, r0 + 5)
+        lo, hi = oracle.visible_band(r0, r1, L, False, w)
+        cols = np.flatnonzero(vis[r0:r1].any(0))
+        assert lo == cols.min() and hi == cols.max() + 1
 
 
 def test_value_shift_and_score_shift_invariance():
@@ -195,7 +219,7 @@ def _loss(q, k, v, R, scale, causal, window):
 
 @pytest.mark.parametrize("Hq,Hkv,L,causal,window", [
     (2, 2, 9, False, 0), (2, 2, 9, True, 0), (2, 1, 8, True, 3), (2, 2, 7, True, 1),
-    (4, 2, 6, False, 0),
+    (4, 2, 6, False, 0), (2, 1, 9, False, 3),
 ])
 def test_backward_matches_finite_differences(Hq, Hkv, L, causal, window):
     """Gradient of <R, O> against central differences, float64, to 1e-6."""
@@ -293,6 +317,20 @@ def test_matches_torch_sdpa_float64(Hq, Hkv, causal, window):
     tk, tv = tk.repeat_interleave(G, 1), tv.repeat_interleave(G, 1)
     mask = torch.from_numpy(oracle.visible_mask(L, L, causal, window))
     ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=mask, scale=0.25)
+    np.testing.assert_allclose(O, ref.numpy(), atol=1e-12)
+
+
+@pytest.mark.parametrize("w", [1, 4, 40])
+def test_two_sided_window_matches_torch_sdpa(w):
+    """Non-causal window against torch SDPA with the band |i - j| < w built here."""
+    B, Hq, Hkv, L, d = 1, 4, 2, 37, 8
+    q, k, v = _rand(B, Hq, L, d), _rand(B, Hkv, L, d), _rand(B, Hkv, L, d)
+    O, _ = oracle.attn_fwd(q, k, v, 0.3, False, w)
+    idx = torch.arange(L)
+    band = (idx[:, None] - idx[None, :]).abs() < w
+    tq, tk, tv = (torch.from_numpy(x) for x in (q, k, v))
+    tk, tv = tk.repeat_interleave(2, 1), tv.repeat_interleave(2, 1)
+    ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=band, scale=0.3)
     np.testing.assert_allclose(O, ref.numpy(), atol=1e-12)
 
 
