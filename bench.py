@@ -46,6 +46,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--all-configs", action="store_true",
+                    help="time attn_fwd and the backward on every workload (one JSON line each); not the bench line")
     return ap.parse_args()
 
 
@@ -221,10 +223,61 @@ def run_reference(args):
     print(json.dumps(line))
 
 
+def all_configs(args):
+    """Forward and backward times of every workload on one GPU (CUDA-event
+    medians), one JSON line each.  The backward runs with a dO drawn for the
+    workload when it has none.  Inputs of the small case fit in L2."""
+    import numpy as np
+    import torch
+    import tiled_exact_attention_02_b200 as ta
+    burst, sustained, hbm, peak_src = peaks()
+    for name, w in WORKLOADS.items():
+        x = make_inputs(w)
+        dev = lambda bits: torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).cuda()
+        q, k, v = (dev(x[n]) for n in ("q", "k", "v"))
+        do = dev(x["do"]) if "do" in x else torch.randn_like(q)
+        o = torch.empty_like(q)
+        lse = torch.empty((w.B, w.Hq, w.Lq), dtype=torch.float32, device="cuda")
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        ws = torch.empty(ta.bwd_workspace_size(w.B, w.Hq, w.Hkv, w.Lq, w.Lk, w.d), dtype=torch.uint8, device="cuda")
+
+        def timed(fn, n):
+            ts = []
+            for it in range(n + 3):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                fn()
+                b.record()
+                torch.cuda.synchronize()
+                if it >= 3:
+                    ts.append(a.elapsed_time(b))
+            return statistics.median(ts)
+
+        n = max(5, min(args.steps, 50))
+        f_ms = timed(lambda: ta.fwd(q, k, v, o, lse, w.causal, w.window, w.scale), n)
+        b_ms = timed(lambda: ta.bwd_phases(q, k, v, o, lse, do, dq, dk, dv, ws, w.causal, w.window, w.scale), n)
+        st, site = ta.device_error()
+        if st != 0:
+            raise SystemExit(f"device error {st} at site {site} on {name}")
+        fwd_bytes = (q.numel() + k.numel() + v.numel() + o.numel()) * 2 + lse.numel() * 4
+        print(json.dumps({
+            "workload": name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.Lq, "d": w.d, "causal": w.causal,
+            "window": w.window, "fwd_ms": f_ms, "fwd_tflops": w.fwd_flops() / f_ms / 1e9,
+            "fwd_frac_spec_2250": w.fwd_flops() / f_ms / 1e9 / 2250.0,
+            "fwd_algorithmic_GBs": fwd_bytes / f_ms / 1e6, "hbm_peak_GBs": hbm,
+            "bwd_ms": b_ms, "bwd_tflops": w.bwd_flops() / b_ms / 1e9,
+            "bwd_frac_spec_2250": w.bwd_flops() / b_ms / 1e9 / 2250.0,
+            "peak_sustained_tflops": sustained, "peak_kind": peak_src}), flush=True)
+        del q, k, v, do, o, lse, dq, dk, dv, ws
+        torch.cuda.empty_cache()
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.all_configs:
+        return all_configs(args)
 
     import torch
     if not torch.cuda.is_available():

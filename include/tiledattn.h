@@ -21,9 +21,11 @@
  *  - GQA/MQA ("高效注意力" §3): Hq must be a multiple of Hkv; query head h
  *    reads K/V head h / (Hq / Hkv) (contiguous groups).
  *  - Masks: causal = 1 makes key j visible to query i only if j <= i (top-left
- *    alignment).  window = w > 0 (requires causal = 1) further restricts it to
- *    i - w < j <= i: the w most recent keys including i itself ("高效注意力"
- *    §4, sliding-window attention).  window = 0 means no window.
+ *    alignment).  window = w > 0 further restricts it to a band ("高效注意力"
+ *    §4, sliding-window attention): with causal = 1 to i - w < j <= i (the w
+ *    most recent keys including i itself); with causal = 0 to the two-sided
+ *    band i - w < j < i + w (w - 1 keys on either side of i, and i).
+ *    window = 0 means no window.
  *  - A query row that sees no key gets O = 0 and LSE = -inf (and dQ = 0).
  *  - LSE is the natural logarithm of sum_j exp(scale * q_i . k_j) over visible j.
  *  - Supported head dimension: d = 64 or d = 128 (d_k = d_v = d).

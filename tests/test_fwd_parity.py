@@ -46,6 +46,11 @@ EDGE = [
     (1, 2, 2, 300, 100, 128, True, 50),
     (2, 2, 2, 513, 513, 64, False, 0),
     (1, 4, 2, 1000, 1000, 128, True, 0),
+    # two-sided window (no causal mask): |i - j| < w
+    (1, 2, 2, 257, 257, 128, False, 1),
+    (1, 4, 2, 700, 700, 128, False, 100),
+    (1, 2, 1, 300, 500, 64, False, 130),
+    (1, 2, 2, 500, 300, 128, False, 64),
 ]
 
 

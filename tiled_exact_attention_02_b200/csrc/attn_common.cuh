@@ -3,7 +3,11 @@
 //
 // Visibility ("注意力优化：FlashAttention 与稀疏注意力", 公式速览: disallowed keys
 // get -inf before the softmax; "高效注意力" §4: sliding window):
-//   key j is visible to query i  iff  (!causal || j <= i) && (window <= 0 || j > i - window)
+//   key j is visible to query i  iff  (!causal || j <= i)
+//                                 && (window <= 0 || j > i - window)
+//                                 && (causal || window <= 0 || j < i + window)
+// i.e. a window is the w keys ending at i under a causal mask, and the
+// two-sided band of w - 1 keys on either side of i without one.
 // A tile of keys is skipped when no key in it is visible to any row of the
 // query tile, processed without masking when every key is visible to every
 // row, and masked element-wise otherwise.
@@ -25,7 +29,7 @@ __host__ __device__ inline int cdiv(int a, int b) { return (a + b - 1) / b; }
 
 // Keys [key_lo, key_hi) visible to query row i (may be empty).
 __host__ __device__ inline void row_key_range(const Problem& p, int i, int& key_lo, int& key_hi) {
-  key_hi = p.causal ? imin(p.Lk, i + 1) : p.Lk;
+  key_hi = p.causal ? imin(p.Lk, i + 1) : (p.window > 0 ? imin(p.Lk, i + p.window) : p.Lk);
   key_lo = p.window > 0 ? imax(0, i - p.window + 1) : 0;
 }
 
@@ -35,7 +39,8 @@ __host__ __device__ inline void kv_tile_range(const Problem& p, int q0, int q1, 
   q1 = imin(q1, p.Lq);
   lo = hi = 0;
   if (q0 >= q1) return;
-  const int key_hi = p.causal ? imin(p.Lk, q1) : p.Lk;  // last row sees the most
+  // The last row reaches furthest forward.
+  const int key_hi = p.causal ? imin(p.Lk, q1) : (p.window > 0 ? imin(p.Lk, q1 - 1 + p.window) : p.Lk);
   const int key_lo = p.window > 0 ? imax(0, q0 - p.window + 1) : 0;  // first row reaches furthest back
   if (key_lo >= key_hi) return;
   lo = key_lo / bn;
@@ -47,7 +52,8 @@ __host__ __device__ inline void q_row_range(const Problem& p, int k0, int k1, in
   k1 = imin(k1, p.Lk);
   q_lo = q_hi = 0;
   if (k0 >= k1) return;
-  int lo = p.causal ? k0 : 0;                                  // j <= i  =>  i >= k0
+  // j <= i  =>  i >= k0;  two-sided band: j < i + w  =>  i > k0 - w
+  int lo = p.causal ? k0 : (p.window > 0 ? imax(0, k0 - p.window + 1) : 0);
   int hi = p.window > 0 ? imin(p.Lq, (k1 - 1) + p.window) : p.Lq;  // j > i - w  =>  i < j + w
   if (lo >= hi) return;
   q_lo = lo;
