@@ -6,6 +6,7 @@ product path never calls it and has no CPU fallback.
 """
 
 from .attention import (  # noqa: F401
+    diag_offset,
     visible_mask,
     visible_band,
     attention_weights,

@@ -35,38 +35,50 @@ import numpy as np
 _ROW_BLOCK_ELEMS = 1 << 24
 
 
-def _visible(i, j, causal: bool, window: int) -> np.ndarray:
-    """Elementwise visibility of key j to query i (broadcasting arrays)."""
+def diag_offset(causal, Lq: int, Lk: int) -> int:
+    """Key index of the causal diagonal for query row 0.
+
+    causal = 1 (or True): top-left alignment, query i sees keys j <= i.
+    causal = 2: bottom-right alignment, query i sits at position i + Lk - Lq
+    of the key sequence (the last query row sees the last key), as when new
+    queries attend to a longer cache of earlier keys.
+    """
+    return Lk - Lq if causal == 2 else 0
+
+
+def _visible(i, j, causal, window: int, off: int = 0) -> np.ndarray:
+    """Elementwise visibility of key j to query i (broadcasting arrays);
+    `off` is diag_offset(causal, Lq, Lk)."""
     vis = np.ones(np.broadcast(i, j).shape, dtype=bool)
     if causal:
-        vis &= j <= i
+        vis &= j <= i + off
     if window > 0:
-        vis &= j > i - window
+        vis &= j > i + off - window
         if not causal:
             vis &= j < i + window
     return vis
 
 
-def visible_mask(Lq: int, Lk: int, causal: bool, window: int) -> np.ndarray:
+def visible_mask(Lq: int, Lk: int, causal, window: int) -> np.ndarray:
     """Boolean [Lq, Lk]: True where key j is visible to query i.
 
-    Causal: j <= i.  Window w > 0: the w keys ending at i when causal
-    (i - w < j <= i, "高效注意力" §4 sliding window); without causal the band
-    reaches w - 1 keys to either side, i - w < j < i + w (the two-sided
-    "前后" reading of the same section).
+    Causal: j <= i (causal = 2: j <= i + Lk - Lq).  Window w > 0: the w keys
+    ending at the query's diagonal when causal (i - w < j <= i, "高效注意力" §4
+    sliding window); without causal the band reaches w - 1 keys to either
+    side, i - w < j < i + w (the two-sided "前后" reading of the same section).
     """
-    return _visible(np.arange(Lq)[:, None], np.arange(Lk)[None, :], causal, window)
+    return _visible(np.arange(Lq)[:, None], np.arange(Lk)[None, :], causal, window, diag_offset(causal, Lq, Lk))
 
 
-def visible_band(r0: int, r1: int, Lk: int, causal: bool, window: int) -> tuple[int, int]:
+def visible_band(r0: int, r1: int, Lk: int, causal, window: int, off: int = 0) -> tuple[int, int]:
     """Columns [lo, hi) that can be visible to any row in [r0, r1)."""
     if causal:
-        hi = min(Lk, r1)
+        hi = min(Lk, r1 + off)
     elif window > 0:
         hi = min(Lk, r1 - 1 + window)
     else:
         hi = Lk
-    lo = max(0, r0 - window + 1) if window > 0 else 0
+    lo = max(0, r0 + off - window + 1) if window > 0 else 0
     return lo, max(lo, hi)
 
 
@@ -98,6 +110,7 @@ def attention_weights(q, k, scale: float, vis: np.ndarray):
 def _head_fwd(qh, kh, vh, scale, causal, window, rows=None):
     """O and LSE for the rows `rows` (default: all) of one head."""
     Lq, Lk = qh.shape[0], kh.shape[0]
+    off = diag_offset(causal, Lq, Lk)
     rows = np.arange(Lq) if rows is None else np.asarray(rows)
     O = np.zeros((rows.size, vh.shape[1]))
     lse = np.full(rows.size, -np.inf)
@@ -110,8 +123,8 @@ def _head_fwd(qh, kh, vh, scale, causal, window, rows=None):
         stop = min(rows.size, start + step)
         blk = rows[start:stop]
         r0, r1 = int(blk.min()), int(blk.max()) + 1
-        lo, hi = visible_band(r0, r1, Lk, causal, window)
-        vis = _band_mask(blk, lo, hi, causal, window)
+        lo, hi = visible_band(r0, r1, Lk, causal, window, off)
+        vis = _band_mask(blk, lo, hi, causal, window, off)
         A, l = attention_weights(qh[blk], kh[lo:hi], scale, vis)
         O[start:stop] = A @ vh[lo:hi]
         lse[start:stop] = l
@@ -119,8 +132,8 @@ def _head_fwd(qh, kh, vh, scale, causal, window, rows=None):
     return O, lse
 
 
-def _band_mask(rows, lo, hi, causal, window):
-    return _visible(np.asarray(rows)[:, None], np.arange(lo, hi)[None, :], causal, window)
+def _band_mask(rows, lo, hi, causal, window, off):
+    return _visible(np.asarray(rows)[:, None], np.arange(lo, hi)[None, :], causal, window, off)
 
 
 def _group(Hq: int, Hkv: int) -> int:
@@ -163,12 +176,13 @@ def attn_fwd_rows(q, k, v, scale, causal, window, b, h, rows):
     qh = _f64(q[b, h])
     kh = _f64(k[b, g])
     vh = _f64(v[b, g])
-    Lk = kh.shape[0]
+    Lq, Lk = qh.shape[0], kh.shape[0]
+    off = diag_offset(causal, Lq, Lk)
     O = np.zeros((rows.size, qh.shape[1]))
     lse = np.zeros(rows.size)
     for n, i in enumerate(rows):
-        lo, hi = visible_band(int(i), int(i) + 1, Lk, causal, window)
-        vis = _band_mask([i], lo, hi, causal, window)
+        lo, hi = visible_band(int(i), int(i) + 1, Lk, causal, window, off)
+        vis = _band_mask([i], lo, hi, causal, window, off)
         A, l = attention_weights(qh[i:i + 1], kh[lo:hi], scale, vis)
         O[n] = (A @ vh[lo:hi])[0]
         lse[n] = l[0]
@@ -178,9 +192,10 @@ def attn_fwd_rows(q, k, v, scale, causal, window, b, h, rows):
 def _rows_bwd(qh, kh, vh, doh, scale, causal, window, r0, r1):
     """Rows [r0, r1) of one head: their O and LSE, their dQ rows, and their
     contributions to dK and dV over the visible key band [lo, hi)."""
-    Lk = kh.shape[0]
-    lo, hi = visible_band(r0, r1, Lk, causal, window)
-    vis = _band_mask(np.arange(r0, r1), lo, hi, causal, window)
+    Lq, Lk = qh.shape[0], kh.shape[0]
+    off = diag_offset(causal, Lq, Lk)
+    lo, hi = visible_band(r0, r1, Lk, causal, window, off)
+    vis = _band_mask(np.arange(r0, r1), lo, hi, causal, window, off)
     A, lse = attention_weights(qh[r0:r1], kh[lo:hi], scale, vis)
     O = A @ vh[lo:hi]
     dO = doh[r0:r1]

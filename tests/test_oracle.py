@@ -133,6 +133,51 @@ def test_two_sided_window_counts_and_band():
         assert lo == cols.min() and hi == cols.max() + 1
 
 
+def test_bottom_right_causal_equals_top_left_when_square():
+    """causal = 2 aligns the last query with the last key; with Lq = Lk that is causal = 1."""
+    L, d = 13, 4
+    q, k, v = _rand(1, 2, L, d), _rand(1, 2, L, d), _rand(1, 2, L, d)
+    for w in (0, 5):
+        a = oracle.attn_fwd(q, k, v, 0.4, 1, w)
+        b = oracle.attn_fwd(q, k, v, 0.4, 2, w)
+        for x, y in zip(a, b):
+            assert np.array_equal(x, y)
+
+
+def test_bottom_right_causal_is_a_suffix_of_the_square_case():
+    """Queries Q over keys K with causal = 2 give the last Lq rows of causal = 1
+    attention of [P; Q] over K, whatever the prefix rows P (the queries sit at
+    positions Lk - Lq .. Lk - 1)."""
+    Lq, Lk, d = 5, 17, 6
+    q, k, v = _rand(1, 1, Lq, d), _rand(1, 1, Lk, d), _rand(1, 1, Lk, d)
+    pre = _rand(1, 1, Lk - Lq, d)
+    full = np.concatenate([pre, q], 2)
+    for w in (0, 3, 40):
+        O, lse = oracle.attn_fwd(q, k, v, 0.3, 2, w)
+        Of, lf = oracle.attn_fwd(full, k, v, 0.3, 1, w)
+        np.testing.assert_allclose(O, Of[:, :, Lk - Lq:], atol=1e-14)
+        np.testing.assert_allclose(lse, lf[:, :, Lk - Lq:], atol=1e-14)
+
+
+def test_bottom_right_single_query_sees_every_key():
+    """A single query aligned to the last key sees the whole cache (no window)."""
+    Lk, d = 21, 5
+    q, k, v = _rand(1, 1, 1, d), _rand(1, 1, Lk, d), _rand(1, 1, Lk, d)
+    np.testing.assert_allclose(oracle.attn_fwd(q, k, v, 0.5, 2, 0)[0], oracle.attn_fwd(q, k, v, 0.5, False, 0)[0],
+                               atol=1e-14)
+
+
+def test_bottom_right_with_more_queries_than_keys():
+    """Lq > Lk with causal = 2: the first Lq - Lk rows see no key (O = 0, LSE = -inf, dQ = 0)."""
+    Lq, Lk, d = 9, 4, 3
+    q, k, v, do = _rand(1, 1, Lq, d), _rand(1, 1, Lk, d), _rand(1, 1, Lk, d), _rand(1, 1, Lq, d)
+    O, lse = oracle.attn_fwd(q, k, v, 0.5, 2, 0)
+    assert np.all(O[0, 0, :Lq - Lk] == 0) and np.all(np.isneginf(lse[0, 0, :Lq - Lk]))
+    assert np.all(np.isfinite(lse[0, 0, Lq - Lk:]))
+    dq, _, _ = oracle.attn_bwd(q, k, v, do, 0.5, 2, 0)
+    assert np.all(dq[0, 0, :Lq - Lk] == 0)
+
+
 def test_value_shift_and_score_shift_invariance():
     """V + 1 c^T gives O + 1 c^T; a per-row constant added to the logits changes nothing."""
     L, d = 19, 4
@@ -219,16 +264,18 @@ def _loss(q, k, v, R, scale, causal, window):
 
 @pytest.mark.parametrize("Hq,Hkv,L,causal,window", [
     (2, 2, 9, False, 0), (2, 2, 9, True, 0), (2, 1, 8, True, 3), (2, 2, 7, True, 1),
-    (4, 2, 6, False, 0), (2, 1, 9, False, 3),
+    (4, 2, 6, False, 0), (2, 1, 9, False, 3), (2, 1, -5, 2, 0), (2, 2, -4, 2, 3),
 ])
 def test_backward_matches_finite_differences(Hq, Hkv, L, causal, window):
-    """Gradient of <R, O> against central differences, float64, to 1e-6."""
+    """Gradient of <R, O> against central differences, float64, to 1e-6.
+    A negative L is a rectangular case: Lq = |L| queries over Lk = |L| + 4 keys."""
     rng = np.random.default_rng(7)
     d = 4
-    q = rng.standard_normal((1, Hq, L, d))
-    k = rng.standard_normal((1, Hkv, L, d))
-    v = rng.standard_normal((1, Hkv, L, d))
-    R = rng.standard_normal((1, Hq, L, d))
+    Lq, Lk = (L, L) if L > 0 else (-L, -L + 4)
+    q = rng.standard_normal((1, Hq, Lq, d))
+    k = rng.standard_normal((1, Hkv, Lk, d))
+    v = rng.standard_normal((1, Hkv, Lk, d))
+    R = rng.standard_normal((1, Hq, Lq, d))
     scale = 0.6
     dq, dk, dv = oracle.attn_bwd(q, k, v, R, scale, causal, window)
     eps = 1e-5
@@ -318,6 +365,25 @@ def test_matches_torch_sdpa_float64(Hq, Hkv, causal, window):
     mask = torch.from_numpy(oracle.visible_mask(L, L, causal, window))
     ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=mask, scale=0.25)
     np.testing.assert_allclose(O, ref.numpy(), atol=1e-12)
+
+
+@pytest.mark.parametrize("Lq,Lk,w", [(7, 30, 0), (30, 30, 0), (12, 40, 6), (40, 12, 0)])
+def test_bottom_right_causal_matches_torch_sdpa(Lq, Lk, w):
+    """causal = 2 against torch SDPA with a lower-triangular mask shifted by Lk - Lq
+    (built here with torch.tril), and the window as a band below it.  Rows
+    with no visible key are compared as zeros (SDPA returns NaN there)."""
+    B, Hq, Hkv, d = 1, 2, 1, 8
+    q, k, v = _rand(B, Hq, Lq, d), _rand(B, Hkv, Lk, d), _rand(B, Hkv, Lk, d)
+    O, _ = oracle.attn_fwd(q, k, v, 0.3, 2, w)
+    mask = torch.ones(Lq, Lk, dtype=torch.bool).tril(diagonal=Lk - Lq)
+    if w > 0:
+        mask &= ~torch.ones(Lq, Lk, dtype=torch.bool).tril(diagonal=Lk - Lq - w)
+    tq, tk, tv = (torch.from_numpy(x) for x in (q, k, v))
+    tk, tv = tk.repeat_interleave(Hq // Hkv, 1), tv.repeat_interleave(Hq // Hkv, 1)
+    ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=mask, scale=0.3).numpy()
+    dead = ~mask.any(1).numpy()
+    ref[:, :, dead] = 0.0
+    np.testing.assert_allclose(O, ref, atol=1e-12)
 
 
 @pytest.mark.parametrize("w", [1, 4, 40])
