@@ -21,11 +21,15 @@
  *  - GQA/MQA ("高效注意力" §3): Hq must be a multiple of Hkv; query head h
  *    reads K/V head h / (Hq / Hkv) (contiguous groups).
  *  - Masks: causal = 1 makes key j visible to query i only if j <= i (top-left
- *    alignment).  window = w > 0 further restricts it to a band ("高效注意力"
- *    §4, sliding-window attention): with causal = 1 to i - w < j <= i (the w
- *    most recent keys including i itself); with causal = 0 to the two-sided
- *    band i - w < j < i + w (w - 1 keys on either side of i, and i).
- *    window = 0 means no window.
+ *    alignment); causal = 2 only if j <= i + Lk - Lq (bottom-right alignment:
+ *    the last query sits at the last key, as for new queries over a longer
+ *    cache of earlier keys; the same as causal = 1 when Lq = Lk).  window =
+ *    w > 0 further restricts it to a band ("高效注意力" §4, sliding-window
+ *    attention): with causal to the w keys ending at the query's diagonal
+ *    (i + off - w < j <= i + off, off = 0 or Lk - Lq); with causal = 0 to the
+ *    two-sided band i - w < j < i + w (w - 1 keys on either side of i, and
+ *    i).  window = 0 means no window.  causal outside {0, 1, 2} or window < 0
+ *    is ATTN_ERR_INVALID_ARG.
  *  - A query row that sees no key gets O = 0 and LSE = -inf (and dQ = 0).
  *  - LSE is the natural logarithm of sum_j exp(scale * q_i . k_j) over visible j.
  *  - Supported head dimension: d = 64 or d = 128 (d_k = d_v = d).

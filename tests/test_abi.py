@@ -55,8 +55,8 @@ def _fwd(ta, B=1, Hq=2, Hkv=2, Lq=8, Lk=8, d=64, scale=0.125, causal=0, window=0
 
 @pytest.mark.parametrize("kw,status", [
     (dict(d=96), 2), (dict(d=256), 2), (dict(Hq=3, Hkv=2), 1), (dict(Hkv=0), 1),
-    (dict(B=-1), 1), (dict(Lq=-5), 1), (dict(causal=1, window=-1), 1),
-    (dict(causal=2), 1), (dict(scale=0.0), 1), (dict(scale=-1.0), 1), (dict(scale=float("nan")), 1),
+    (dict(B=-1), 1), (dict(Lq=-5), 1), (dict(causal=1, window=-1), 1), (dict(causal=3), 1), (dict(causal=-1), 1),
+    (dict(scale=0.0), 1), (dict(scale=-1.0), 1), (dict(scale=float("nan")), 1),
     (dict(scale=float("inf")), 1), (dict(q=0), 1), (dict(o=P + 8), 1), (dict(lse=P + 4), 1),
     (dict(k=0), 1), (dict(v=P + 2), 1),
 ])
@@ -75,7 +75,7 @@ def _bwd(ta, B=1, Hq=2, Hkv=1, Lq=8, Lk=8, d=128, scale=0.1, causal=1, window=0,
 
 
 @pytest.mark.parametrize("kw,status", [
-    (dict(d=80), 2), (dict(Hq=3, Hkv=2), 1), (dict(window=-3, causal=0), 1), (dict(ws=0), 1),
+    (dict(d=80), 2), (dict(Hq=3, Hkv=2), 1), (dict(window=-3, causal=0), 1), (dict(causal=3), 1), (dict(ws=0), 1),
     (dict(wsb=16), 1), (dict(ptrs=[P] * 5 + [0] + [P] * 3), 1), (dict(ptrs=[P] * 8 + [P + 1]), 1),
     (dict(scale=0.0), 1), (dict(ws=P + 64), 1),
 ])
@@ -100,3 +100,12 @@ def test_binding_has_no_cpu_path(ta):
     src = open(os.path.join(ROOT, "tiled_exact_attention_02_b200", "__init__.py")).read()
     for banned in ("softmax", "oracle", "matmul", "@", "scaled_dot_product"):
         assert banned not in src.replace("@staticmethod", ""), banned
+
+
+def test_causal_argument_codes(ta):
+    """The binding maps the causal argument to the ABI code (0 none, 1 top-left, 2 bottom-right)."""
+    f = ta._causal_code
+    assert [f(x) for x in (False, True, 0, 1, 2)] == [0, 1, 0, 1, 2]
+    assert [f(x) for x in ("none", "top_left", "bottom_right")] == [0, 1, 2]
+    with pytest.raises(ValueError):
+        f("diagonal")

@@ -51,6 +51,12 @@ EDGE = [
     (1, 4, 2, 700, 700, 128, False, 100),
     (1, 2, 1, 300, 500, 64, False, 130),
     (1, 2, 2, 500, 300, 128, False, 64),
+    # bottom-right causal (causal = 2): query i at key position i + Lk - Lq
+    (1, 2, 2, 100, 333, 128, 2, 0),
+    (1, 4, 2, 1, 1000, 128, 2, 0),
+    (2, 2, 1, 333, 100, 64, 2, 0),
+    (1, 2, 2, 200, 700, 128, 2, 64),
+    (1, 4, 4, 129, 129, 128, 2, 0),
 ]
 
 

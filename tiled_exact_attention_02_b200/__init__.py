@@ -98,6 +98,17 @@ def _require(t, name, dtype=None):
         raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
 
 
+def _causal_code(causal) -> int:
+    """The ABI's mask code: False/0 none, True/1 top-left, 2 or "bottom_right"
+    bottom-right alignment (query i at key position i + Lk - Lq)."""
+    if isinstance(causal, str):
+        codes = {"none": 0, "top_left": 1, "bottom_right": 2}
+        if causal not in codes:
+            raise ValueError(f"causal must be one of {sorted(codes)}, got {causal!r}")
+        return codes[causal]
+    return 2 if causal == 2 and not isinstance(causal, bool) else int(bool(causal))
+
+
 def fwd(q, k, v, o, lse, causal: bool = False, window: int = 0, scale: float | None = None, stream=None):
     """attn_fwd on torch tensors (bf16 q/k/v/o, fp32 lse), asynchronous on `stream`."""
     import torch
@@ -109,7 +120,7 @@ def fwd(q, k, v, o, lse, causal: bool = False, window: int = 0, scale: float | N
         raise ValueError("v/o/lse shape mismatch")
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     st = lib.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                      B, Hq, Hkv, Lq, Lk, d, scale, int(bool(causal)), int(window), _stream_ptr(stream))
+                      B, Hq, Hkv, Lq, Lk, d, scale, _causal_code(causal), int(window), _stream_ptr(stream))
     _check(st, "attn_fwd")
 
 
@@ -129,7 +140,7 @@ def bwd(q, k, v, o, lse, do, dq, dk, dv, workspace, causal: bool = False, window
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     st = lib.attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
                       dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv, Lq, Lk, d, scale,
-                      int(bool(causal)), int(window), workspace.data_ptr(),
+                      _causal_code(causal), int(window), workspace.data_ptr(),
                       workspace.numel() * workspace.element_size(), _stream_ptr(stream))
     _check(st, "attn_bwd")
 
@@ -146,7 +157,7 @@ def bwd_phases(q, k, v, o, lse, do, dq, dk, dv, workspace, causal: bool = False,
     _check(lib.attn_bwd_preprocess(o.data_ptr(), do.data_ptr(), B, Hq, Lq, d, ws, wsb, sp), "attn_bwd_preprocess")
     hook(1)
     _check(lib.attn_bwd_main(q.data_ptr(), k.data_ptr(), v.data_ptr(), lse.data_ptr(), do.data_ptr(),
-                             dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv, Lq, Lk, d, scale, int(bool(causal)),
+                             dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv, Lq, Lk, d, scale, _causal_code(causal),
                              int(window), ws, wsb, sp), "attn_bwd_main")
     hook(2)
     _check(lib.attn_bwd_finalize(dq.data_ptr(), B, Hq, Lq, d, scale, ws, wsb, sp), "attn_bwd_finalize")

@@ -83,7 +83,7 @@ int check_shape(int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale, int 
   if (Hkv == 0 && Hq > 0) return ATTN_ERR_INVALID_ARG;
   if (Hkv > 0 && Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
   if (Hq == 0 && Hkv > 0) return ATTN_ERR_INVALID_ARG;
-  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (causal < 0 || causal > 2) return ATTN_ERR_INVALID_ARG;
   if (window < 0) return ATTN_ERR_INVALID_ARG;
   if (!std::isfinite(scale) || scale <= 0.f) return ATTN_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;

@@ -321,8 +321,9 @@ __device__ void grad_rows(const BwdParams& P, const Unit& u, uint8_t* smem, Bars
   // Queries [vis_lo, vis_hi) see this key.
   int vis_lo = 0, vis_hi = 0;
   if (key < p.Lk) {
-    vis_lo = p.causal ? key : (p.window > 0 ? imax(0, key - p.window + 1) : 0);
-    vis_hi = p.window > 0 ? imin(p.Lq, key + p.window) : p.Lq;
+    const int off = diag_off(p);
+    vis_lo = p.causal ? imax(0, key - off) : (p.window > 0 ? imax(0, key - p.window + 1) : 0);
+    vis_hi = p.window > 0 ? imin(p.Lq, key - off + p.window) : p.Lq;
   }
   const float c = P.scale_log2;
   float* vec = reinterpret_cast<float*>(smem + C::OFF_VEC) + grp * (2 * 2 * CW);

@@ -2,12 +2,14 @@
 // the forward and backward kernels and their host-side launchers.
 //
 // Visibility ("注意力优化：FlashAttention 与稀疏注意力", 公式速览: disallowed keys
-// get -inf before the softmax; "高效注意力" §4: sliding window):
-//   key j is visible to query i  iff  (!causal || j <= i)
-//                                 && (window <= 0 || j > i - window)
+// get -inf before the softmax; "高效注意力" §4: sliding window).  With
+// off = Lk - Lq for causal = 2 (bottom-right alignment: query i sits at key
+// position i + Lk - Lq) and off = 0 otherwise,
+//   key j is visible to query i  iff  (!causal || j <= i + off)
+//                                 && (window <= 0 || j > i + off - window)
 //                                 && (causal || window <= 0 || j < i + window)
-// i.e. a window is the w keys ending at i under a causal mask, and the
-// two-sided band of w - 1 keys on either side of i without one.
+// i.e. a window is the w keys ending at the query's diagonal under a causal
+// mask, and the two-sided band of w - 1 keys on either side of i without one.
 // A tile of keys is skipped when no key in it is visible to any row of the
 // query tile, processed without masking when every key is visible to every
 // row, and masked element-wise otherwise.
@@ -19,7 +21,7 @@ namespace tea {
 
 struct Problem {
   int B, Hq, Hkv, Lq, Lk, d;
-  int causal, window;
+  int causal, window;  // causal: 0 none, 1 top-left, 2 bottom-right
   float scale;
 };
 
@@ -27,10 +29,14 @@ __host__ __device__ inline int imin(int a, int b) { return a < b ? a : b; }
 __host__ __device__ inline int imax(int a, int b) { return a > b ? a : b; }
 __host__ __device__ inline int cdiv(int a, int b) { return (a + b - 1) / b; }
 
-// Keys [key_lo, key_hi) visible to query row i (may be empty).
+// Key index of query row 0's causal diagonal.
+__host__ __device__ inline int diag_off(const Problem& p) { return p.causal == 2 ? p.Lk - p.Lq : 0; }
+
+// Keys [key_lo, key_hi) visible to query row i (empty when key_lo >= key_hi).
 __host__ __device__ inline void row_key_range(const Problem& p, int i, int& key_lo, int& key_hi) {
-  key_hi = p.causal ? imin(p.Lk, i + 1) : (p.window > 0 ? imin(p.Lk, i + p.window) : p.Lk);
-  key_lo = p.window > 0 ? imax(0, i - p.window + 1) : 0;
+  const int off = diag_off(p);
+  key_hi = p.causal ? imin(p.Lk, i + off + 1) : (p.window > 0 ? imin(p.Lk, i + p.window) : p.Lk);
+  key_lo = p.window > 0 ? imax(0, i + off - p.window + 1) : 0;
 }
 
 // Key tiles [lo, hi) (tiles of bn keys) holding any key visible to any query
@@ -39,9 +45,10 @@ __host__ __device__ inline void kv_tile_range(const Problem& p, int q0, int q1, 
   q1 = imin(q1, p.Lq);
   lo = hi = 0;
   if (q0 >= q1) return;
-  // The last row reaches furthest forward.
-  const int key_hi = p.causal ? imin(p.Lk, q1) : (p.window > 0 ? imin(p.Lk, q1 - 1 + p.window) : p.Lk);
-  const int key_lo = p.window > 0 ? imax(0, q0 - p.window + 1) : 0;  // first row reaches furthest back
+  const int off = diag_off(p);
+  // The last row reaches furthest forward, the first row furthest back.
+  const int key_hi = p.causal ? imin(p.Lk, q1 + off) : (p.window > 0 ? imin(p.Lk, q1 - 1 + p.window) : p.Lk);
+  const int key_lo = p.window > 0 ? imax(0, q0 + off - p.window + 1) : 0;
   if (key_lo >= key_hi) return;
   lo = key_lo / bn;
   hi = cdiv(key_hi, bn);
@@ -52,9 +59,11 @@ __host__ __device__ inline void q_row_range(const Problem& p, int k0, int k1, in
   k1 = imin(k1, p.Lk);
   q_lo = q_hi = 0;
   if (k0 >= k1) return;
-  // j <= i  =>  i >= k0;  two-sided band: j < i + w  =>  i > k0 - w
-  int lo = p.causal ? k0 : (p.window > 0 ? imax(0, k0 - p.window + 1) : 0);
-  int hi = p.window > 0 ? imin(p.Lq, (k1 - 1) + p.window) : p.Lq;  // j > i - w  =>  i < j + w
+  const int off = diag_off(p);
+  // j <= i + off  =>  i >= k0 - off;  two-sided band: j < i + w  =>  i > k0 - w
+  int lo = p.causal ? imax(0, k0 - off) : (p.window > 0 ? imax(0, k0 - p.window + 1) : 0);
+  // j > i + off - w  =>  i < j - off + w
+  int hi = p.window > 0 ? imin(p.Lq, (k1 - 1) - off + p.window) : p.Lq;
   if (lo >= hi) return;
   q_lo = lo;
   q_hi = hi;
