@@ -255,6 +255,13 @@ def all_configs(args):
 
         n = max(5, min(args.steps, 50))
         f_ms = timed(lambda: ta.fwd(q, k, v, o, lse, w.causal, w.window, w.scale), n)
+        ns = ta.lib.attn_fwd_split_default(w.B, w.Hq, w.Hkv, w.Lq, w.Lk, w.d, ta._causal_code(w.causal), w.window)
+        split = None
+        if ns > 1:
+            sws = torch.empty(max(256, ta.lib.attn_fwd_split_workspace_size(w.B, w.Hq, w.Hkv, w.Lq, w.Lk, w.d, ns)),
+                              dtype=torch.uint8, device="cuda")
+            s_ms = timed(lambda: ta.fwd_split(q, k, v, o, lse, ns, sws, w.causal, w.window, w.scale), n)
+            split = {"n_split": ns, "fwd_ms": s_ms, "fwd_tflops": w.fwd_flops() / s_ms / 1e9}
         b_ms = timed(lambda: ta.bwd_phases(q, k, v, o, lse, do, dq, dk, dv, ws, w.causal, w.window, w.scale), n)
         st, site = ta.device_error()
         if st != 0:
@@ -265,6 +272,7 @@ def all_configs(args):
             "window": w.window, "fwd_ms": f_ms, "fwd_tflops": w.fwd_flops() / f_ms / 1e9,
             "fwd_frac_spec_2250": w.fwd_flops() / f_ms / 1e9 / 2250.0,
             "fwd_algorithmic_GBs": fwd_bytes / f_ms / 1e6, "hbm_peak_GBs": hbm,
+            "fwd_split": None if split is None else dict(split, fwd_algorithmic_GBs=fwd_bytes / split["fwd_ms"] / 1e6),
             "bwd_ms": b_ms, "bwd_tflops": w.bwd_flops() / b_ms / 1e9,
             "bwd_frac_spec_2250": w.bwd_flops() / b_ms / 1e9 / 2250.0,
             "peak_sustained_tflops": sustained, "peak_kind": peak_src}), flush=True)

@@ -87,6 +87,38 @@ ATTN_API int attn_fwd(const void* q, const void* k, const void* v, void* o, floa
              int Lk, int d, float scale, int causal, int window, void* stream);
 
 /*
+ * Forward pass with the key range split across CTAs (for few query rows over
+ * many keys, e.g. new queries over a long cache with causal = 2).  Each query
+ * tile's visible key tiles are cut into n_split contiguous slices, each
+ * computed by its own CTA into an fp32 partial (O normalised by the slice's
+ * own sum, and the slice's LSE).  A second kernel then combines the slices
+ * exactly, with weights exp(LSE_k - max_k LSE_k): the online-softmax merge of
+ * "高效注意力：FlashAttention 与线性注意力" 原理与机制 applied to whole slices.
+ * The result equals attn_fwd's up to rounding.
+ *
+ *  q, k, v, o, lse, sizes, scale, causal, window: as attn_fwd.
+ *  n_split    1..64 slices (1: plain attn_fwd, the workspace is not used).
+ *  workspace  caller-owned device memory, 256-byte aligned, at least
+ *             attn_fwd_split_workspace_size(...) bytes; overwritten.
+ *
+ * Returns ATTN_OK or an attn_status error code (n_split out of range or a
+ * short / misaligned workspace: ATTN_ERR_INVALID_ARG).
+ */
+ATTN_API int attn_fwd_split(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                            int Lq, int Lk, int d, float scale, int causal, int window, int n_split, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
+/* Workspace bytes attn_fwd_split needs: n_split x (fp32 O [B,Hq,Lq,d] + fp32
+ * LSE [B,Hq,Lq]), each part padded to 256 bytes.  0 for n_split = 1, an empty
+ * problem or invalid sizes. */
+ATTN_API size_t attn_fwd_split_workspace_size(int B, int Hq, int Hkv, int Lq, int Lk, int d, int n_split);
+
+/* A slice count for this problem on the current device: enough CTAs to cover
+ * every SM about twice, no slice shorter than two 128-key tiles, at most 64;
+ * 1 when splitting would not help.  Host-only (no launch). */
+ATTN_API int attn_fwd_split_default(int B, int Hq, int Hkv, int Lq, int Lk, int d, int causal, int window);
+
+/*
  * Bytes of device workspace attn_bwd needs for this shape: the per-row
  * D_i = dO_i . O_i (fp32 [B,Hq,Lq]) and an fp32 dQ accumulator [B,Hq,Lq,d].
  * Returns 0 for an empty problem or invalid sizes.

@@ -16,6 +16,9 @@ Mistral example on the same page):
   gqa_causal_8192   B=4, Hq=32/Hkv=8, L=8192, d=128, causal, Q scaled by 2
   gqa_window_32768  B=1, Hq=32/Hkv=8, L=32768, d=128, causal window 4096
   mha_causal_fwdbwd B=2, Hq=Hkv=32,  L=4096,  d=128, causal, plus dO
+  gqa_decode_32768  B=4, Hq=32/Hkv=8, Lq=16 over Lk=32768, d=128, bottom-right
+                    causal (new queries over a long cache, the KV-cache
+                    setting of "高效注意力" §3)
 """
 
 from dataclasses import dataclass, field
@@ -33,8 +36,8 @@ class Workload:
     Lq: int
     Lk: int
     d: int
-    causal: bool
-    window: int = 0          # 0: no window; >0: key j visible iff i-window < j <= i
+    causal: int              # 0 none, 1 top-left (j <= i), 2 bottom-right (j <= i + Lk - Lq)
+    window: int = 0          # 0: no window; >0: causal band of w keys, or |i - j| < w without causal
     q_mult: float = 1.0      # applied after bf16 rounding (a power of two: exact)
     backward: bool = False
     seed: int = 42
@@ -45,10 +48,14 @@ class Workload:
 
     def visible_pairs_per_head(self) -> int:
         """Number of (i, j) pairs with key j visible to query i."""
+        off = self.Lk - self.Lq if self.causal == 2 else 0
         total = 0
         for i in range(self.Lq):
-            hi = min(i + 1, self.Lk) if self.causal else self.Lk
-            lo = max(0, i - self.window + 1) if self.window > 0 else 0
+            if self.causal:
+                hi = min(i + off + 1, self.Lk)
+            else:
+                hi = min(i + self.window, self.Lk) if self.window > 0 else self.Lk
+            lo = max(0, i + off - self.window + 1) if self.window > 0 else 0
             total += max(0, hi - lo)
         return total
 
@@ -69,6 +76,8 @@ WORKLOADS = {
         Workload("gqa_causal_8192", 4, 32, 8, 8192, 8192, 128, True, q_mult=2.0, seed=44),
         Workload("gqa_window_32768", 1, 32, 8, 32768, 32768, 128, True, window=4096, seed=45),
         Workload("mha_causal_fwdbwd", 2, 32, 32, 4096, 4096, 128, True, backward=True, seed=46),
+        # 16 new queries per sequence over a 32768-key cache (bottom-right causal)
+        Workload("gqa_decode_32768", 4, 32, 8, 16, 32768, 128, 2, seed=47),
     ]
 }
 

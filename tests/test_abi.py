@@ -95,6 +95,39 @@ def test_bwd_workspace_size(ta):
     assert ta.bwd_workspace_size(1, 4, 2, 100, 50, 72) == 0
 
 
+def test_fwd_split_workspace_size(ta):
+    """n_split x (fp32 O rows x d + fp32 LSE rows), each part padded to 256 bytes; 0 for one slice."""
+    ws = ta.lib.attn_fwd_split_workspace_size
+    rows = 1 * 2 * 10
+    assert ws(1, 2, 2, 10, 300, 64, 4) == -(-4 * rows * 64 * 4 // 256) * 256 + -(-4 * rows * 4 // 256) * 256
+    assert ws(1, 2, 2, 10, 300, 64, 1) == 0
+    assert ws(1, 2, 2, 10, 300, 64, 0) == 0 and ws(1, 2, 2, 10, 300, 64, 65) == 0
+    assert ws(0, 2, 2, 10, 300, 64, 4) == 0
+
+
+def test_fwd_split_default_is_in_range(ta):
+    d = ta.lib.attn_fwd_split_default
+    assert d(1, 8, 2, 1, 32768, 128, 2, 0) > 1          # a decode problem splits
+    assert 1 <= d(8, 32, 8, 1, 32768, 128, 2, 0) <= 64
+    assert d(2, 32, 32, 4096, 4096, 128, 1, 0) == 1     # a full grid does not
+    assert d(1, 2, 2, 1, 100, 64, 2, 0) == 1            # a single key tile does not
+
+
+def _split(ta, n_split=4, ws=P, wsb=1 << 20, **kw):
+    a = dict(B=1, Hq=2, Hkv=2, Lq=8, Lk=300, d=64, scale=0.125, causal=2, window=0)
+    a.update(kw)
+    return ta.lib.attn_fwd_split(P, P, P, P, P, a["B"], a["Hq"], a["Hkv"], a["Lq"], a["Lk"], a["d"], a["scale"],
+                                 a["causal"], a["window"], n_split, ws, wsb, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(n_split=0), 1), (dict(n_split=65), 1), (dict(wsb=64), 1), (dict(ws=0), 1), (dict(ws=P + 16), 1),
+    (dict(causal=3), 1), (dict(d=80), 2), (dict(Hq=3, Hkv=2), 1),
+])
+def test_fwd_split_rejects_bad_arguments(ta, kw, status):
+    assert _split(ta, **kw) == status
+
+
 def test_binding_has_no_cpu_path(ta):
     """The binding only marshals: no numpy/torch attention math in the package."""
     src = open(os.path.join(ROOT, "tiled_exact_attention_02_b200", "__init__.py")).read()

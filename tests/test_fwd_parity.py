@@ -70,6 +70,32 @@ def test_fwd_edge_shapes(ta, B, Hq, Hkv, Lq, Lk, d, causal, window):
     check_lse(lse, rl, "LSE")
 
 
+# (B, Hq, Hkv, Lq, Lk, d, causal, window, n_split); n_split None: the library's choice
+SPLIT = [
+    (2, 8, 2, 1, 3000, 128, 2, 0, 8),
+    (1, 4, 4, 64, 2048, 64, 2, 500, 5),
+    (1, 2, 2, 300, 300, 128, 1, 0, 3),
+    (1, 2, 1, 17, 5000, 128, 2, 0, None),
+    (1, 2, 2, 200, 100, 128, 2, 0, 7),
+    (1, 2, 2, 100, 900, 128, 0, 64, 4),
+    (1, 2, 2, 50, 700, 128, 0, 0, 64),
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Lq,Lk,d,causal,window,n_split", SPLIT)
+def test_fwd_split_kv(ta, B, Hq, Hkv, Lq, Lk, d, causal, window, n_split):
+    """Split-KV forward (slices merged by their LSE) against the oracle."""
+    x = make_shape_inputs(B, Hq, Hkv, Lq, Lk, d, seed=Lq * 5 + Lk + d + 3)
+    scale = d ** -0.5
+    q, k, v = (to_dev(x[n]) for n in "qkv")
+    o, lse = ta.attention_split(q, k, v, causal, window, scale, n_split)
+    st, site = ta.device_error()
+    assert st == 0, f"device error {st} at site {site}"
+    ro, rl = oracle.attn_fwd(x["q"], x["k"], x["v"], scale, causal, window)
+    check_o(to_f64(o), ro, "O")
+    check_lse(to_f64(lse), rl, "LSE")
+
+
 def test_fwd_no_keys(ta):
     """Lk = 0: every row sees nothing: O = 0, LSE = -inf."""
     import torch

@@ -40,6 +40,12 @@ def _load() -> ctypes.CDLL:
     vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     lib.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, vp]
     lib.attn_fwd.restype = i
+    lib.attn_fwd_split.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i, vp, sz, vp]
+    lib.attn_fwd_split.restype = i
+    lib.attn_fwd_split_workspace_size.argtypes = [i, i, i, i, i, i, i]
+    lib.attn_fwd_split_workspace_size.restype = sz
+    lib.attn_fwd_split_default.argtypes = [i, i, i, i, i, i, i, i]
+    lib.attn_fwd_split_default.restype = i
     lib.attn_bwd_workspace_size.argtypes = [i, i, i, i, i, i]
     lib.attn_bwd_workspace_size.restype = sz
     lib.attn_bwd.argtypes = [vp] * 9 + [i] * 6 + [f, i, i, vp, sz, vp]
@@ -178,6 +184,35 @@ def attention(q, k, v, causal: bool = False, window: int = 0, scale: float | Non
     o = torch.empty_like(q)
     lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
     fwd(q, k, v, o, lse, causal, window, scale)
+    return o, lse
+
+
+def fwd_split(q, k, v, o, lse, n_split: int, workspace, causal: bool = False, window: int = 0,
+              scale: float | None = None, stream=None):
+    """attn_fwd_split: the key range of every query tile cut into n_split
+    slices computed by separate CTAs, then merged exactly."""
+    B, Hq, Hkv, Lq, Lk, d = _shapes(q, k)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    ws = workspace.data_ptr() if workspace is not None else None
+    wsb = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib.attn_fwd_split(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                              B, Hq, Hkv, Lq, Lk, d, scale, _causal_code(causal), int(window), int(n_split), ws, wsb,
+                              _stream_ptr(stream)), "attn_fwd_split")
+
+
+def attention_split(q, k, v, causal: bool = False, window: int = 0, scale: float | None = None,
+                    n_split: int | None = None):
+    """Allocate O, LSE and the workspace with torch and run the split-KV
+    forward (n_split None: the library's suggestion for this shape)."""
+    import torch
+    B, Hq, Hkv, Lq, Lk, d = _shapes(q, k)
+    if n_split is None:
+        n_split = lib.attn_fwd_split_default(B, Hq, Hkv, Lq, Lk, d, _causal_code(causal), int(window))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
+    nbytes = lib.attn_fwd_split_workspace_size(B, Hq, Hkv, Lq, Lk, d, int(n_split))
+    ws = torch.empty(max(256, nbytes), dtype=torch.uint8, device=q.device)
+    fwd_split(q, k, v, o, lse, n_split, ws, causal, window, scale)
     return o, lse
 
 

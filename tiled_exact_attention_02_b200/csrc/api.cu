@@ -169,6 +169,76 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   return e == cudaSuccess ? ATTN_OK : cuda_fail("attn_fwd launch", e);
 }
 
+// ------------------------------------------------------------------ split-KV forward
+static constexpr int kMaxSplit = 64;
+
+size_t attn_fwd_split_workspace_size(int B, int Hq, int Hkv, int Lq, int Lk, int d, int n_split) {
+  if (check_shape(B, Hq, Hkv, Lq, Lk, d, 1.f, 0, 0) != ATTN_OK) return 0;
+  if (n_split < 1 || n_split > kMaxSplit || B == 0 || Hq == 0 || Lq == 0) return 0;
+  if (n_split == 1) return 0;
+  const size_t rows = (size_t)B * Hq * Lq;
+  return ((size_t)n_split * rows * d * 4 + 255) / 256 * 256 + ((size_t)n_split * rows * 4 + 255) / 256 * 256;
+}
+
+int attn_fwd_split_default(int B, int Hq, int Hkv, int Lq, int Lk, int d, int causal, int window) {
+  if (check_shape(B, Hq, Hkv, Lq, Lk, d, 1.f, causal, window) != ATTN_OK) return 1;
+  if (B == 0 || Hq == 0 || Lq == 0 || Lk == 0) return 1;
+  Problem p{B, Hq, Hkv, Lq, Lk, d, causal, window, 1.f};
+  int n_units, pair;
+  fwd_plan(p, &n_units, &pair);
+  int sms = 148;
+  int dev;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // Enough slices that the grid covers every SM about twice, but no slice
+  // shorter than two key tiles.
+  const int tiles = (Lk + 127) / 128;
+  int n = (2 * sms + n_units - 1) / n_units;
+  n = n < tiles / 2 ? n : tiles / 2;
+  n = n < kMaxSplit ? n : kMaxSplit;
+  return n < 1 ? 1 : n;
+}
+
+int attn_fwd_split(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Lq,
+                   int Lk, int d, float scale, int causal, int window, int n_split, void* workspace,
+                   size_t workspace_bytes, void* stream) {
+  if (n_split < 1 || n_split > kMaxSplit) return ATTN_ERR_INVALID_ARG;
+  if (n_split == 1) return attn_fwd(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, scale, causal, window, stream);
+  int st = check_shape(B, Hq, Hkv, Lq, Lk, d, scale, causal, window);
+  if (st != ATTN_OK) return st;
+  if (B == 0 || Hq == 0 || Lq == 0) return ATTN_OK;
+  if (!q || !o || !lse || !aligned16(q) || !aligned16(o) || !aligned16(lse)) return ATTN_ERR_INVALID_ARG;
+  if (Lk > 0 && (!k || !v || !aligned16(k) || !aligned16(v))) return ATTN_ERR_INVALID_ARG;
+  const size_t need = attn_fwd_split_workspace_size(B, Hq, Hkv, Lq, Lk, d, n_split);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need)
+    return ATTN_ERR_INVALID_ARG;
+  EncodeTiledFn enc;
+  if ((st = get_encoder(&enc)) != ATTN_OK) return st;
+  FwdParams P;
+  memset(&P, 0, sizeof(P));
+  P.prob = Problem{B, Hq, Hkv, Lq, Lk, d, causal, window, scale};
+  const void* kp = Lk > 0 ? k : q;
+  const void* vp = Lk > 0 ? v : q;
+  if ((st = make_map(enc, &P.tm_q, q, B * Hq, Lq, d)) != ATTN_OK) return st;
+  if ((st = make_map(enc, &P.tm_k, kp, Lk > 0 ? B * Hkv : B * Hq, Lk > 0 ? Lk : Lq, d)) != ATTN_OK) return st;
+  if ((st = make_map(enc, &P.tm_v, vp, Lk > 0 ? B * Hkv : B * Hq, Lk > 0 ? Lk : Lq, d)) != ATTN_OK) return st;
+  P.o = o;
+  P.lse = lse;
+  P.scale_log2 = scale * 1.4426950408889634f;
+  fwd_plan(P.prob, &P.n_units, &P.pair_heads);
+  P.n_split = n_split;
+  const size_t rows = (size_t)B * Hq * Lq;
+  P.part_o = static_cast<float*>(workspace);
+  P.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                        ((size_t)n_split * rows * d * 4 + 255) / 256 * 256);
+  if ((int64_t)P.n_units * n_split > 0x7fffffff) return ATTN_ERR_UNSUPPORTED;
+  if ((st = get_err_word(&P.err)) != ATTN_OK) return st;
+  P.limit_ns = kWaitLimitNs;
+  cudaError_t e = launch_fwd(P, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail("attn_fwd_split launch", e);
+  e = launch_fwd_merge(P, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ATTN_OK : cuda_fail("attn_fwd_split merge launch", e);
+}
+
 size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int Lq, int Lk, int d) {
   if (check_shape(B, Hq, Hkv, Lq, Lk, d, 1.f, 0, 0) != ATTN_OK) return 0;
   if (B == 0 || Hq == 0 || Lq == 0) return 0;

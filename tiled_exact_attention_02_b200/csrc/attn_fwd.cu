@@ -116,6 +116,7 @@ struct Unit {
   int q0[2];
   int lo[2], hi[2];  // key tile range per slot (empty: lo == hi)
   int ulo, uhi;      // union of the two ranges
+  int split;         // key-range slice of a split problem (0 otherwise)
 };
 
 __device__ __forceinline__ Unit decode_unit(const FwdParams& P, int idx) {
@@ -160,6 +161,37 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& P, int idx) {
     }
   }
   if (u.uhi == 0) u.ulo = 0;
+  return u;
+}
+
+// Unit of CTA `idx` when every unit's key range is cut into n_split slices
+// (consecutive CTAs take the slices of one unit): slice k keeps key tiles
+// [ulo + k*len/n, ulo + (k+1)*len/n) of the union range, intersected with
+// each slot's own range.  An empty slice leaves both slots empty.
+__device__ __forceinline__ Unit decode_unit_split(const FwdParams& P, int idx) {
+  if (P.n_split <= 1) {
+    Unit u = decode_unit(P, idx);
+    u.split = 0;
+    return u;
+  }
+  Unit u = decode_unit(P, idx / P.n_split);
+  u.split = idx % P.n_split;
+  const int len = u.uhi - u.ulo;
+  const int s_lo = u.ulo + (int)((long long)u.split * len / P.n_split);
+  const int s_hi = u.ulo + (int)((long long)(u.split + 1) * len / P.n_split);
+  int nlo = 1 << 30, nhi = 0;
+  for (int s = 0; s < 2; s++) {
+    u.lo[s] = imax(u.lo[s], s_lo);
+    u.hi[s] = imin(u.hi[s], s_hi);
+    if (u.lo[s] >= u.hi[s]) {
+      u.lo[s] = u.hi[s] = 0;
+    } else {
+      nlo = imin(nlo, u.lo[s]);
+      nhi = imax(nhi, u.hi[s]);
+    }
+  }
+  u.ulo = nhi > 0 ? nlo : 0;
+  u.uhi = nhi;
   return u;
 }
 
@@ -402,6 +434,32 @@ __device__ void softmax_slot(const FwdParams& P, const Unit& u, int s, Bars& bar
   const bool write = q_row < p.Lq;
   const float inv_l = l > 0.f ? 1.f / l : 0.f;
   const size_t row_off = ((size_t)(u.b * p.Hq + head_s) * p.Lq + q_row);
+  const float lse_row = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
+  if (P.n_split > 1) {
+    // One key-range slice of a split problem: fp32 O normalised by this
+    // slice's own sum, and the slice's LSE; the merge kernel combines them.
+    const size_t part_row = (size_t)u.split * ((size_t)p.B * p.Hq * p.Lq) + row_off;
+    float4* outp = reinterpret_cast<float4*>(P.part_o + part_row * D);
+#pragma unroll
+    for (int q = 0; q < D / 32; q++) {
+      uint32_t o[32];
+      if (has) {
+        tmem_ld32p(t_o + 32 * q, o);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; e++) o[e] = 0u;
+      }
+      if (write) {
+#pragma unroll
+        for (int v = 0; v < 8; v++)
+          outp[q * 8 + v] = make_float4(__uint_as_float(o[4 * v]) * inv_l, __uint_as_float(o[4 * v + 1]) * inv_l,
+                                        __uint_as_float(o[4 * v + 2]) * inv_l, __uint_as_float(o[4 * v + 3]) * inv_l);
+      }
+    }
+    if (write) P.part_lse[part_row] = lse_row;
+    return;
+  }
   uint4* out = reinterpret_cast<uint4*>(static_cast<uint16_t*>(P.o) + row_off * D);
 #pragma unroll
   for (int q = 0; q < D / 32; q++) {
@@ -422,7 +480,7 @@ __device__ void softmax_slot(const FwdParams& P, const Unit& u, int s, Bars& bar
       for (int v = 0; v < 4; v++) out[q * 4 + v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
     }
   }
-  if (write) P.lse[row_off] = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
+  if (write) P.lse[row_off] = lse_row;
 }
 
 // ------------------------------------------------------------------ kernel
@@ -434,7 +492,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_kernel(const __grid_const
   Bars& bars = *reinterpret_cast<Bars*>(smem + C::OFF_BAR);
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  const Unit u = decode_unit(P, blockIdx.x);
+  const Unit u = decode_unit_split(P, blockIdx.x);
   const WaitGuard g{P.err, &bars.abort_flag, P.limit_ns, 0};
 
   if (threadIdx.x == 0) {
@@ -482,7 +540,67 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_kernel(const __grid_const
   }
 }
 
+// ------------------------------------------------------------------ split merge
+// Row i of a split problem: with w_k = exp(LSE_k - max_k LSE_k) over the
+// slices k, O_i = sum_k w_k O_k / sum_k w_k and LSE_i = max + log(sum_k w_k)
+// (each O_k is already normalised by its own slice's sum, so this is the
+// exact softmax over the union of the slices).  A row no slice saw keeps
+// O = 0 and LSE = -inf.  One warp per row, D / 32 elements per lane.
+template <int D>
+__global__ void __launch_bounds__(256) fwd_merge_kernel(const float* __restrict__ part_o,
+                                                        const float* __restrict__ part_lse, uint16_t* __restrict__ o,
+                                                        float* __restrict__ lse, int64_t rows, int n_split) {
+  constexpr int PER = D / 32;
+  const int64_t row = (int64_t)blockIdx.x * 8 + threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  if (row >= rows) return;
+  float mx = -INFINITY;
+  for (int k = 0; k < n_split; k++) mx = fmaxf(mx, part_lse[(int64_t)k * rows + row]);
+  float acc[PER];
+#pragma unroll
+  for (int e = 0; e < PER; e++) acc[e] = 0.f;
+  float sum = 0.f;
+  if (mx != -INFINITY) {
+    for (int k = 0; k < n_split; k++) {
+      const float lk = part_lse[(int64_t)k * rows + row];
+      if (lk == -INFINITY) continue;
+      const float w = expf(lk - mx);
+      sum += w;
+      const float* src = part_o + ((int64_t)k * rows + row) * D + lane * PER;
+      if constexpr (PER == 4) {
+        const float4 x = *reinterpret_cast<const float4*>(src);
+        acc[0] += w * x.x, acc[1] += w * x.y, acc[2] += w * x.z, acc[3] += w * x.w;
+      } else {
+        const float2 x = *reinterpret_cast<const float2*>(src);
+        acc[0] += w * x.x, acc[1] += w * x.y;
+      }
+    }
+  }
+  const float inv = sum > 0.f ? 1.f / sum : 0.f;
+  uint16_t* dst = o + row * D + lane * PER;
+  if constexpr (PER == 4) {
+    *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv));
+  } else {
+    *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+  }
+  if (lane == 0) lse[row] = sum > 0.f ? mx + logf(sum) : -INFINITY;
+}
+
 }  // namespace fwd
+
+cudaError_t launch_fwd_merge(const FwdParams& P, cudaStream_t stream) {
+  const int64_t rows = (int64_t)P.prob.B * P.prob.Hq * P.prob.Lq;
+  if (rows == 0) return cudaSuccess;
+  const unsigned grid = (unsigned)((rows + 7) / 8);
+  if (P.prob.d == 128)
+    fwd::fwd_merge_kernel<128><<<grid, 256, 0, stream>>>(P.part_o, P.part_lse, static_cast<uint16_t*>(P.o), P.lse,
+                                                          rows, P.n_split);
+  else
+    fwd::fwd_merge_kernel<64><<<grid, 256, 0, stream>>>(P.part_o, P.part_lse, static_cast<uint16_t*>(P.o), P.lse,
+                                                         rows, P.n_split);
+  return cudaGetLastError();
+}
+
 
 void fwd_plan(const Problem& p, int* n_units, int* pair_heads) {
   const int G = p.Hq / p.Hkv;
@@ -501,7 +619,7 @@ static cudaError_t launch_fwd_d(const FwdParams& P, cudaStream_t stream) {
   constexpr int smem = fwd::Cfg<D>::SMEM;
   cudaError_t e = cudaFuncSetAttribute(fwd::attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  fwd::attn_fwd_kernel<D><<<P.n_units, fwd::THREADS, smem, stream>>>(P);
+  fwd::attn_fwd_kernel<D><<<P.n_units * imax(1, P.n_split), fwd::THREADS, smem, stream>>>(P);
   return cudaGetLastError();
 }
 

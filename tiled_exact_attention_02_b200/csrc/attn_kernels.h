@@ -16,7 +16,10 @@ struct FwdParams {
   float* lse;        // fp32 [B, Hq, Lq]
   float scale_log2;  // scale * log2(e)
   int pair_heads;    // 1: a CTA takes two heads of one GQA group at the same rows
-  int n_units;       // CTAs in the grid
+  int n_units;       // work units (two query tiles each); the grid is n_units * n_split CTAs
+  int n_split;       // key-range slices per unit (1: the CTA writes O and LSE itself)
+  float* part_o;     // n_split > 1: fp32 [n_split][B*Hq][Lq][d], O of each slice normalised by its own sum
+  float* part_lse;   // n_split > 1: fp32 [n_split][B*Hq][Lq], natural-log LSE of each slice (-inf: empty)
   int* err;          // device error word
   uint64_t limit_ns; // bounded-wait limit
 };
@@ -67,5 +70,7 @@ cudaError_t launch_bwd_post(const float* dq_acc, void* dq, int BH, int Lq, int l
 // Number of CTAs of the forward grid and whether heads are paired.
 void fwd_plan(const Problem& p, int* n_units, int* pair_heads);
 cudaError_t launch_fwd(const FwdParams& P, cudaStream_t stream);
+// Combine n_split partial (O, LSE) of every row into bf16 O and fp32 LSE.
+cudaError_t launch_fwd_merge(const FwdParams& P, cudaStream_t stream);
 
 }  // namespace tea
