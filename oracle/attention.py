@@ -147,21 +147,35 @@ def _kv_head(h: int, Hq: int, Hkv: int) -> int:
     return h // _group(Hq, Hkv)
 
 
-def attn_fwd(q, k, v, scale: float, causal: bool = False, window: int = 0, heads=None):
+def _lengths(seqlens, b: int, full: int) -> int:
+    return full if seqlens is None else min(full, int(seqlens[b]))
+
+
+def attn_fwd(q, k, v, scale: float, causal: bool = False, window: int = 0, heads=None, seqlens_q=None,
+             seqlens_k=None):
     """O [B,Hq,Lq,d] and LSE [B,Hq,Lq] in float64.
 
     q: [B,Hq,Lq,d]; k, v: [B,Hkv,Lk,d] (float or bf16 bits as uint16).
     heads: optional list of (b, h) to evaluate; other heads are left NaN.
+    seqlens_q / seqlens_k: optional per-sequence lengths of a padded batch
+    ("大模型高效注意力机制全解析" §5.2.2: requests of different lengths are padded
+    into one batch and each output is cut back to its own length):
+    sequence b is its own attention problem over its first seqlens_q[b]
+    queries and seqlens_k[b] keys (a bottom-right causal diagonal is placed by
+    those lengths); padded query rows get O = 0 and LSE = -inf.
     """
     q, k, v = _f64(q), _f64(k), _f64(v)
     B, Hq, Lq, d = q.shape
-    Hkv = k.shape[1]
+    Hkv, Lk = k.shape[1], k.shape[2]
     O = np.full((B, Hq, Lq, v.shape[-1]), np.nan)
     lse = np.full((B, Hq, Lq), np.nan)
     todo = heads if heads is not None else [(b, h) for b in range(B) for h in range(Hq)]
     for b, h in todo:
         g = _kv_head(h, Hq, Hkv)
-        O[b, h], lse[b, h] = _head_fwd(q[b, h], k[b, g], v[b, g], scale, causal, window)
+        nq, nk = _lengths(seqlens_q, b, Lq), _lengths(seqlens_k, b, Lk)
+        O[b, h] = 0.0
+        lse[b, h] = -np.inf
+        O[b, h, :nq], lse[b, h, :nq] = _head_fwd(q[b, h, :nq], k[b, g, :nk], v[b, g, :nk], scale, causal, window)
     return O, lse
 
 
@@ -237,27 +251,31 @@ def attn_row_block(q, k, v, do, scale, causal, window, b, h, r0, r1):
     return O, lse, dq, lo, hi, dk, dv
 
 
-def attn_bwd(q, k, v, do, scale: float, causal: bool = False, window: int = 0, heads=None):
+def attn_bwd(q, k, v, do, scale: float, causal: bool = False, window: int = 0, heads=None, seqlens_q=None,
+             seqlens_k=None):
     """dQ [B,Hq,Lq,d], dK and dV [B,Hkv,Lk,d] in float64.
 
     dK/dV of a K/V head are summed over the query heads that share it.
     heads: optional list of (b, hkv): only those K/V heads (and all query
     heads of their groups) are evaluated; the rest is left NaN.
+    seqlens_q / seqlens_k: as attn_fwd; padded rows and keys get zero gradients.
     """
     q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
     B, Hq, Lq, d = q.shape
-    Hkv = k.shape[1]
+    Hkv, Lk = k.shape[1], k.shape[2]
     _group(Hq, Hkv)
     dq = np.full(q.shape, np.nan)
     dk = np.full(k.shape, np.nan)
     dv = np.full(v.shape, np.nan)
     todo = heads if heads is not None else [(b, g) for b in range(B) for g in range(Hkv)]
     for b, g in todo:
+        nq, nk = _lengths(seqlens_q, b, Lq), _lengths(seqlens_k, b, Lk)
         dk[b, g] = 0.0
         dv[b, g] = 0.0
         for h in (h for h in range(Hq) if _kv_head(h, Hq, Hkv) == g):
-            dqh, dkh, dvh = _head_bwd(q[b, h], k[b, g], v[b, g], do[b, h], scale, causal, window)
-            dq[b, h] = dqh
-            dk[b, g] += dkh
-            dv[b, g] += dvh
+            dq[b, h] = 0.0
+            dqh, dkh, dvh = _head_bwd(q[b, h, :nq], k[b, g, :nk], v[b, g, :nk], do[b, h, :nq], scale, causal, window)
+            dq[b, h, :nq] = dqh
+            dk[b, g, :nk] += dkh
+            dv[b, g, :nk] += dvh
     return dq, dk, dv

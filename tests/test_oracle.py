@@ -178,6 +178,49 @@ def test_bottom_right_with_more_queries_than_keys():
     assert np.all(dq[0, 0, :Lq - Lk] == 0)
 
 
+def test_padded_batch_equals_separate_sequences():
+    """Per-sequence lengths: each sequence of a padded batch is its own problem
+    (evaluated here on the sliced arrays), padding rows are O = 0, LSE = -inf,
+    and the padding's contents change nothing."""
+    B, Hq, Hkv, Lq, Lk, d = 3, 4, 2, 11, 13, 5
+    q, k, v, do = _rand(B, Hq, Lq, d), _rand(B, Hkv, Lk, d), _rand(B, Hkv, Lk, d), _rand(B, Hq, Lq, d)
+    lq, lk = [11, 4, 0], [13, 9, 6]
+    for causal, w in ((False, 0), (True, 0), (2, 0), (2, 3), (False, 3)):
+        O, lse = oracle.attn_fwd(q, k, v, 0.4, causal, w, seqlens_q=lq, seqlens_k=lk)
+        dq, dk, dv = oracle.attn_bwd(q, k, v, do, 0.4, causal, w, seqlens_q=lq, seqlens_k=lk)
+        for b in range(B):
+            sl = slice(b, b + 1)
+            Ob, lb = oracle.attn_fwd(q[sl, :, :lq[b]], k[sl, :, :lk[b]], v[sl, :, :lk[b]], 0.4, causal, w)
+            np.testing.assert_array_equal(O[b, :, :lq[b]], Ob[0])
+            np.testing.assert_array_equal(lse[b, :, :lq[b]], lb[0])
+            assert np.all(O[b, :, lq[b]:] == 0) and np.all(np.isneginf(lse[b, :, lq[b]:]))
+            gb = oracle.attn_bwd(q[sl, :, :lq[b]], k[sl, :, :lk[b]], v[sl, :, :lk[b]], do[sl, :, :lq[b]], 0.4, causal, w)
+            np.testing.assert_array_equal(dq[b, :, :lq[b]], gb[0][0])
+            np.testing.assert_array_equal(dk[b, :, :lk[b]], gb[1][0])
+            assert np.all(dq[b, :, lq[b]:] == 0) and np.all(dk[b, :, lk[b]:] == 0) and np.all(dv[b, :, lk[b]:] == 0)
+        # garbage in the padding changes nothing
+        q2, k2, v2 = q.copy(), k.copy(), v.copy()
+        q2[1, :, 4:] = 1e3
+        k2[1, :, 9:] = -7e2
+        v2[2, :, 6:] = np.nan
+        O2, l2 = oracle.attn_fwd(q2, k2, v2, 0.4, causal, w, seqlens_q=lq, seqlens_k=lk)
+        np.testing.assert_array_equal(O2, O)
+        np.testing.assert_array_equal(l2, lse)
+
+
+def test_padded_batch_matches_torch_sdpa_key_padding_mask():
+    """Per-sequence key lengths against torch SDPA with a key-padding mask built here."""
+    B, H, L, d = 2, 2, 10, 4
+    q, k, v = _rand(B, H, L, d), _rand(B, H, L, d), _rand(B, H, L, d)
+    lk = [10, 6]
+    O, _ = oracle.attn_fwd(q, k, v, 0.5, False, 0, seqlens_k=lk)
+    keep = torch.arange(L)[None, :] < torch.tensor(lk)[:, None]
+    mask = keep[:, None, None, :].expand(B, H, L, L)
+    ref = torch.nn.functional.scaled_dot_product_attention(*(torch.from_numpy(x) for x in (q, k, v)),
+                                                           attn_mask=mask, scale=0.5)
+    np.testing.assert_allclose(O, ref.numpy(), atol=1e-12)
+
+
 def test_value_shift_and_score_shift_invariance():
     """V + 1 c^T gives O + 1 c^T; a per-row constant added to the logits changes nothing."""
     L, d = 19, 4
