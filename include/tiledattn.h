@@ -87,6 +87,25 @@ ATTN_API int attn_fwd(const void* q, const void* k, const void* v, void* o, floa
              int Lk, int d, float scale, int causal, int window, void* stream);
 
 /*
+ * Forward pass over a padded batch of sequences of different lengths
+ * ("大模型高效注意力机制全解析" §5.2.2: requests are padded into one batch and
+ * each output cut back to its own length).  Tensors keep the padded [B, H, L,
+ * d] layout of attn_fwd; sequence b is its own attention problem over its
+ * first seqlens_q[b] queries and seqlens_k[b] keys (a bottom-right causal
+ * diagonal is placed by those lengths).  Padded query rows get O = 0 and LSE =
+ * -inf; padded keys are never visible.  Key tiles past a sequence's end are
+ * skipped.
+ *
+ *  seqlens_q, seqlens_k  device int32 [B] (4-byte aligned), or NULL for "all
+ *                        Lq" / "all Lk"; values are clamped to [0, Lq] and
+ *                        [0, Lk].  Read by the kernels, not by the host.
+ *  other arguments       as attn_fwd.
+ */
+ATTN_API int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int* seqlens_q,
+                             const int* seqlens_k, int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale,
+                             int causal, int window, void* stream);
+
+/*
  * Forward pass with the key range split across CTAs (for few query rows over
  * many keys, e.g. new queries over a long cache with causal = 2).  Each query
  * tile's visible key tiles are cut into n_split contiguous slices, each
@@ -145,6 +164,15 @@ ATTN_API int attn_bwd(const void* q, const void* k, const void* v, const void* o
              void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * attn_bwd over a padded batch (see attn_fwd_varlen): the same lengths as the
+ * forward pass; padded query rows get dQ = 0 and padded keys dK = dV = 0.
+ */
+ATTN_API int attn_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                             const void* dO, void* dq, void* dk, void* dv, const int* seqlens_q, const int* seqlens_k,
+                             int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale, int causal, int window,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * The three phases attn_bwd runs, for callers that schedule or time them
  * separately (same arguments and rules as attn_bwd; call them in this order
  * on one stream with the same workspace):
@@ -157,6 +185,12 @@ ATTN_API int attn_bwd_preprocess(const void* o, const void* dO, int B, int Hq, i
 ATTN_API int attn_bwd_main(const void* q, const void* k, const void* v, const float* lse, const void* dO, void* dk,
                            void* dv, int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale, int causal, int window,
                            void* workspace, size_t workspace_bytes, void* stream);
+
+/* attn_bwd_main over a padded batch (phase 2 of attn_bwd_varlen). */
+ATTN_API int attn_bwd_main_varlen(const void* q, const void* k, const void* v, const float* lse, const void* dO,
+                                  void* dk, void* dv, const int* seqlens_q, const int* seqlens_k, int B, int Hq,
+                                  int Hkv, int Lq, int Lk, int d, float scale, int causal, int window,
+                                  void* workspace, size_t workspace_bytes, void* stream);
 ATTN_API int attn_bwd_finalize(void* dq, int B, int Hq, int Lq, int d, float scale, void* workspace,
                                size_t workspace_bytes, void* stream);
 

@@ -73,6 +73,37 @@ def test_bwd_edge_shapes(ta, B, Hq, Hkv, Lq, Lk, d, causal, window):
     check_grad(dv, rv, "dV")
 
 
+VARLEN = [
+    (3, 4, 2, 300, 300, 128, 1, 0, [300, 129, 0], [300, 129, 0]),
+    (3, 2, 2, 257, 400, 128, 2, 0, [1, 100, 257], [400, 37, 256]),
+    (2, 4, 4, 200, 200, 64, 0, 0, [200, 77], [150, 200]),
+    (2, 2, 1, 500, 500, 128, 1, 64, [500, 333], [500, 333]),
+    (2, 2, 2, 300, 300, 128, 0, 50, [300, 128], [10, 300]),
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Lq,Lk,d,causal,window,lq,lk", VARLEN)
+def test_bwd_varlen(ta, B, Hq, Hkv, Lq, Lk, d, causal, window, lq, lk):
+    """Per-sequence lengths: gradients against the oracle, zeros in the padding."""
+    import torch
+    x = make_shape_inputs(B, Hq, Hkv, Lq, Lk, d, seed=Lq * 13 + Lk + d + 9, with_do=True)
+    scale = d ** -0.5
+    q, k, v, do = (to_dev(x[n]) for n in ("q", "k", "v", "do"))
+    tq = torch.tensor(lq, dtype=torch.int32, device="cuda")
+    tk = torch.tensor(lk, dtype=torch.int32, device="cuda")
+    o, lse = ta.attention(q, k, v, causal, window, scale, seqlens_q=tq, seqlens_k=tk)
+    dq, dk, dv = ta.attention_backward(q, k, v, o, lse, do, causal, window, scale, seqlens_q=tq, seqlens_k=tk)
+    st, site = ta.device_error()
+    assert st == 0, f"device error {st} at site {site}"
+    rq, rk, rv = oracle.attn_bwd(x["q"], x["k"], x["v"], x["do"], scale, causal, window, seqlens_q=lq, seqlens_k=lk)
+    check_grad(to_f64(dq), rq, "dQ")
+    check_grad(to_f64(dk), rk, "dK")
+    check_grad(to_f64(dv), rv, "dV")
+    for b in range(B):
+        assert np.all(to_f64(dq)[b, :, lq[b]:] == 0)
+        assert np.all(to_f64(dk)[b, :, lk[b]:] == 0) and np.all(to_f64(dv)[b, :, lk[b]:] == 0)
+
+
 def test_bwd_gqa_window_2048(ta):
     x = make_shape_inputs(1, 8, 2, 2048, 2048, 128, seed=17, with_do=True)
     dq, dk, dv = run_fwd_bwd(ta, x, True, 300, 128 ** -0.5)

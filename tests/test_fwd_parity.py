@@ -96,6 +96,33 @@ def test_fwd_split_kv(ta, B, Hq, Hkv, Lq, Lk, d, causal, window, n_split):
     check_lse(to_f64(lse), rl, "LSE")
 
 
+# (B, Hq, Hkv, Lq, Lk, d, causal, window, seqlens_q, seqlens_k): padded batches
+VARLEN = [
+    (3, 4, 2, 300, 300, 128, 1, 0, [300, 129, 0], [300, 129, 0]),
+    (3, 2, 2, 257, 400, 128, 2, 0, [1, 100, 257], [400, 37, 256]),
+    (2, 4, 4, 200, 200, 64, 0, 0, [200, 77], [150, 200]),
+    (2, 2, 1, 500, 500, 128, 1, 64, [500, 333], [500, 333]),
+    (2, 2, 2, 300, 300, 128, 0, 50, [300, 128], [10, 300]),
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Lq,Lk,d,causal,window,lq,lk", VARLEN)
+def test_fwd_varlen(ta, B, Hq, Hkv, Lq, Lk, d, causal, window, lq, lk):
+    """Per-sequence lengths of a padded batch against the oracle (padding rows: O = 0, LSE = -inf)."""
+    import torch
+    x = make_shape_inputs(B, Hq, Hkv, Lq, Lk, d, seed=Lq * 11 + Lk + d + 5)
+    scale = d ** -0.5
+    q, k, v = (to_dev(x[n]) for n in "qkv")
+    tq = torch.tensor(lq, dtype=torch.int32, device="cuda")
+    tk = torch.tensor(lk, dtype=torch.int32, device="cuda")
+    o, lse = ta.attention(q, k, v, causal, window, scale, seqlens_q=tq, seqlens_k=tk)
+    st, site = ta.device_error()
+    assert st == 0, f"device error {st} at site {site}"
+    ro, rl = oracle.attn_fwd(x["q"], x["k"], x["v"], scale, causal, window, seqlens_q=lq, seqlens_k=lk)
+    check_o(to_f64(o), ro, "O")
+    check_lse(to_f64(lse), rl, "LSE")
+
+
 def test_fwd_no_keys(ta):
     """Lk = 0: every row sees nothing: O = 0, LSE = -inf."""
     import torch

@@ -46,6 +46,12 @@ def _load() -> ctypes.CDLL:
     lib.attn_fwd_split_workspace_size.restype = sz
     lib.attn_fwd_split_default.argtypes = [i, i, i, i, i, i, i, i]
     lib.attn_fwd_split_default.restype = i
+    lib.attn_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, vp]
+    lib.attn_fwd_varlen.restype = i
+    lib.attn_bwd_varlen.argtypes = [vp] * 11 + [i] * 6 + [f, i, i, vp, sz, vp]
+    lib.attn_bwd_varlen.restype = i
+    lib.attn_bwd_main_varlen.argtypes = [vp] * 9 + [i] * 6 + [f, i, i, vp, sz, vp]
+    lib.attn_bwd_main_varlen.restype = i
     lib.attn_bwd_workspace_size.argtypes = [i, i, i, i, i, i]
     lib.attn_bwd_workspace_size.restype = sz
     lib.attn_bwd.argtypes = [vp] * 9 + [i] * 6 + [f, i, i, vp, sz, vp]
@@ -115,8 +121,21 @@ def _causal_code(causal) -> int:
     return 2 if causal == 2 and not isinstance(causal, bool) else int(bool(causal))
 
 
-def fwd(q, k, v, o, lse, causal: bool = False, window: int = 0, scale: float | None = None, stream=None):
-    """attn_fwd on torch tensors (bf16 q/k/v/o, fp32 lse), asynchronous on `stream`."""
+def _lens(seqlens, B, name):
+    """Device pointer of optional per-sequence lengths (int32 CUDA tensor [B])."""
+    import torch
+    if seqlens is None:
+        return None
+    _require(seqlens, name, torch.int32)
+    if tuple(seqlens.shape) != (B,):
+        raise ValueError(f"{name} must have shape ({B},)")
+    return seqlens.data_ptr()
+
+
+def fwd(q, k, v, o, lse, causal: bool = False, window: int = 0, scale: float | None = None, stream=None,
+        seqlens_q=None, seqlens_k=None):
+    """attn_fwd on torch tensors (bf16 q/k/v/o, fp32 lse), asynchronous on
+    `stream`; with seqlens_q / seqlens_k (int32 CUDA [B]) attn_fwd_varlen."""
     import torch
     for n, t in (("q", q), ("k", k), ("v", v), ("o", o)):
         _require(t, n, torch.bfloat16)
@@ -125,9 +144,15 @@ def fwd(q, k, v, o, lse, causal: bool = False, window: int = 0, scale: float | N
     if tuple(v.shape) != tuple(k.shape) or tuple(o.shape) != tuple(q.shape) or tuple(lse.shape) != (B, Hq, Lq):
         raise ValueError("v/o/lse shape mismatch")
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
-    st = lib.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                      B, Hq, Hkv, Lq, Lk, d, scale, _causal_code(causal), int(window), _stream_ptr(stream))
-    _check(st, "attn_fwd")
+    lq, lk = _lens(seqlens_q, B, "seqlens_q"), _lens(seqlens_k, B, "seqlens_k")
+    if lq is None and lk is None:
+        st = lib.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                          B, Hq, Hkv, Lq, Lk, d, scale, _causal_code(causal), int(window), _stream_ptr(stream))
+        _check(st, "attn_fwd")
+        return
+    st = lib.attn_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), lq, lk,
+                             B, Hq, Hkv, Lq, Lk, d, scale, _causal_code(causal), int(window), _stream_ptr(stream))
+    _check(st, "attn_fwd_varlen")
 
 
 def bwd_workspace_size(B, Hq, Hkv, Lq, Lk, d) -> int:
@@ -135,8 +160,9 @@ def bwd_workspace_size(B, Hq, Hkv, Lq, Lk, d) -> int:
 
 
 def bwd(q, k, v, o, lse, do, dq, dk, dv, workspace, causal: bool = False, window: int = 0,
-        scale: float | None = None, stream=None):
-    """attn_bwd on torch tensors; `workspace` is a uint8 CUDA tensor."""
+        scale: float | None = None, stream=None, seqlens_q=None, seqlens_k=None):
+    """attn_bwd on torch tensors; `workspace` is a uint8 CUDA tensor; with
+    seqlens_q / seqlens_k attn_bwd_varlen."""
     import torch
     for n, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do), ("dq", dq), ("dk", dk), ("dv", dv)):
         _require(t, n, torch.bfloat16)
@@ -144,11 +170,18 @@ def bwd(q, k, v, o, lse, do, dq, dk, dv, workspace, causal: bool = False, window
     _require(workspace, "workspace")
     B, Hq, Hkv, Lq, Lk, d = _shapes(q, k)
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
-    st = lib.attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
-                      dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv, Lq, Lk, d, scale,
-                      _causal_code(causal), int(window), workspace.data_ptr(),
-                      workspace.numel() * workspace.element_size(), _stream_ptr(stream))
-    _check(st, "attn_bwd")
+    lq, lk = _lens(seqlens_q, B, "seqlens_q"), _lens(seqlens_k, B, "seqlens_k")
+    wsp, wsb = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    if lq is None and lk is None:
+        st = lib.attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
+                          dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv, Lq, Lk, d, scale,
+                          _causal_code(causal), int(window), wsp, wsb, _stream_ptr(stream))
+        _check(st, "attn_bwd")
+        return
+    st = lib.attn_bwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
+                             dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), lq, lk, B, Hq, Hkv, Lq, Lk, d, scale,
+                             _causal_code(causal), int(window), wsp, wsb, _stream_ptr(stream))
+    _check(st, "attn_bwd_varlen")
 
 
 def bwd_phases(q, k, v, o, lse, do, dq, dk, dv, workspace, causal: bool = False, window: int = 0,
@@ -177,13 +210,14 @@ def device_error(stream=None) -> tuple[int, int]:
     return st, site.value
 
 
-def attention(q, k, v, causal: bool = False, window: int = 0, scale: float | None = None):
+def attention(q, k, v, causal: bool = False, window: int = 0, scale: float | None = None, seqlens_q=None,
+              seqlens_k=None):
     """Allocate O and LSE with torch and run the forward pass."""
     import torch
     B, Hq, Hkv, Lq, Lk, d = _shapes(q, k)
     o = torch.empty_like(q)
     lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
-    fwd(q, k, v, o, lse, causal, window, scale)
+    fwd(q, k, v, o, lse, causal, window, scale, seqlens_q=seqlens_q, seqlens_k=seqlens_k)
     return o, lse
 
 
@@ -216,13 +250,14 @@ def attention_split(q, k, v, causal: bool = False, window: int = 0, scale: float
     return o, lse
 
 
-def attention_backward(q, k, v, o, lse, do, causal: bool = False, window: int = 0, scale: float | None = None):
+def attention_backward(q, k, v, o, lse, do, causal: bool = False, window: int = 0, scale: float | None = None,
+                       seqlens_q=None, seqlens_k=None):
     """Allocate dQ/dK/dV and the workspace with torch and run the backward pass."""
     import torch
     B, Hq, Hkv, Lq, Lk, d = _shapes(q, k)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     ws = torch.empty(max(1, bwd_workspace_size(B, Hq, Hkv, Lq, Lk, d)), dtype=torch.uint8, device=q.device)
-    bwd(q, k, v, o, lse, do, dq, dk, dv, ws, causal, window, scale)
+    bwd(q, k, v, o, lse, do, dq, dk, dv, ws, causal, window, scale, seqlens_q=seqlens_q, seqlens_k=seqlens_k)
     return dq, dk, dv
 
 

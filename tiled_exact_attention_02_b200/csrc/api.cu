@@ -141,18 +141,26 @@ const char* attn_status_string(int status) {
   }
 }
 
-int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Lq,
-             int Lk, int d, float scale, int causal, int window, void* stream) {
+// Forward for every entry point: lens_q / lens_k optional per-sequence
+// lengths (device int32 [B]); n_split > 1 cuts each unit's key range into
+// slices written to `workspace` and merged.
+static int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, const int* lens_q,
+                    const int* lens_k, int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale, int causal,
+                    int window, int n_split, void* workspace, void* stream) {
   int st = check_shape(B, Hq, Hkv, Lq, Lk, d, scale, causal, window);
   if (st != ATTN_OK) return st;
   if (B == 0 || Hq == 0 || Lq == 0) return ATTN_OK;
   if (!q || !o || !lse || !aligned16(q) || !aligned16(o) || !aligned16(lse)) return ATTN_ERR_INVALID_ARG;
   if (Lk > 0 && (!k || !v || !aligned16(k) || !aligned16(v))) return ATTN_ERR_INVALID_ARG;
+  if ((lens_q && (reinterpret_cast<uintptr_t>(lens_q) & 3u)) || (lens_k && (reinterpret_cast<uintptr_t>(lens_k) & 3u)))
+    return ATTN_ERR_INVALID_ARG;
   EncodeTiledFn enc;
   if ((st = get_encoder(&enc)) != ATTN_OK) return st;
   FwdParams P;
   memset(&P, 0, sizeof(P));
   P.prob = Problem{B, Hq, Hkv, Lq, Lk, d, causal, window, scale};
+  P.prob.len_q = lens_q;
+  P.prob.len_k = lens_k;
   // With Lk == 0 nothing reads K/V; map Q's memory so the descriptors stay valid.
   const void* kp = Lk > 0 ? k : q;
   const void* vp = Lk > 0 ? v : q;
@@ -163,10 +171,35 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   P.lse = lse;
   P.scale_log2 = scale * 1.4426950408889634f;
   fwd_plan(P.prob, &P.n_units, &P.pair_heads);
+  P.n_split = n_split;
+  if (n_split > 1) {
+    const size_t rows = (size_t)B * Hq * Lq;
+    P.part_o = static_cast<float*>(workspace);
+    P.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                          ((size_t)n_split * rows * d * 4 + 255) / 256 * 256);
+    if ((int64_t)P.n_units * n_split > 0x7fffffff) return ATTN_ERR_UNSUPPORTED;
+  }
   if ((st = get_err_word(&P.err)) != ATTN_OK) return st;
   P.limit_ns = kWaitLimitNs;
-  const cudaError_t e = launch_fwd(P, static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? ATTN_OK : cuda_fail("attn_fwd launch", e);
+  cudaError_t e = launch_fwd(P, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail("attn_fwd launch", e);
+  if (n_split > 1) {
+    e = launch_fwd_merge(P, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail("attn_fwd_split merge launch", e);
+  }
+  return ATTN_OK;
+}
+
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Lq,
+             int Lk, int d, float scale, int causal, int window, void* stream) {
+  return fwd_impl(q, k, v, o, lse, nullptr, nullptr, B, Hq, Hkv, Lq, Lk, d, scale, causal, window, 1, nullptr, stream);
+}
+
+int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int* seqlens_q,
+                    const int* seqlens_k, int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale, int causal,
+                    int window, void* stream) {
+  return fwd_impl(q, k, v, o, lse, seqlens_q, seqlens_k, B, Hq, Hkv, Lq, Lk, d, scale, causal, window, 1, nullptr,
+                  stream);
 }
 
 // ------------------------------------------------------------------ split-KV forward
@@ -203,40 +236,14 @@ int attn_fwd_split(const void* q, const void* k, const void* v, void* o, float* 
                    size_t workspace_bytes, void* stream) {
   if (n_split < 1 || n_split > kMaxSplit) return ATTN_ERR_INVALID_ARG;
   if (n_split == 1) return attn_fwd(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, scale, causal, window, stream);
-  int st = check_shape(B, Hq, Hkv, Lq, Lk, d, scale, causal, window);
+  const int st = check_shape(B, Hq, Hkv, Lq, Lk, d, scale, causal, window);
   if (st != ATTN_OK) return st;
   if (B == 0 || Hq == 0 || Lq == 0) return ATTN_OK;
-  if (!q || !o || !lse || !aligned16(q) || !aligned16(o) || !aligned16(lse)) return ATTN_ERR_INVALID_ARG;
-  if (Lk > 0 && (!k || !v || !aligned16(k) || !aligned16(v))) return ATTN_ERR_INVALID_ARG;
   const size_t need = attn_fwd_split_workspace_size(B, Hq, Hkv, Lq, Lk, d, n_split);
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need)
     return ATTN_ERR_INVALID_ARG;
-  EncodeTiledFn enc;
-  if ((st = get_encoder(&enc)) != ATTN_OK) return st;
-  FwdParams P;
-  memset(&P, 0, sizeof(P));
-  P.prob = Problem{B, Hq, Hkv, Lq, Lk, d, causal, window, scale};
-  const void* kp = Lk > 0 ? k : q;
-  const void* vp = Lk > 0 ? v : q;
-  if ((st = make_map(enc, &P.tm_q, q, B * Hq, Lq, d)) != ATTN_OK) return st;
-  if ((st = make_map(enc, &P.tm_k, kp, Lk > 0 ? B * Hkv : B * Hq, Lk > 0 ? Lk : Lq, d)) != ATTN_OK) return st;
-  if ((st = make_map(enc, &P.tm_v, vp, Lk > 0 ? B * Hkv : B * Hq, Lk > 0 ? Lk : Lq, d)) != ATTN_OK) return st;
-  P.o = o;
-  P.lse = lse;
-  P.scale_log2 = scale * 1.4426950408889634f;
-  fwd_plan(P.prob, &P.n_units, &P.pair_heads);
-  P.n_split = n_split;
-  const size_t rows = (size_t)B * Hq * Lq;
-  P.part_o = static_cast<float*>(workspace);
-  P.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
-                                        ((size_t)n_split * rows * d * 4 + 255) / 256 * 256);
-  if ((int64_t)P.n_units * n_split > 0x7fffffff) return ATTN_ERR_UNSUPPORTED;
-  if ((st = get_err_word(&P.err)) != ATTN_OK) return st;
-  P.limit_ns = kWaitLimitNs;
-  cudaError_t e = launch_fwd(P, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail("attn_fwd_split launch", e);
-  e = launch_fwd_merge(P, static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? ATTN_OK : cuda_fail("attn_fwd_split merge launch", e);
+  return fwd_impl(q, k, v, o, lse, nullptr, nullptr, B, Hq, Hkv, Lq, Lk, d, scale, causal, window, n_split, workspace,
+                  stream);
 }
 
 size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int Lq, int Lk, int d) {
@@ -273,9 +280,9 @@ int attn_bwd_preprocess(const void* o, const void* dO, int B, int Hq, int Lq, in
   return e == cudaSuccess ? ATTN_OK : cuda_fail("attn_bwd_preprocess launch", e);
 }
 
-int attn_bwd_main(const void* q, const void* k, const void* v, const float* lse, const void* dO, void* dk, void* dv,
-                  int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale, int causal, int window, void* workspace,
-                  size_t workspace_bytes, void* stream) {
+static int bwd_main_impl(const void* q, const void* k, const void* v, const float* lse, const void* dO, void* dk,
+                         void* dv, const int* lens_q, const int* lens_k, int B, int Hq, int Hkv, int Lq, int Lk, int d,
+                         float scale, int causal, int window, void* workspace, size_t workspace_bytes, void* stream) {
   int st = check_shape(B, Hq, Hkv, Lq, Lk, d, scale, causal, window);
   if (st != ATTN_OK) return st;
   if (B == 0 || Hq == 0 || Lk == 0) return ATTN_OK;
@@ -295,7 +302,11 @@ int attn_bwd_main(const void* q, const void* k, const void* v, const float* lse,
   if ((st = get_encoder(&enc)) != ATTN_OK) return st;
   BwdParams P;
   memset(&P, 0, sizeof(P));
+  if ((lens_q && (reinterpret_cast<uintptr_t>(lens_q) & 3u)) || (lens_k && (reinterpret_cast<uintptr_t>(lens_k) & 3u)))
+    return ATTN_ERR_INVALID_ARG;
   P.prob = Problem{B, Hq, Hkv, Lq, Lk, d, causal, window, scale};
+  P.prob.len_q = lens_q;
+  P.prob.len_k = lens_k;
   const int bm = bwd_block_m(d);
   if ((st = make_map(enc, &P.tm_q, q, B * Hq, Lq, d, bm)) != ATTN_OK) return st;
   if ((st = make_map(enc, &P.tm_do, dO, B * Hq, Lq, d, bm)) != ATTN_OK) return st;
@@ -328,6 +339,21 @@ int attn_bwd_main(const void* q, const void* k, const void* v, const float* lse,
   return e == cudaSuccess ? ATTN_OK : cuda_fail("attn_bwd_main launch", e);
 }
 
+int attn_bwd_main(const void* q, const void* k, const void* v, const float* lse, const void* dO, void* dk, void* dv,
+                  int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale, int causal, int window, void* workspace,
+                  size_t workspace_bytes, void* stream) {
+  return bwd_main_impl(q, k, v, lse, dO, dk, dv, nullptr, nullptr, B, Hq, Hkv, Lq, Lk, d, scale, causal, window,
+                       workspace, workspace_bytes, stream);
+}
+
+int attn_bwd_main_varlen(const void* q, const void* k, const void* v, const float* lse, const void* dO, void* dk,
+                         void* dv, const int* seqlens_q, const int* seqlens_k, int B, int Hq, int Hkv, int Lq, int Lk,
+                         int d, float scale, int causal, int window, void* workspace, size_t workspace_bytes,
+                         void* stream) {
+  return bwd_main_impl(q, k, v, lse, dO, dk, dv, seqlens_q, seqlens_k, B, Hq, Hkv, Lq, Lk, d, scale, causal, window,
+                       workspace, workspace_bytes, stream);
+}
+
 int attn_bwd_finalize(void* dq, int B, int Hq, int Lq, int d, float scale, void* workspace, size_t workspace_bytes,
                       void* stream) {
   int st = check_shape(B, Hq, Hq > 0 ? 1 : 0, Lq, 1, d, scale, 0, 0);
@@ -340,16 +366,17 @@ int attn_bwd_finalize(void* dq, int B, int Hq, int Lq, int d, float scale, void*
   return e == cudaSuccess ? ATTN_OK : cuda_fail("attn_bwd_finalize launch", e);
 }
 
-int attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO, void* dq,
-             void* dk, void* dv, int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale, int causal, int window,
-             void* workspace, size_t workspace_bytes, void* stream) {
+static int bwd_impl(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                    void* dq, void* dk, void* dv, const int* lens_q, const int* lens_k, int B, int Hq, int Hkv, int Lq,
+                    int Lk, int d, float scale, int causal, int window, void* workspace, size_t workspace_bytes,
+                    void* stream) {
   int st = check_shape(B, Hq, Hkv, Lq, Lk, d, scale, causal, window);
   if (st != ATTN_OK) return st;
   if (B == 0 || Hq == 0) return ATTN_OK;
   if (Lq == 0 || Lk == 0) {
     if (Lq == 0)  // dK = dV = 0
-      return attn_bwd_main(q, k, v, lse, dO, dk, dv, B, Hq, Hkv, Lq, Lk, d, scale, causal, window, workspace,
-                           workspace_bytes, stream);
+      return bwd_main_impl(q, k, v, lse, dO, dk, dv, lens_q, lens_k, B, Hq, Hkv, Lq, Lk, d, scale, causal, window,
+                           workspace, workspace_bytes, stream);
     // No key: every row is fully masked, dQ = 0.
     if (!dq || !aligned16(dq)) return ATTN_ERR_INVALID_ARG;
     const cudaError_t e = cudaMemsetAsync(dq, 0, (size_t)B * Hq * Lq * d * 2, static_cast<cudaStream_t>(stream));
@@ -362,10 +389,25 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
   float *dvec, *dq_acc;
   if ((st = split_workspace(B, Hq, Lq, d, workspace, workspace_bytes, &dvec, &dq_acc)) != ATTN_OK) return st;
   if ((st = attn_bwd_preprocess(o, dO, B, Hq, Lq, d, workspace, workspace_bytes, stream)) != ATTN_OK) return st;
-  if ((st = attn_bwd_main(q, k, v, lse, dO, dk, dv, B, Hq, Hkv, Lq, Lk, d, scale, causal, window, workspace,
-                          workspace_bytes, stream)) != ATTN_OK)
+  if ((st = bwd_main_impl(q, k, v, lse, dO, dk, dv, lens_q, lens_k, B, Hq, Hkv, Lq, Lk, d, scale, causal, window,
+                          workspace, workspace_bytes, stream)) != ATTN_OK)
     return st;
   return attn_bwd_finalize(dq, B, Hq, Lq, d, scale, workspace, workspace_bytes, stream);
+}
+
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO, void* dq,
+             void* dk, void* dv, int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale, int causal, int window,
+             void* workspace, size_t workspace_bytes, void* stream) {
+  return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, nullptr, nullptr, B, Hq, Hkv, Lq, Lk, d, scale, causal, window,
+                  workspace, workspace_bytes, stream);
+}
+
+int attn_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                    void* dq, void* dk, void* dv, const int* seqlens_q, const int* seqlens_k, int B, int Hq, int Hkv,
+                    int Lq, int Lk, int d, float scale, int causal, int window, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+  return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, seqlens_q, seqlens_k, B, Hq, Hkv, Lq, Lk, d, scale, causal, window,
+                  workspace, workspace_bytes, stream);
 }
 
 const char* attn_last_cuda_error(void) { return g_last_err; }

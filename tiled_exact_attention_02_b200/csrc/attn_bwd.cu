@@ -129,7 +129,7 @@ __device__ __forceinline__ Unit decode_unit(const BwdParams& P, int idx) {
   u.k0 = n * BN;
   u.G = p.Hq / p.Hkv;
   int q_lo, q_hi;
-  q_row_range(p, u.k0, u.k0 + BN, q_lo, q_hi);
+  q_row_range(seq_problem(p, u.b), u.k0, u.k0 + BN, q_lo, q_hi);
   constexpr int BM = Cfg<D>::BM;
   u.qt_lo = q_lo / BM;
   u.nq = q_hi > q_lo ? cdiv(q_hi, BM) - u.qt_lo : 0;
@@ -320,10 +320,11 @@ __device__ void grad_rows(const BwdParams& P, const Unit& u, uint8_t* smem, Bars
   const uint32_t lane_base = (uint32_t)(wl * 32) << 16;
   // Queries [vis_lo, vis_hi) see this key.
   int vis_lo = 0, vis_hi = 0;
-  if (key < p.Lk) {
-    const int off = diag_off(p);
-    vis_lo = p.causal ? imax(0, key - off) : (p.window > 0 ? imax(0, key - p.window + 1) : 0);
-    vis_hi = p.window > 0 ? imin(p.Lq, key - off + p.window) : p.Lq;
+  const Problem ps = seq_problem(p, u.b);  // this sequence's lengths (padded batches)
+  if (key < ps.Lk) {
+    const int off = diag_off(ps);
+    vis_lo = ps.causal ? imax(0, key - off) : (ps.window > 0 ? imax(0, key - ps.window + 1) : 0);
+    vis_hi = ps.window > 0 ? imin(ps.Lq, key - off + ps.window) : ps.Lq;
   }
   const float c = P.scale_log2;
   float* vec = reinterpret_cast<float*>(smem + C::OFF_VEC) + grp * (2 * 2 * CW);
@@ -341,7 +342,7 @@ __device__ void grad_rows(const BwdParams& P, const Unit& u, uint8_t* smem, Bars
     const int q = q0 + col0 + row;
     l = INFINITY;
     dv = 0.f;
-    if (row < CW && q < p.Lq) {
+    if (row < CW && q < ps.Lq) {
       const size_t r = (size_t)(u.b * p.Hq + h) * p.Lq + q;
       l = P.lse[r];
       dv = P.dvec[r];

@@ -23,7 +23,22 @@ struct Problem {
   int B, Hq, Hkv, Lq, Lk, d;
   int causal, window;  // causal: 0 none, 1 top-left, 2 bottom-right
   float scale;
+  // Optional per-sequence lengths of a padded batch (device int32 [B], may be
+  // null): sequence b uses only its first len_q[b] queries and len_k[b] keys
+  // (clamped to [0, Lq] and [0, Lk]); Lq and Lk stay the padded extents that
+  // every tensor is laid out with.
+  const int* len_q = nullptr;
+  const int* len_k = nullptr;
 };
+
+// The problem of sequence b: Lq and Lk replaced by its own lengths (for the
+// masks and tile ranges; indexing keeps using the padded extents).
+__device__ inline Problem seq_problem(const Problem& p, int b) {
+  Problem s = p;
+  if (p.len_q) s.Lq = p.len_q[b] < 0 ? 0 : (p.len_q[b] > p.Lq ? p.Lq : p.len_q[b]);
+  if (p.len_k) s.Lk = p.len_k[b] < 0 ? 0 : (p.len_k[b] > p.Lk ? p.Lk : p.len_k[b]);
+  return s;
+}
 
 __host__ __device__ inline int imin(int a, int b) { return a < b ? a : b; }
 __host__ __device__ inline int imax(int a, int b) { return a > b ? a : b; }
@@ -34,6 +49,10 @@ __host__ __device__ inline int diag_off(const Problem& p) { return p.causal == 2
 
 // Keys [key_lo, key_hi) visible to query row i (empty when key_lo >= key_hi).
 __host__ __device__ inline void row_key_range(const Problem& p, int i, int& key_lo, int& key_hi) {
+  if (i >= p.Lq) {  // a row past the (sequence's) queries sees nothing
+    key_lo = key_hi = 0;
+    return;
+  }
   const int off = diag_off(p);
   key_hi = p.causal ? imin(p.Lk, i + off + 1) : (p.window > 0 ? imin(p.Lk, i + p.window) : p.Lk);
   key_lo = p.window > 0 ? imax(0, i + off - p.window + 1) : 0;

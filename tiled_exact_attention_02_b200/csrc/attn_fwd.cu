@@ -151,10 +151,11 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& P, int idx) {
     u.q0[1] = qi * 2 * BM + BM;
   }
   u.kvh = u.head[0] / G;
+  const Problem ps = seq_problem(p, u.b);  // this sequence's lengths (padded batches)
   u.ulo = 1 << 30;
   u.uhi = 0;
   for (int s = 0; s < 2; s++) {
-    kv_tile_range(p, u.q0[s], u.q0[s] + BM, BN, u.lo[s], u.hi[s]);
+    kv_tile_range(ps, u.q0[s], u.q0[s] + BM, BN, u.lo[s], u.hi[s]);
     if (u.lo[s] < u.hi[s]) {
       u.ulo = imin(u.ulo, u.lo[s]);
       u.uhi = imax(u.uhi, u.hi[s]);
@@ -325,7 +326,7 @@ __device__ void softmax_slot(const FwdParams& P, const Unit& u, int s, Bars& bar
   const int head_s = s ? u.head[1] : u.head[0];
   const int q_row = (s ? u.q0[1] : u.q0[0]) + row;
   int key_lo, key_hi;
-  row_key_range(p, q_row, key_lo, key_hi);
+  row_key_range(seq_problem(p, u.b), q_row, key_lo, key_hi);
   const float c = P.scale_log2;
   const uint32_t lane_base = (uint32_t)(wl * 32) << 16;
   const uint32_t t_s = tmem + lane_base + s_col(s);
