@@ -46,9 +46,11 @@ def diag_offset(causal, Lq: int, Lk: int) -> int:
     return Lk - Lq if causal == 2 else 0
 
 
-def _visible(i, j, causal, window: int, off: int = 0) -> np.ndarray:
+def _visible(i, j, causal, window: int, off: int = 0, glob=(0, 0, 0)) -> np.ndarray:
     """Elementwise visibility of key j to query i (broadcasting arrays);
-    `off` is diag_offset(causal, Lq, Lk)."""
+    `off` is diag_offset(causal, Lq, Lk); glob = (global_head, global_tail, Lk):
+    the first global_head and the last global_tail key positions are visible
+    to every query (still subject to the causal mask)."""
     vis = np.ones(np.broadcast(i, j).shape, dtype=bool)
     if causal:
         vis &= j <= i + off
@@ -56,10 +58,16 @@ def _visible(i, j, causal, window: int, off: int = 0) -> np.ndarray:
         vis &= j > i + off - window
         if not causal:
             vis &= j < i + window
+    gh, gt, lk = glob
+    if gh > 0 or gt > 0:
+        g = (j < gh) | (j >= lk - gt)
+        if causal:
+            g = g & (j <= i + off)
+        vis = vis | g
     return vis
 
 
-def visible_mask(Lq: int, Lk: int, causal, window: int) -> np.ndarray:
+def visible_mask(Lq: int, Lk: int, causal, window: int, global_head: int = 0, global_tail: int = 0) -> np.ndarray:
     """Boolean [Lq, Lk]: True where key j is visible to query i.
 
     Causal: j <= i (causal = 2: j <= i + Lk - Lq).  Window w > 0: the w keys
@@ -67,18 +75,19 @@ def visible_mask(Lq: int, Lk: int, causal, window: int) -> np.ndarray:
     sliding window); without causal the band reaches w - 1 keys to either
     side, i - w < j < i + w (the two-sided "前后" reading of the same section).
     """
-    return _visible(np.arange(Lq)[:, None], np.arange(Lk)[None, :], causal, window, diag_offset(causal, Lq, Lk))
+    return _visible(np.arange(Lq)[:, None], np.arange(Lk)[None, :], causal, window, diag_offset(causal, Lq, Lk),
+                    (global_head, global_tail, Lk))
 
 
-def visible_band(r0: int, r1: int, Lk: int, causal, window: int, off: int = 0) -> tuple[int, int]:
+def visible_band(r0: int, r1: int, Lk: int, causal, window: int, off: int = 0, glob=(0, 0, 0)) -> tuple[int, int]:
     """Columns [lo, hi) that can be visible to any row in [r0, r1)."""
     if causal:
         hi = min(Lk, r1 + off)
-    elif window > 0:
+    elif window > 0 and glob[1] == 0:
         hi = min(Lk, r1 - 1 + window)
     else:
         hi = Lk
-    lo = max(0, r0 + off - window + 1) if window > 0 else 0
+    lo = max(0, r0 + off - window + 1) if window > 0 and glob[0] == 0 else 0
     return lo, max(lo, hi)
 
 
@@ -107,7 +116,7 @@ def attention_weights(q, k, scale: float, vis: np.ndarray):
     return A, lse
 
 
-def _head_fwd(qh, kh, vh, scale, causal, window, rows=None):
+def _head_fwd(qh, kh, vh, scale, causal, window, rows=None, gl=(0, 0)):
     """O and LSE for the rows `rows` (default: all) of one head."""
     Lq, Lk = qh.shape[0], kh.shape[0]
     off = diag_offset(causal, Lq, Lk)
@@ -123,8 +132,9 @@ def _head_fwd(qh, kh, vh, scale, causal, window, rows=None):
         stop = min(rows.size, start + step)
         blk = rows[start:stop]
         r0, r1 = int(blk.min()), int(blk.max()) + 1
-        lo, hi = visible_band(r0, r1, Lk, causal, window, off)
-        vis = _band_mask(blk, lo, hi, causal, window, off)
+        glob = (gl[0], gl[1], Lk)
+        lo, hi = visible_band(r0, r1, Lk, causal, window, off, glob)
+        vis = _band_mask(blk, lo, hi, causal, window, off, glob)
         A, l = attention_weights(qh[blk], kh[lo:hi], scale, vis)
         O[start:stop] = A @ vh[lo:hi]
         lse[start:stop] = l
@@ -132,8 +142,8 @@ def _head_fwd(qh, kh, vh, scale, causal, window, rows=None):
     return O, lse
 
 
-def _band_mask(rows, lo, hi, causal, window, off):
-    return _visible(np.asarray(rows)[:, None], np.arange(lo, hi)[None, :], causal, window, off)
+def _band_mask(rows, lo, hi, causal, window, off, glob=(0, 0, 0)):
+    return _visible(np.asarray(rows)[:, None], np.arange(lo, hi)[None, :], causal, window, off, glob)
 
 
 def _group(Hq: int, Hkv: int) -> int:
@@ -152,7 +162,7 @@ def _lengths(seqlens, b: int, full: int) -> int:
 
 
 def attn_fwd(q, k, v, scale: float, causal: bool = False, window: int = 0, heads=None, seqlens_q=None,
-             seqlens_k=None):
+             seqlens_k=None, global_head: int = 0, global_tail: int = 0):
     """O [B,Hq,Lq,d] and LSE [B,Hq,Lq] in float64.
 
     q: [B,Hq,Lq,d]; k, v: [B,Hkv,Lk,d] (float or bf16 bits as uint16).
@@ -175,7 +185,8 @@ def attn_fwd(q, k, v, scale: float, causal: bool = False, window: int = 0, heads
         nq, nk = _lengths(seqlens_q, b, Lq), _lengths(seqlens_k, b, Lk)
         O[b, h] = 0.0
         lse[b, h] = -np.inf
-        O[b, h, :nq], lse[b, h, :nq] = _head_fwd(q[b, h, :nq], k[b, g, :nk], v[b, g, :nk], scale, causal, window)
+        O[b, h, :nq], lse[b, h, :nq] = _head_fwd(q[b, h, :nq], k[b, g, :nk], v[b, g, :nk], scale, causal, window,
+                                                 gl=(global_head, global_tail))
     return O, lse
 
 
@@ -203,13 +214,14 @@ def attn_fwd_rows(q, k, v, scale, causal, window, b, h, rows):
     return O, lse
 
 
-def _rows_bwd(qh, kh, vh, doh, scale, causal, window, r0, r1):
+def _rows_bwd(qh, kh, vh, doh, scale, causal, window, r0, r1, gl=(0, 0)):
     """Rows [r0, r1) of one head: their O and LSE, their dQ rows, and their
     contributions to dK and dV over the visible key band [lo, hi)."""
     Lq, Lk = qh.shape[0], kh.shape[0]
     off = diag_offset(causal, Lq, Lk)
-    lo, hi = visible_band(r0, r1, Lk, causal, window, off)
-    vis = _band_mask(np.arange(r0, r1), lo, hi, causal, window, off)
+    glob = (gl[0], gl[1], Lk)
+    lo, hi = visible_band(r0, r1, Lk, causal, window, off, glob)
+    vis = _band_mask(np.arange(r0, r1), lo, hi, causal, window, off, glob)
     A, lse = attention_weights(qh[r0:r1], kh[lo:hi], scale, vis)
     O = A @ vh[lo:hi]
     dO = doh[r0:r1]
@@ -222,7 +234,7 @@ def _rows_bwd(qh, kh, vh, doh, scale, causal, window, r0, r1):
     return lo, hi, O, lse, dq, dk, dv
 
 
-def _head_bwd(qh, kh, vh, doh, scale, causal, window):
+def _head_bwd(qh, kh, vh, doh, scale, causal, window, gl=(0, 0)):
     """dQ, dK, dV for one (query head, kv head) pair; textbook softmax gradient."""
     Lq, Lk = qh.shape[0], kh.shape[0]
     dq = np.zeros_like(qh)
@@ -231,7 +243,7 @@ def _head_bwd(qh, kh, vh, doh, scale, causal, window):
     step = max(1, _ROW_BLOCK_ELEMS // max(1, Lk))
     for r0 in range(0, Lq, step):
         r1 = min(Lq, r0 + step)
-        lo, hi, _, _, dqb, dkb, dvb = _rows_bwd(qh, kh, vh, doh, scale, causal, window, r0, r1)
+        lo, hi, _, _, dqb, dkb, dvb = _rows_bwd(qh, kh, vh, doh, scale, causal, window, r0, r1, gl)
         dq[r0:r1] = dqb
         dk[lo:hi] += dkb
         dv[lo:hi] += dvb
@@ -252,13 +264,14 @@ def attn_row_block(q, k, v, do, scale, causal, window, b, h, r0, r1):
 
 
 def attn_bwd(q, k, v, do, scale: float, causal: bool = False, window: int = 0, heads=None, seqlens_q=None,
-             seqlens_k=None):
+             seqlens_k=None, global_head: int = 0, global_tail: int = 0):
     """dQ [B,Hq,Lq,d], dK and dV [B,Hkv,Lk,d] in float64.
 
     dK/dV of a K/V head are summed over the query heads that share it.
     heads: optional list of (b, hkv): only those K/V heads (and all query
     heads of their groups) are evaluated; the rest is left NaN.
-    seqlens_q / seqlens_k: as attn_fwd; padded rows and keys get zero gradients.
+    seqlens_q / seqlens_k, global_head / global_tail: as attn_fwd; padded rows
+    and keys get zero gradients.
     """
     q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
     B, Hq, Lq, d = q.shape
@@ -274,7 +287,8 @@ def attn_bwd(q, k, v, do, scale: float, causal: bool = False, window: int = 0, h
         dv[b, g] = 0.0
         for h in (h for h in range(Hq) if _kv_head(h, Hq, Hkv) == g):
             dq[b, h] = 0.0
-            dqh, dkh, dvh = _head_bwd(q[b, h, :nq], k[b, g, :nk], v[b, g, :nk], do[b, h, :nq], scale, causal, window)
+            dqh, dkh, dvh = _head_bwd(q[b, h, :nq], k[b, g, :nk], v[b, g, :nk], do[b, h, :nq], scale, causal, window,
+                                      (global_head, global_tail))
             dq[b, h, :nq] = dqh
             dk[b, g, :nk] += dkh
             dv[b, g, :nk] += dvh

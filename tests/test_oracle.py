@@ -221,6 +221,54 @@ def test_padded_batch_matches_torch_sdpa_key_padding_mask():
     np.testing.assert_allclose(O, ref.numpy(), atol=1e-12)
 
 
+@pytest.mark.parametrize("causal,w,gh,gt", [(False, 4, 1, 1), (False, 3, 5, 0), (True, 4, 2, 0), (2, 3, 1, 2),
+                                             (False, 0, 3, 3)])
+def test_global_tokens_match_torch_sdpa(causal, w, gh, gt):
+    """Leading / trailing global key positions on top of a window, against torch
+    SDPA with the mask built here from its own expression."""
+    B, H, Lq, Lk, d = 1, 2, 20, 20 if causal != 2 else 26, 6
+    q, k, v = _rand(B, H, Lq, d), _rand(B, H, Lk, d), _rand(B, H, Lk, d)
+    O, _ = oracle.attn_fwd(q, k, v, 0.4, causal, w, global_head=gh, global_tail=gt)
+    i = torch.arange(Lq)[:, None]
+    j = torch.arange(Lk)[None, :]
+    off = Lk - Lq if causal == 2 else 0
+    base = torch.ones(Lq, Lk, dtype=torch.bool)
+    if causal:
+        base &= j <= i + off
+        if w:
+            base &= j > i + off - w
+    elif w:
+        base &= (i - j).abs() < w
+    glob = ((j < gh) | (j >= Lk - gt)).expand(Lq, Lk)
+    if causal:
+        glob = glob & (j <= i + off)
+    mask = base | glob
+    ref = torch.nn.functional.scaled_dot_product_attention(*(torch.from_numpy(x) for x in (q, k, v)),
+                                                           attn_mask=mask, scale=0.4)
+    np.testing.assert_allclose(O, ref.numpy(), atol=1e-12)
+
+
+def test_global_tokens_backward_finite_differences():
+    """Gradient with global head/tail keys on a two-sided window, against central differences."""
+    rng = np.random.default_rng(11)
+    q, k, v, R = (rng.standard_normal((1, 2, 9, 3)) for _ in range(4))
+    dq, dk, dv = oracle.attn_bwd(q, k, v, R, 0.5, False, 2, global_head=1, global_tail=2)
+    eps = 1e-5
+    for X, G in ((q, dq), (k, dk), (v, dv)):
+        num = np.zeros_like(X)
+        it = np.nditer(X, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            old = X[idx]
+            X[idx] = old + eps
+            fp = float(np.sum(oracle.attn_fwd(q, k, v, 0.5, False, 2, global_head=1, global_tail=2)[0] * R))
+            X[idx] = old - eps
+            fm = float(np.sum(oracle.attn_fwd(q, k, v, 0.5, False, 2, global_head=1, global_tail=2)[0] * R))
+            X[idx] = old
+            num[idx] = (fp - fm) / (2 * eps)
+        np.testing.assert_allclose(G, num, atol=1e-6, rtol=0)
+
+
 def test_value_shift_and_score_shift_invariance():
     """V + 1 c^T gives O + 1 c^T; a per-row constant added to the logits changes nothing."""
     L, d = 19, 4
@@ -536,9 +584,9 @@ def _transposed_weights(orig, q, k, s, vis):
 
 
 def _bwd_with(ds_fn, dk_scale=True):
-    def head_bwd(qh, kh, vh, doh, scale, causal, window):
+    def head_bwd(qh, kh, vh, doh, scale, causal, window, gl=(0, 0)):
         Lq, Lk = qh.shape[0], kh.shape[0]
-        vis = oracle.visible_mask(Lq, Lk, causal, window)
+        vis = oracle.visible_mask(Lq, Lk, causal, window, *gl)
         A, _ = oa.attention_weights(qh, kh, scale, vis)
         O = A @ vh
         dP = doh @ vh.T
