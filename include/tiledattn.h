@@ -87,6 +87,41 @@ ATTN_API int attn_fwd(const void* q, const void* k, const void* v, void* o, floa
              int Lk, int d, float scale, int causal, int window, void* stream);
 
 /*
+ * Every mask option at once, for attn_fwd_ex / attn_bwd_ex.
+ *  causal, window          as attn_fwd (causal 0 / 1 / 2, window 0 or w > 0)
+ *  global_head, global_tail  >= 0: that many leading / trailing key positions
+ *                          (of each sequence) are visible to every query on
+ *                          top of the window, still subject to the causal
+ *                          mask ("大模型高效注意力机制全解析" §5.1.2,
+ *                          global_tokens [0, -1]: the first and last tokens
+ *                          globally visible); 0 for none
+ *  seqlens_q, seqlens_k    as attn_fwd_varlen (device int32 [B] or NULL)
+ */
+typedef struct {
+  int causal;
+  int window;
+  int global_head;
+  int global_tail;
+  const int* seqlens_q;
+  const int* seqlens_k;
+} attn_mask;
+
+/*
+ * Forward pass with any combination of the mask options above, optionally
+ * split across the key range (n_split as attn_fwd_split, 1 = no split; the
+ * workspace is only needed for n_split > 1).  Global tokens add the key
+ * tiles of the global positions to each query tile's walk.
+ */
+ATTN_API int attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                         int Lq, int Lk, int d, float scale, const attn_mask* mask, int n_split, void* workspace,
+                         size_t workspace_bytes, void* stream);
+
+/* Backward pass with any combination of the mask options (workspace as attn_bwd). */
+ATTN_API int attn_bwd_ex(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                         const void* dO, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Lq, int Lk, int d,
+                         float scale, const attn_mask* mask, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Forward pass over a padded batch of sequences of different lengths
  * ("大模型高效注意力机制全解析" §5.2.2: requests are padded into one batch and
  * each output cut back to its own length).  Tensors keep the padded [B, H, L,

@@ -142,3 +142,19 @@ def test_causal_argument_codes(ta):
     assert [f(x) for x in ("none", "top_left", "bottom_right")] == [0, 1, 2]
     with pytest.raises(ValueError):
         f("diagonal")
+
+
+def test_fwd_ex_and_bwd_ex_validate_the_mask(ta):
+    """attn_fwd_ex / attn_bwd_ex: a NULL mask, negative global counts and a bad
+    slice count are rejected before any launch."""
+    import ctypes
+    m = ta.AttnMask(1, 0, -1, 0, None, None)
+    args = (P, P, P, P, P, 1, 2, 2, 8, 8, 64, 0.125)
+    assert ta.lib.attn_fwd_ex(*args, None, 1, None, 0, None) == 1
+    assert ta.lib.attn_fwd_ex(*args, ctypes.byref(m), 1, None, 0, None) == 1
+    m.global_head = 0
+    assert ta.lib.attn_fwd_ex(*args, ctypes.byref(m), 0, None, 0, None) == 1
+    assert ta.lib.attn_fwd_ex(*args, ctypes.byref(m), 4, None, 0, None) == 1  # split needs a workspace
+    m.global_tail = -2
+    assert ta.lib.attn_bwd_ex(*([P] * 9), 1, 2, 2, 8, 8, 64, 0.125, ctypes.byref(m), P, 1 << 20, None) == 1
+    assert ta.lib.attn_bwd_ex(*([P] * 9), 1, 2, 2, 8, 8, 64, 0.125, None, P, 1 << 20, None) == 1

@@ -104,6 +104,31 @@ def test_bwd_varlen(ta, B, Hq, Hkv, Lq, Lk, d, causal, window, lq, lk):
         assert np.all(to_f64(dk)[b, :, lk[b]:] == 0) and np.all(to_f64(dv)[b, :, lk[b]:] == 0)
 
 
+GLOBAL = [
+    (1, 2, 2, 700, 700, 128, 0, 64, 1, 1),
+    (1, 4, 2, 1000, 1000, 128, 1, 128, 4, 0),
+    (2, 2, 1, 300, 500, 64, 2, 50, 130, 20),
+    (1, 2, 2, 257, 257, 128, 0, 8, 0, 3),
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Lq,Lk,d,causal,window,gh,gt", GLOBAL)
+def test_bwd_global_tokens(ta, B, Hq, Hkv, Lq, Lk, d, causal, window, gh, gt):
+    """Gradients with global head/tail key positions, against the oracle."""
+    x = make_shape_inputs(B, Hq, Hkv, Lq, Lk, d, seed=Lq * 19 + Lk + d + gh + 5 * gt, with_do=True)
+    scale = d ** -0.5
+    q, k, v, do = (to_dev(x[n]) for n in ("q", "k", "v", "do"))
+    o, lse = ta.attention(q, k, v, causal, window, scale, global_head=gh, global_tail=gt)
+    dq, dk, dv = ta.attention_backward(q, k, v, o, lse, do, causal, window, scale, global_head=gh, global_tail=gt)
+    st, site = ta.device_error()
+    assert st == 0, f"device error {st} at site {site}"
+    rq, rk, rv = oracle.attn_bwd(x["q"], x["k"], x["v"], x["do"], scale, causal, window, global_head=gh,
+                                 global_tail=gt)
+    check_grad(to_f64(dq), rq, "dQ")
+    check_grad(to_f64(dk), rk, "dK")
+    check_grad(to_f64(dv), rv, "dV")
+
+
 def test_bwd_gqa_window_2048(ta):
     x = make_shape_inputs(1, 8, 2, 2048, 2048, 128, seed=17, with_do=True)
     dq, dk, dv = run_fwd_bwd(ta, x, True, 300, 128 ** -0.5)

@@ -123,6 +123,57 @@ def test_fwd_varlen(ta, B, Hq, Hkv, Lq, Lk, d, causal, window, lq, lk):
     check_lse(to_f64(lse), rl, "LSE")
 
 
+# (B, Hq, Hkv, Lq, Lk, d, causal, window, global_head, global_tail)
+GLOBAL = [
+    (1, 2, 2, 700, 700, 128, 0, 64, 1, 1),
+    (1, 4, 2, 1000, 1000, 128, 1, 128, 4, 0),
+    (2, 2, 1, 300, 500, 64, 2, 50, 130, 20),
+    (1, 2, 2, 257, 257, 128, 0, 8, 0, 3),
+    (1, 2, 2, 400, 400, 128, 0, 0, 5, 5),
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Lq,Lk,d,causal,window,gh,gt", GLOBAL)
+def test_fwd_global_tokens(ta, B, Hq, Hkv, Lq, Lk, d, causal, window, gh, gt):
+    """Global head/tail key positions on top of the window, against the oracle."""
+    x = make_shape_inputs(B, Hq, Hkv, Lq, Lk, d, seed=Lq * 17 + Lk + d + gh + 7 * gt)
+    scale = d ** -0.5
+    q, k, v = (to_dev(x[n]) for n in "qkv")
+    o, lse = ta.attention(q, k, v, causal, window, scale, global_head=gh, global_tail=gt)
+    st, site = ta.device_error()
+    assert st == 0, f"device error {st} at site {site}"
+    ro, rl = oracle.attn_fwd(x["q"], x["k"], x["v"], scale, causal, window, global_head=gh, global_tail=gt)
+    check_o(to_f64(o), ro, "O")
+    check_lse(to_f64(lse), rl, "LSE")
+
+
+def test_fwd_global_tokens_split_and_varlen(ta):
+    """attn_fwd_ex with global tokens, per-sequence lengths and a split key walk at once."""
+    import ctypes
+    import torch
+    B, Hq, Hkv, Lq, Lk, d, w, gh, gt, ns = 2, 4, 2, 100, 2000, 128, 96, 3, 2, 6
+    lq, lk = [100, 37], [2000, 1500]
+    x = make_shape_inputs(B, Hq, Hkv, Lq, Lk, d, seed=99)
+    scale = d ** -0.5
+    q, k, v = (to_dev(x[n]) for n in "qkv")
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device="cuda")
+    tq = torch.tensor(lq, dtype=torch.int32, device="cuda")
+    tk = torch.tensor(lk, dtype=torch.int32, device="cuda")
+    m = ta.AttnMask(2, w, gh, gt, tq.data_ptr(), tk.data_ptr())
+    ws = torch.empty(ta.lib.attn_fwd_split_workspace_size(B, Hq, Hkv, Lq, Lk, d, ns), dtype=torch.uint8, device="cuda")
+    st = ta.lib.attn_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, Hq, Hkv, Lq,
+                            Lk, d, scale, ctypes.byref(m), ns, ws.data_ptr(), ws.numel(),
+                            torch.cuda.current_stream().cuda_stream)
+    assert st == 0
+    st, site = ta.device_error()
+    assert st == 0, f"device error {st} at site {site}"
+    ro, rl = oracle.attn_fwd(x["q"], x["k"], x["v"], scale, 2, w, seqlens_q=lq, seqlens_k=lk, global_head=gh,
+                             global_tail=gt)
+    check_o(to_f64(o), ro, "O")
+    check_lse(to_f64(lse), rl, "LSE")
+
+
 def test_fwd_no_keys(ta):
     """Lk = 0: every row sees nothing: O = 0, LSE = -inf."""
     import torch

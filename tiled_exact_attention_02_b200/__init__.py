@@ -32,6 +32,12 @@ class AttnError(RuntimeError):
         super().__init__(msg)
 
 
+class AttnMask(ctypes.Structure):
+    """The C ABI's attn_mask."""
+    _fields_ = [("causal", ctypes.c_int), ("window", ctypes.c_int), ("global_head", ctypes.c_int),
+                ("global_tail", ctypes.c_int), ("seqlens_q", ctypes.c_void_p), ("seqlens_k", ctypes.c_void_p)]
+
+
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
@@ -52,6 +58,11 @@ def _load() -> ctypes.CDLL:
     lib.attn_bwd_varlen.restype = i
     lib.attn_bwd_main_varlen.argtypes = [vp] * 9 + [i] * 6 + [f, i, i, vp, sz, vp]
     lib.attn_bwd_main_varlen.restype = i
+    mp = ctypes.POINTER(AttnMask)
+    lib.attn_fwd_ex.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, mp, i, vp, sz, vp]
+    lib.attn_fwd_ex.restype = i
+    lib.attn_bwd_ex.argtypes = [vp] * 9 + [i] * 6 + [f, mp, vp, sz, vp]
+    lib.attn_bwd_ex.restype = i
     lib.attn_bwd_workspace_size.argtypes = [i, i, i, i, i, i]
     lib.attn_bwd_workspace_size.restype = sz
     lib.attn_bwd.argtypes = [vp] * 9 + [i] * 6 + [f, i, i, vp, sz, vp]
@@ -133,7 +144,7 @@ def _lens(seqlens, B, name):
 
 
 def fwd(q, k, v, o, lse, causal: bool = False, window: int = 0, scale: float | None = None, stream=None,
-        seqlens_q=None, seqlens_k=None):
+        seqlens_q=None, seqlens_k=None, global_head: int = 0, global_tail: int = 0):
     """attn_fwd on torch tensors (bf16 q/k/v/o, fp32 lse), asynchronous on
     `stream`; with seqlens_q / seqlens_k (int32 CUDA [B]) attn_fwd_varlen."""
     import torch
@@ -145,6 +156,12 @@ def fwd(q, k, v, o, lse, causal: bool = False, window: int = 0, scale: float | N
         raise ValueError("v/o/lse shape mismatch")
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     lq, lk = _lens(seqlens_q, B, "seqlens_q"), _lens(seqlens_k, B, "seqlens_k")
+    if global_head or global_tail:
+        m = AttnMask(_causal_code(causal), int(window), int(global_head), int(global_tail), lq, lk)
+        st = lib.attn_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                             B, Hq, Hkv, Lq, Lk, d, scale, ctypes.byref(m), 1, None, 0, _stream_ptr(stream))
+        _check(st, "attn_fwd_ex")
+        return
     if lq is None and lk is None:
         st = lib.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
                           B, Hq, Hkv, Lq, Lk, d, scale, _causal_code(causal), int(window), _stream_ptr(stream))
@@ -160,7 +177,8 @@ def bwd_workspace_size(B, Hq, Hkv, Lq, Lk, d) -> int:
 
 
 def bwd(q, k, v, o, lse, do, dq, dk, dv, workspace, causal: bool = False, window: int = 0,
-        scale: float | None = None, stream=None, seqlens_q=None, seqlens_k=None):
+        scale: float | None = None, stream=None, seqlens_q=None, seqlens_k=None, global_head: int = 0,
+        global_tail: int = 0):
     """attn_bwd on torch tensors; `workspace` is a uint8 CUDA tensor; with
     seqlens_q / seqlens_k attn_bwd_varlen."""
     import torch
@@ -172,6 +190,13 @@ def bwd(q, k, v, o, lse, do, dq, dk, dv, workspace, causal: bool = False, window
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     lq, lk = _lens(seqlens_q, B, "seqlens_q"), _lens(seqlens_k, B, "seqlens_k")
     wsp, wsb = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    if global_head or global_tail:
+        m = AttnMask(_causal_code(causal), int(window), int(global_head), int(global_tail), lq, lk)
+        st = lib.attn_bwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
+                             dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv, Lq, Lk, d, scale,
+                             ctypes.byref(m), wsp, wsb, _stream_ptr(stream))
+        _check(st, "attn_bwd_ex")
+        return
     if lq is None and lk is None:
         st = lib.attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
                           dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv, Lq, Lk, d, scale,
@@ -211,13 +236,14 @@ def device_error(stream=None) -> tuple[int, int]:
 
 
 def attention(q, k, v, causal: bool = False, window: int = 0, scale: float | None = None, seqlens_q=None,
-              seqlens_k=None):
+              seqlens_k=None, global_head: int = 0, global_tail: int = 0):
     """Allocate O and LSE with torch and run the forward pass."""
     import torch
     B, Hq, Hkv, Lq, Lk, d = _shapes(q, k)
     o = torch.empty_like(q)
     lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
-    fwd(q, k, v, o, lse, causal, window, scale, seqlens_q=seqlens_q, seqlens_k=seqlens_k)
+    fwd(q, k, v, o, lse, causal, window, scale, seqlens_q=seqlens_q, seqlens_k=seqlens_k, global_head=global_head,
+        global_tail=global_tail)
     return o, lse
 
 
@@ -251,13 +277,14 @@ def attention_split(q, k, v, causal: bool = False, window: int = 0, scale: float
 
 
 def attention_backward(q, k, v, o, lse, do, causal: bool = False, window: int = 0, scale: float | None = None,
-                       seqlens_q=None, seqlens_k=None):
+                       seqlens_q=None, seqlens_k=None, global_head: int = 0, global_tail: int = 0):
     """Allocate dQ/dK/dV and the workspace with torch and run the backward pass."""
     import torch
     B, Hq, Hkv, Lq, Lk, d = _shapes(q, k)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     ws = torch.empty(max(1, bwd_workspace_size(B, Hq, Hkv, Lq, Lk, d)), dtype=torch.uint8, device=q.device)
-    bwd(q, k, v, o, lse, do, dq, dk, dv, ws, causal, window, scale, seqlens_q=seqlens_q, seqlens_k=seqlens_k)
+    bwd(q, k, v, o, lse, do, dq, dk, dv, ws, causal, window, scale, seqlens_q=seqlens_q, seqlens_k=seqlens_k,
+        global_head=global_head, global_tail=global_tail)
     return dq, dk, dv
 
 

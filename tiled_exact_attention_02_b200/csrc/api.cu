@@ -146,9 +146,10 @@ const char* attn_status_string(int status) {
 // slices written to `workspace` and merged.
 static int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, const int* lens_q,
                     const int* lens_k, int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale, int causal,
-                    int window, int n_split, void* workspace, void* stream) {
+                    int window, int gh, int gt, int n_split, void* workspace, void* stream) {
   int st = check_shape(B, Hq, Hkv, Lq, Lk, d, scale, causal, window);
   if (st != ATTN_OK) return st;
+  if (gh < 0 || gt < 0) return ATTN_ERR_INVALID_ARG;
   if (B == 0 || Hq == 0 || Lq == 0) return ATTN_OK;
   if (!q || !o || !lse || !aligned16(q) || !aligned16(o) || !aligned16(lse)) return ATTN_ERR_INVALID_ARG;
   if (Lk > 0 && (!k || !v || !aligned16(k) || !aligned16(v))) return ATTN_ERR_INVALID_ARG;
@@ -161,6 +162,8 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, float*
   P.prob = Problem{B, Hq, Hkv, Lq, Lk, d, causal, window, scale};
   P.prob.len_q = lens_q;
   P.prob.len_k = lens_k;
+  P.prob.global_head = gh;
+  P.prob.global_tail = gt;
   // With Lk == 0 nothing reads K/V; map Q's memory so the descriptors stay valid.
   const void* kp = Lk > 0 ? k : q;
   const void* vp = Lk > 0 ? v : q;
@@ -192,14 +195,15 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, float*
 
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Lq,
              int Lk, int d, float scale, int causal, int window, void* stream) {
-  return fwd_impl(q, k, v, o, lse, nullptr, nullptr, B, Hq, Hkv, Lq, Lk, d, scale, causal, window, 1, nullptr, stream);
+  return fwd_impl(q, k, v, o, lse, nullptr, nullptr, B, Hq, Hkv, Lq, Lk, d, scale, causal, window, 0, 0, 1, nullptr,
+                  stream);
 }
 
 int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int* seqlens_q,
                     const int* seqlens_k, int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale, int causal,
                     int window, void* stream) {
-  return fwd_impl(q, k, v, o, lse, seqlens_q, seqlens_k, B, Hq, Hkv, Lq, Lk, d, scale, causal, window, 1, nullptr,
-                  stream);
+  return fwd_impl(q, k, v, o, lse, seqlens_q, seqlens_k, B, Hq, Hkv, Lq, Lk, d, scale, causal, window, 0, 0, 1,
+                  nullptr, stream);
 }
 
 // ------------------------------------------------------------------ split-KV forward
@@ -242,8 +246,8 @@ int attn_fwd_split(const void* q, const void* k, const void* v, void* o, float* 
   const size_t need = attn_fwd_split_workspace_size(B, Hq, Hkv, Lq, Lk, d, n_split);
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need)
     return ATTN_ERR_INVALID_ARG;
-  return fwd_impl(q, k, v, o, lse, nullptr, nullptr, B, Hq, Hkv, Lq, Lk, d, scale, causal, window, n_split, workspace,
-                  stream);
+  return fwd_impl(q, k, v, o, lse, nullptr, nullptr, B, Hq, Hkv, Lq, Lk, d, scale, causal, window, 0, 0, n_split,
+                  workspace, stream);
 }
 
 size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int Lq, int Lk, int d) {
@@ -282,8 +286,10 @@ int attn_bwd_preprocess(const void* o, const void* dO, int B, int Hq, int Lq, in
 
 static int bwd_main_impl(const void* q, const void* k, const void* v, const float* lse, const void* dO, void* dk,
                          void* dv, const int* lens_q, const int* lens_k, int B, int Hq, int Hkv, int Lq, int Lk, int d,
-                         float scale, int causal, int window, void* workspace, size_t workspace_bytes, void* stream) {
+                         float scale, int causal, int window, int gh, int gt, void* workspace,
+                         size_t workspace_bytes, void* stream) {
   int st = check_shape(B, Hq, Hkv, Lq, Lk, d, scale, causal, window);
+  if (st == ATTN_OK && (gh < 0 || gt < 0)) st = ATTN_ERR_INVALID_ARG;
   if (st != ATTN_OK) return st;
   if (B == 0 || Hq == 0 || Lk == 0) return ATTN_OK;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -307,6 +313,8 @@ static int bwd_main_impl(const void* q, const void* k, const void* v, const floa
   P.prob = Problem{B, Hq, Hkv, Lq, Lk, d, causal, window, scale};
   P.prob.len_q = lens_q;
   P.prob.len_k = lens_k;
+  P.prob.global_head = gh;
+  P.prob.global_tail = gt;
   const int bm = bwd_block_m(d);
   if ((st = make_map(enc, &P.tm_q, q, B * Hq, Lq, d, bm)) != ATTN_OK) return st;
   if ((st = make_map(enc, &P.tm_do, dO, B * Hq, Lq, d, bm)) != ATTN_OK) return st;
@@ -342,8 +350,8 @@ static int bwd_main_impl(const void* q, const void* k, const void* v, const floa
 int attn_bwd_main(const void* q, const void* k, const void* v, const float* lse, const void* dO, void* dk, void* dv,
                   int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale, int causal, int window, void* workspace,
                   size_t workspace_bytes, void* stream) {
-  return bwd_main_impl(q, k, v, lse, dO, dk, dv, nullptr, nullptr, B, Hq, Hkv, Lq, Lk, d, scale, causal, window,
-                       workspace, workspace_bytes, stream);
+  return bwd_main_impl(q, k, v, lse, dO, dk, dv, nullptr, nullptr, B, Hq, Hkv, Lq, Lk, d, scale, causal, window, 0,
+                       0, workspace, workspace_bytes, stream);
 }
 
 int attn_bwd_main_varlen(const void* q, const void* k, const void* v, const float* lse, const void* dO, void* dk,
@@ -351,7 +359,7 @@ int attn_bwd_main_varlen(const void* q, const void* k, const void* v, const floa
                          int d, float scale, int causal, int window, void* workspace, size_t workspace_bytes,
                          void* stream) {
   return bwd_main_impl(q, k, v, lse, dO, dk, dv, seqlens_q, seqlens_k, B, Hq, Hkv, Lq, Lk, d, scale, causal, window,
-                       workspace, workspace_bytes, stream);
+                       0, 0, workspace, workspace_bytes, stream);
 }
 
 int attn_bwd_finalize(void* dq, int B, int Hq, int Lq, int d, float scale, void* workspace, size_t workspace_bytes,
@@ -368,15 +376,16 @@ int attn_bwd_finalize(void* dq, int B, int Hq, int Lq, int d, float scale, void*
 
 static int bwd_impl(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
                     void* dq, void* dk, void* dv, const int* lens_q, const int* lens_k, int B, int Hq, int Hkv, int Lq,
-                    int Lk, int d, float scale, int causal, int window, void* workspace, size_t workspace_bytes,
-                    void* stream) {
+                    int Lk, int d, float scale, int causal, int window, int gh, int gt, void* workspace,
+                    size_t workspace_bytes, void* stream) {
   int st = check_shape(B, Hq, Hkv, Lq, Lk, d, scale, causal, window);
   if (st != ATTN_OK) return st;
+  if (gh < 0 || gt < 0) return ATTN_ERR_INVALID_ARG;
   if (B == 0 || Hq == 0) return ATTN_OK;
   if (Lq == 0 || Lk == 0) {
     if (Lq == 0)  // dK = dV = 0
       return bwd_main_impl(q, k, v, lse, dO, dk, dv, lens_q, lens_k, B, Hq, Hkv, Lq, Lk, d, scale, causal, window,
-                           workspace, workspace_bytes, stream);
+                           gh, gt, workspace, workspace_bytes, stream);
     // No key: every row is fully masked, dQ = 0.
     if (!dq || !aligned16(dq)) return ATTN_ERR_INVALID_ARG;
     const cudaError_t e = cudaMemsetAsync(dq, 0, (size_t)B * Hq * Lq * d * 2, static_cast<cudaStream_t>(stream));
@@ -390,7 +399,7 @@ static int bwd_impl(const void* q, const void* k, const void* v, const void* o, 
   if ((st = split_workspace(B, Hq, Lq, d, workspace, workspace_bytes, &dvec, &dq_acc)) != ATTN_OK) return st;
   if ((st = attn_bwd_preprocess(o, dO, B, Hq, Lq, d, workspace, workspace_bytes, stream)) != ATTN_OK) return st;
   if ((st = bwd_main_impl(q, k, v, lse, dO, dk, dv, lens_q, lens_k, B, Hq, Hkv, Lq, Lk, d, scale, causal, window,
-                          workspace, workspace_bytes, stream)) != ATTN_OK)
+                          gh, gt, workspace, workspace_bytes, stream)) != ATTN_OK)
     return st;
   return attn_bwd_finalize(dq, B, Hq, Lq, d, scale, workspace, workspace_bytes, stream);
 }
@@ -398,8 +407,8 @@ static int bwd_impl(const void* q, const void* k, const void* v, const void* o, 
 int attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO, void* dq,
              void* dk, void* dv, int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale, int causal, int window,
              void* workspace, size_t workspace_bytes, void* stream) {
-  return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, nullptr, nullptr, B, Hq, Hkv, Lq, Lk, d, scale, causal, window,
-                  workspace, workspace_bytes, stream);
+  return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, nullptr, nullptr, B, Hq, Hkv, Lq, Lk, d, scale, causal, window, 0,
+                  0, workspace, workspace_bytes, stream);
 }
 
 int attn_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
@@ -407,10 +416,34 @@ int attn_bwd_varlen(const void* q, const void* k, const void* v, const void* o, 
                     int Lq, int Lk, int d, float scale, int causal, int window, void* workspace,
                     size_t workspace_bytes, void* stream) {
   return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, seqlens_q, seqlens_k, B, Hq, Hkv, Lq, Lk, d, scale, causal, window,
-                  workspace, workspace_bytes, stream);
+                  0, 0, workspace, workspace_bytes, stream);
 }
 
 const char* attn_last_cuda_error(void) { return g_last_err; }
+
+int attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Lq,
+                int Lk, int d, float scale, const attn_mask* mask, int n_split, void* workspace,
+                size_t workspace_bytes, void* stream) {
+  if (!mask) return ATTN_ERR_INVALID_ARG;
+  if (n_split < 1 || n_split > kMaxSplit) return ATTN_ERR_INVALID_ARG;
+  if (n_split > 1) {
+    const int st = check_shape(B, Hq, Hkv, Lq, Lk, d, scale, mask->causal, mask->window);
+    if (st != ATTN_OK) return st;
+    const size_t need = attn_fwd_split_workspace_size(B, Hq, Hkv, Lq, Lk, d, n_split);
+    if (need > 0 && (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need))
+      return ATTN_ERR_INVALID_ARG;
+  }
+  return fwd_impl(q, k, v, o, lse, mask->seqlens_q, mask->seqlens_k, B, Hq, Hkv, Lq, Lk, d, scale, mask->causal,
+                  mask->window, mask->global_head, mask->global_tail, n_split, workspace, stream);
+}
+
+int attn_bwd_ex(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO, void* dq,
+                void* dk, void* dv, int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale, const attn_mask* mask,
+                void* workspace, size_t workspace_bytes, void* stream) {
+  if (!mask) return ATTN_ERR_INVALID_ARG;
+  return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, mask->seqlens_q, mask->seqlens_k, B, Hq, Hkv, Lq, Lk, d, scale,
+                  mask->causal, mask->window, mask->global_head, mask->global_tail, workspace, workspace_bytes, stream);
+}
 
 int attn_get_device_error(void* stream, int* site) {
   int* addr = nullptr;

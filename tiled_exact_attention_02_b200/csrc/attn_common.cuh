@@ -29,6 +29,12 @@ struct Problem {
   // every tensor is laid out with.
   const int* len_q = nullptr;
   const int* len_k = nullptr;
+  // Global key positions ("大模型高效注意力机制全解析" §5.1.2 global_tokens
+  // [0, -1]): the first global_head and the last global_tail keys of a
+  // sequence are visible to every query besides the window, still subject
+  // to the causal mask.
+  int global_head = 0;
+  int global_tail = 0;
 };
 
 // The problem of sequence b: Lq and Lk replaced by its own lengths (for the
@@ -46,6 +52,90 @@ __host__ __device__ inline int cdiv(int a, int b) { return (a + b - 1) / b; }
 
 // Key index of query row 0's causal diagonal.
 __host__ __device__ inline int diag_off(const Problem& p) { return p.causal == 2 ? p.Lk - p.Lq : 0; }
+
+__host__ __device__ inline bool has_global(const Problem& p) { return p.global_head > 0 || p.global_tail > 0; }
+// First key of the global tail (Lk when there is none).
+__host__ __device__ inline int tail_start(const Problem& p) { return imax(0, p.Lk - p.global_tail); }
+
+// Key j visible to query i through the global positions (not through the band).
+__host__ __device__ inline bool global_visible(const Problem& p, int i, int j) {
+  if (i >= p.Lq || j >= p.Lk) return false;
+  if (!(j < p.global_head || j >= tail_start(p))) return false;
+  return !p.causal || j <= i + diag_off(p);
+}
+
+// The key tiles a query tile walks, as three ranges in walk order: the global
+// head tiles, the window band, the global tail tiles (an empty range has
+// lo == hi).  norm() merges overlapping or touching ranges, so the walk is
+// sorted and visits no tile twice.  Every index below is a constant, so the
+// ranges stay in registers.
+struct Segs {
+  int lo[3] = {0, 0, 0}, hi[3] = {0, 0, 0};
+  __host__ __device__ bool empty(int k) const { return lo[k] >= hi[k]; }
+  __host__ __device__ int count() const {
+    return (hi[0] - lo[0]) * !empty(0) + (hi[1] - lo[1]) * !empty(1) + (hi[2] - lo[2]) * !empty(2);
+  }
+  __host__ __device__ bool any() const { return !empty(0) || !empty(1) || !empty(2); }
+  // Tile at position t of the walk (t < count()).
+  __host__ __device__ int at(int t) const {
+    int r = -1;
+#pragma unroll
+    for (int k = 0; k < 3; k++) {
+      if (!empty(k) && r < 0) {
+        const int len = hi[k] - lo[k];
+        if (t < len) r = lo[k] + t;
+        else t -= len;
+      }
+    }
+    return r;
+  }
+  __host__ __device__ bool contains(int j) const {
+    bool c = false;
+#pragma unroll
+    for (int k = 0; k < 3; k++)
+      if (j >= lo[k] && j < hi[k]) c = true;
+    return c;
+  }
+  // Merge range b into range a if they overlap or touch (both non-empty).
+  __host__ __device__ void merge(int a, int b) {
+    if (empty(a) || empty(b) || hi[a] < lo[b] || hi[b] < lo[a]) return;
+    lo[a] = lo[a] < lo[b] ? lo[a] : lo[b];
+    hi[a] = hi[a] > hi[b] ? hi[a] : hi[b];
+    lo[b] = hi[b] = 0;
+  }
+  __host__ __device__ void norm() {
+#pragma unroll
+    for (int k = 0; k < 3; k++)
+      if (empty(k)) lo[k] = hi[k] = 0;
+    merge(1, 0);  // head into band
+    merge(1, 2);  // tail into band
+    merge(0, 2);  // tail into head (when the band is empty)
+    merge(1, 0);  // a grown head into the band
+  }
+  // Range-wise union with another walk of the same shape.
+  __host__ __device__ void unite(const Segs& o) {
+#pragma unroll
+    for (int k = 0; k < 3; k++) {
+      if (o.empty(k)) continue;
+      if (empty(k)) {
+        lo[k] = o.lo[k], hi[k] = o.hi[k];
+      } else {
+        lo[k] = lo[k] < o.lo[k] ? lo[k] : o.lo[k];
+        hi[k] = hi[k] > o.hi[k] ? hi[k] : o.hi[k];
+      }
+    }
+    norm();
+  }
+  // Keep only tiles in [a, b).
+  __host__ __device__ void clip(int a, int b) {
+#pragma unroll
+    for (int k = 0; k < 3; k++) {
+      lo[k] = lo[k] > a ? lo[k] : a;
+      hi[k] = hi[k] < b ? hi[k] : b;
+      if (lo[k] >= hi[k]) lo[k] = hi[k] = 0;
+    }
+  }
+};
 
 // Keys [key_lo, key_hi) visible to query row i (empty when key_lo >= key_hi).
 __host__ __device__ inline void row_key_range(const Problem& p, int i, int& key_lo, int& key_hi) {
@@ -73,6 +163,25 @@ __host__ __device__ inline void kv_tile_range(const Problem& p, int q0, int q1, 
   hi = cdiv(key_hi, bn);
 }
 
+// Key tiles (of bn keys) holding any key visible to any query row in
+// [q0, q1): the band of kv_tile_range plus the tiles of the global head and
+// tail keys those rows may see.
+__host__ __device__ inline Segs kv_tile_segs(const Problem& p, int q0, int q1, int bn) {
+  Segs s;
+  kv_tile_range(p, q0, q1, bn, s.lo[1], s.hi[1]);
+  q1 = imin(q1, p.Lq);
+  if (has_global(p) && q0 < q1) {
+    // Under a causal mask the last row sees the most keys.
+    const int lim = p.causal ? imin(p.Lk, q1 + diag_off(p)) : p.Lk;
+    const int h = imin(p.global_head, lim);
+    if (h > 0) s.lo[0] = 0, s.hi[0] = cdiv(h, bn);
+    const int t0 = tail_start(p);
+    if (p.global_tail > 0 && t0 < lim) s.lo[2] = t0 / bn, s.hi[2] = cdiv(lim, bn);
+  }
+  s.norm();
+  return s;
+}
+
 // Query rows [q_lo, q_hi) that see any key in [k0, k1) (backward pass).
 __host__ __device__ inline void q_row_range(const Problem& p, int k0, int k1, int& q_lo, int& q_hi) {
   k1 = imin(k1, p.Lk);
@@ -83,6 +192,20 @@ __host__ __device__ inline void q_row_range(const Problem& p, int k0, int k1, in
   int lo = p.causal ? imax(0, k0 - off) : (p.window > 0 ? imax(0, k0 - p.window + 1) : 0);
   // j > i + off - w  =>  i < j - off + w
   int hi = p.window > 0 ? imin(p.Lq, (k1 - 1) - off + p.window) : p.Lq;
+  // A global key in the tile is seen by every row (every row at or past it
+  // under a causal mask); the band's rows lie inside that range.
+  if (has_global(p)) {
+    int jg = -1;
+    if (k0 < p.global_head) jg = k0;
+    else if (k1 > tail_start(p)) jg = imax(k0, tail_start(p));
+    if (jg >= 0) {
+      const int glo = p.causal ? imax(0, jg - off) : 0;
+      if (glo < p.Lq) {
+        lo = lo < hi ? imin(lo, glo) : glo;
+        hi = p.Lq;
+      }
+    }
+  }
   if (lo >= hi) return;
   q_lo = lo;
   q_hi = hi;

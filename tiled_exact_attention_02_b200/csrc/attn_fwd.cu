@@ -114,8 +114,8 @@ struct Unit {
   int b, kvh;
   int head[2];
   int q0[2];
-  int lo[2], hi[2];  // key tile range per slot (empty: lo == hi)
-  int ulo, uhi;      // union of the two ranges
+  Segs seg[2];       // key tiles of each slot, in walk order (band, plus global head/tail tiles)
+  Segs useg;         // their union: the tiles the CTA streams
   int split;         // key-range slice of a split problem (0 otherwise)
 };
 
@@ -152,23 +152,18 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& P, int idx) {
   }
   u.kvh = u.head[0] / G;
   const Problem ps = seq_problem(p, u.b);  // this sequence's lengths (padded batches)
-  u.ulo = 1 << 30;
-  u.uhi = 0;
-  for (int s = 0; s < 2; s++) {
-    kv_tile_range(ps, u.q0[s], u.q0[s] + BM, BN, u.lo[s], u.hi[s]);
-    if (u.lo[s] < u.hi[s]) {
-      u.ulo = imin(u.ulo, u.lo[s]);
-      u.uhi = imax(u.uhi, u.hi[s]);
-    }
-  }
-  if (u.uhi == 0) u.ulo = 0;
+  u.seg[0] = kv_tile_segs(ps, u.q0[0], u.q0[0] + BM, BN);
+  u.seg[1] = kv_tile_segs(ps, u.q0[1], u.q0[1] + BM, BN);
+  u.useg = u.seg[0];
+  u.useg.unite(u.seg[1]);
   return u;
 }
 
-// Unit of CTA `idx` when every unit's key range is cut into n_split slices
-// (consecutive CTAs take the slices of one unit): slice k keeps key tiles
-// [ulo + k*len/n, ulo + (k+1)*len/n) of the union range, intersected with
-// each slot's own range.  An empty slice leaves both slots empty.
+// Unit of CTA `idx` when every unit's key walk is cut into n_split slices
+// (consecutive CTAs take the slices of one unit): slice k keeps positions
+// [k*n/ns, (k+1)*n/ns) of the union walk (n tiles), i.e. the tiles between
+// the first and last of them, in each slot's walk as well.  An empty slice
+// leaves both slots empty.
 __device__ __forceinline__ Unit decode_unit_split(const FwdParams& P, int idx) {
   if (P.n_split <= 1) {
     Unit u = decode_unit(P, idx);
@@ -177,26 +172,18 @@ __device__ __forceinline__ Unit decode_unit_split(const FwdParams& P, int idx) {
   }
   Unit u = decode_unit(P, idx / P.n_split);
   u.split = idx % P.n_split;
-  const int len = u.uhi - u.ulo;
-  const int s_lo = u.ulo + (int)((long long)u.split * len / P.n_split);
-  const int s_hi = u.ulo + (int)((long long)(u.split + 1) * len / P.n_split);
-  int nlo = 1 << 30, nhi = 0;
-  for (int s = 0; s < 2; s++) {
-    u.lo[s] = imax(u.lo[s], s_lo);
-    u.hi[s] = imin(u.hi[s], s_hi);
-    if (u.lo[s] >= u.hi[s]) {
-      u.lo[s] = u.hi[s] = 0;
-    } else {
-      nlo = imin(nlo, u.lo[s]);
-      nhi = imax(nhi, u.hi[s]);
-    }
-  }
-  u.ulo = nhi > 0 ? nlo : 0;
-  u.uhi = nhi;
+  const int n = u.useg.count();
+  const int p0 = (int)((long long)u.split * n / P.n_split);
+  const int p1 = (int)((long long)(u.split + 1) * n / P.n_split);
+  const int a = p0 < p1 ? u.useg.at(p0) : 0;
+  const int b = p0 < p1 ? u.useg.at(p1 - 1) + 1 : 0;
+  u.useg.clip(a, b);
+  u.seg[0].clip(a, b);
+  u.seg[1].clip(a, b);
   return u;
 }
 
-__device__ __forceinline__ bool active(const Unit& u, int s, int j) { return j >= u.lo[s] && j < u.hi[s]; }
+__device__ __forceinline__ bool active(const Unit& u, int s, int j) { return u.seg[s].contains(j); }
 
 // ------------------------------------------------------------------ producer
 template <int D>
@@ -208,16 +195,18 @@ __device__ void producer(const FwdParams& P, const Unit& u, uint8_t* smem, Bars&
   tma_prefetch_desc(&P.tm_v);
 #pragma unroll
   for (int s = 0; s < 2; s++) {
-    if (u.lo[s] >= u.hi[s]) continue;
+    if (!u.seg[s].any()) continue;
     mbar_arrive_expect_tx(&bars.q_full[s], C::TILE);
     for (int pnl = 0; pnl < C::PANELS; pnl++)
       tma_load_3d(smem + C::OFF_Q + s * C::TILE + pnl * PANEL, &P.tm_q, &bars.q_full[s], pnl * 64, u.q0[s],
                   u.b * p.Hq + u.head[s]);
   }
   int issued = 0;
-  for (int j = u.ulo; j < u.uhi; j++) {
+  const int un = u.useg.count();
+  for (int t = 0; t < un; t++) {
+    const int j = u.useg.at(t);
     for (int which = 0; which < 2; which++) {
-      const int r = 2 * (j - u.ulo) + which;
+      const int r = 2 * t + which;
       const int st = r % C::NST;
       const uint32_t ph = (r / C::NST) & 1;
       if (!mbar_wait(&bars.kv_empty[st], ph ^ 1, g, 1)) goto drain;
@@ -237,7 +226,7 @@ drain:
     for (int r = imax(0, issued - C::NST); r < issued; r++) mbar_wait_ignore_abort(&bars.kv_full[r % C::NST], (r / C::NST) & 1, g2);
 #pragma unroll
     for (int s = 0; s < 2; s++)
-      if (u.lo[s] < u.hi[s]) mbar_wait_ignore_abort(&bars.q_full[s], 0, g2);
+      if (u.seg[s].any()) mbar_wait_ignore_abort(&bars.q_full[s], 0, g2);
   }
 }
 
@@ -254,14 +243,16 @@ __device__ void mma_issuer(const FwdParams& P, const Unit& u, uint8_t* smem, Bar
   const uint64_t kv_kmaj = sw128_desc(smem_u32(smem + C::OFF_KV), 16, 1024);
   const uint64_t kv_mn = sw128_desc(smem_u32(smem + C::OFF_KV), PANEL, 1024);
   auto adv = [](uint64_t d, uint32_t bytes) { return d + (uint64_t)(bytes >> 4); };
-  if (u.uhi <= u.ulo) return;
+  const int un = u.useg.count();
+  if (un == 0) return;
 
-  auto stage_of = [&](int j, int which) { return (2 * (j - u.ulo) + which) % C::NST; };
-  auto phase_of = [&](int j, int which) { return (uint32_t)(((2 * (j - u.ulo) + which) / C::NST) & 1); };
+  // K of walk position t sits in ring slot 2t, V in 2t + 1.
+  auto stage_of = [&](int t, int which) { return (2 * t + which) % C::NST; };
+  auto phase_of = [&](int t, int which) { return (uint32_t)(((2 * t + which) / C::NST) & 1); };
 
-  auto issue_s = [&](int s, int j) {
+  auto issue_s = [&](int s, int t) {
     const uint64_t qd = adv(q_kmaj, s * C::TILE);
-    const uint64_t kd = adv(kv_kmaj, stage_of(j, 0) * C::TILE);
+    const uint64_t kd = adv(kv_kmaj, stage_of(t, 0) * C::TILE);
 #pragma unroll
     for (int kk = 0; kk < D / 16; kk++) {
       const uint32_t off = (kk / 4) * PANEL + (kk % 4) * 32;
@@ -269,40 +260,51 @@ __device__ void mma_issuer(const FwdParams& P, const Unit& u, uint8_t* smem, Bar
     }
     mma_commit(&bars.s_full[s]);
   };
+  // Tiles of each slot's walk done so far, and the walk lengths.
+  int done0 = 0, done1 = 0;
+  const int n0 = u.seg[0].count(), n1 = u.seg[1].count();
 
   for (int s = 0; s < 2; s++)
-    if (u.lo[s] < u.hi[s] && !mbar_wait(&bars.q_full[s], 0, g, 10)) goto out;
+    if (u.seg[s].any() && !mbar_wait(&bars.q_full[s], 0, g, 10)) goto out;
 
-  // Prologue: S for the first tile.
-  if (!mbar_wait(&bars.kv_full[stage_of(u.ulo, 0)], phase_of(u.ulo, 0), g, 11)) goto out;
-  tc_fence_after();
+  {
+    // Prologue: S for the first tile of the walk.
+    const int j0 = u.useg.at(0);
+    if (!mbar_wait(&bars.kv_full[stage_of(0, 0)], phase_of(0, 0), g, 11)) goto out;
+    tc_fence_after();
 #pragma unroll
-  for (int s = 0; s < 2; s++)
-    if (active(u, s, u.ulo)) issue_s(s, u.ulo);
-  mma_commit(&bars.kv_empty[stage_of(u.ulo, 0)]);
+    for (int s = 0; s < 2; s++)
+      if (active(u, s, j0)) issue_s(s, 0);
+    mma_commit(&bars.kv_empty[stage_of(0, 0)]);
+  }
 
-  for (int j = u.ulo; j < u.uhi; j++) {
-    if (!mbar_wait(&bars.kv_full[stage_of(j, 1)], phase_of(j, 1), g, 12)) goto out;
-    const bool next = j + 1 < u.uhi;
+  for (int t = 0; t < un; t++) {
+    const int j = u.useg.at(t);
+    if (!mbar_wait(&bars.kv_full[stage_of(t, 1)], phase_of(t, 1), g, 12)) goto out;
+    const bool next = t + 1 < un;
+    const int jn = next ? u.useg.at(t + 1) : -1;
     if (next) {
-      if (!mbar_wait(&bars.kv_full[stage_of(j + 1, 0)], phase_of(j + 1, 0), g, 13)) goto out;
+      if (!mbar_wait(&bars.kv_full[stage_of(t + 1, 0)], phase_of(t + 1, 0), g, 13)) goto out;
     }
-    const uint64_t vd = adv(kv_mn, stage_of(j, 1) * C::TILE);
+    const uint64_t vd = adv(kv_mn, stage_of(t, 1) * C::TILE);
 #pragma unroll
     for (int s = 0; s < 2; s++) {
       if (active(u, s, j)) {
-        if (!mbar_wait(&bars.p_full[s], (j - u.lo[s]) & 1, g, 14 + s)) goto out;
+        const int done = s ? done1 : done0;
+        const int ns = s ? n1 : n0;
+        if (!mbar_wait(&bars.p_full[s], done & 1, g, 14 + s)) goto out;
         tc_fence_after();
-        const uint32_t acc0 = j > u.lo[s];
+        const uint32_t acc0 = done > 0;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; kk++)
           mma_ts(tmem + o_col(s), tmem + s_col(s) + kk * 8, adv(vd, kk * 2048), idesc_pv, kk > 0 ? 1u : acc0);
-        if (j == u.hi[s] - 1) mma_commit(&bars.o_full[s]);
+        if (done == ns - 1) mma_commit(&bars.o_full[s]);
+        if (s) done1++; else done0++;
       }
-      if (next && active(u, s, j + 1)) issue_s(s, j + 1);
+      if (next && active(u, s, jn)) issue_s(s, t + 1);
     }
-    mma_commit(&bars.kv_empty[stage_of(j, 1)]);
-    if (next) mma_commit(&bars.kv_empty[stage_of(j + 1, 0)]);
+    mma_commit(&bars.kv_empty[stage_of(t, 1)]);
+    if (next) mma_commit(&bars.kv_empty[stage_of(t + 1, 0)]);
   }
 out:
   // Drain: wait until every MMA this thread issued has completed.
@@ -321,12 +323,24 @@ __device__ void softmax_slot(const FwdParams& P, const Unit& u, int s, Bars& bar
   const int lane = threadIdx.x % 32;
   const int row = wl * 32 + lane;
   // Slot fields as scalars (a runtime index into Unit would put it in local memory).
-  const int lo_s = s ? u.lo[1] : u.lo[0];
-  const int hi_s = s ? u.hi[1] : u.hi[0];
+  const Segs walk = s ? u.seg[1] : u.seg[0];  // this slot's key tiles, in order
+  const int n_walk = walk.count();
   const int head_s = s ? u.head[1] : u.head[0];
   const int q_row = (s ? u.q0[1] : u.q0[0]) + row;
-  int key_lo, key_hi;
-  row_key_range(seq_problem(p, u.b), q_row, key_lo, key_hi);
+  int key_lo, key_hi;  // the row's band
+  int gh_hi = 0, gt_lo = 0, gt_hi = 0;  // global keys it also sees: [0, gh_hi) and [gt_lo, gt_hi)
+  {
+    const Problem ps = seq_problem(p, u.b);  // this sequence's lengths and masks
+    row_key_range(ps, q_row, key_lo, key_hi);
+    if (has_global(ps) && q_row < ps.Lq) {
+      const int lim = ps.causal ? imin(ps.Lk, q_row + diag_off(ps) + 1) : ps.Lk;
+      gh_hi = imin(ps.global_head, lim);
+      gt_lo = tail_start(ps);
+      gt_hi = ps.global_tail > 0 ? lim : 0;
+      if (gt_hi <= gt_lo) gt_lo = gt_hi = 0;  // empty: the unsigned range test below needs lo <= hi
+    }
+    if (key_hi < key_lo) key_hi = key_lo;
+  }
   const float c = P.scale_log2;
   const uint32_t lane_base = (uint32_t)(wl * 32) << 16;
   const uint32_t t_s = tmem + lane_base + s_col(s);
@@ -334,8 +348,8 @@ __device__ void softmax_slot(const FwdParams& P, const Unit& u, int s, Bars& bar
   float m = -INFINITY;  // reference max, log2 units (scaled)
   float l = 0.f;        // running sum of exp2(c*S - m)
 
-  for (int j = lo_s; j < hi_s; j++) {
-    const int it = j - lo_s;
+  for (int it = 0; it < n_walk; it++) {
+    const int j = walk.at(it);
     if (!mbar_wait(&bars.s_full[s], it & 1, g, 20 + s)) return;
     tc_fence_after();
     uint32_t x[BN];
@@ -347,10 +361,21 @@ __device__ void softmax_slot(const FwdParams& P, const Unit& u, int s, Bars& bar
     const int key0 = j * BN;
     const bool masked = key0 < key_lo || key0 + BN > key_hi;
     if (masked) {
+      if (gh_hi > 0 || gt_hi > gt_lo) {
+        // Global keys on top of the band (rare: only global-token masks).
 #pragma unroll
-      for (int cc = 0; cc < BN; cc++) {
-        const int key = key0 + cc;
-        if (key < key_lo || key >= key_hi) x[cc] = __float_as_uint(-INFINITY);
+        for (int cc = 0; cc < BN; cc++) {
+          const int key = key0 + cc;
+          const bool vis = (unsigned)(key - key_lo) < (unsigned)(key_hi - key_lo) || key < gh_hi ||
+                           (unsigned)(key - gt_lo) < (unsigned)(gt_hi - gt_lo);
+          if (!vis) x[cc] = __float_as_uint(-INFINITY);
+        }
+      } else {
+#pragma unroll
+        for (int cc = 0; cc < BN; cc++) {
+          const int key = key0 + cc;
+          if (key < key_lo || key >= key_hi) x[cc] = __float_as_uint(-INFINITY);
+        }
       }
     }
     float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
@@ -427,7 +452,7 @@ __device__ void softmax_slot(const FwdParams& P, const Unit& u, int s, Bars& bar
   }
 
   // Epilogue: O / l in bf16 and the natural-log LSE.
-  const bool has = lo_s < hi_s;
+  const bool has = n_walk > 0;
   if (has) {
     if (!mbar_wait(&bars.o_full[s], 0, g, 22 + s)) return;
     tc_fence_after();
