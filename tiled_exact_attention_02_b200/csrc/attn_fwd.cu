@@ -119,6 +119,25 @@ struct Unit {
   int split;         // key-range slice of a split problem (0 otherwise)
 };
 
+// Walk accessors.  W = false (no global tokens): the walk is the band alone,
+// which kv_tile_segs always keeps in range 1, so every accessor is the plain
+// contiguous-range arithmetic and the rest of Segs is dead code.
+template <bool W>
+__device__ __forceinline__ int walk_count(const Segs& s) {
+  if constexpr (W) return s.count();
+  else return s.hi[1] > s.lo[1] ? s.hi[1] - s.lo[1] : 0;
+}
+template <bool W>
+__device__ __forceinline__ int walk_at(const Segs& s, int t) {
+  if constexpr (W) return s.at(t);
+  else return s.lo[1] + t;
+}
+template <bool W>
+__device__ __forceinline__ bool walk_has(const Segs& s, int j) {
+  if constexpr (W) return s.contains(j);
+  else return j >= s.lo[1] && j < s.hi[1];
+}
+
 __device__ __forceinline__ Unit decode_unit(const FwdParams& P, int idx) {
   const Problem& p = P.prob;
   Unit u;
@@ -164,6 +183,7 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& P, int idx) {
 // [k*n/ns, (k+1)*n/ns) of the union walk (n tiles), i.e. the tiles between
 // the first and last of them, in each slot's walk as well.  An empty slice
 // leaves both slots empty.
+template <bool W>
 __device__ __forceinline__ Unit decode_unit_split(const FwdParams& P, int idx) {
   if (P.n_split <= 1) {
     Unit u = decode_unit(P, idx);
@@ -172,21 +192,22 @@ __device__ __forceinline__ Unit decode_unit_split(const FwdParams& P, int idx) {
   }
   Unit u = decode_unit(P, idx / P.n_split);
   u.split = idx % P.n_split;
-  const int n = u.useg.count();
+  const int n = walk_count<W>(u.useg);
   const int p0 = (int)((long long)u.split * n / P.n_split);
   const int p1 = (int)((long long)(u.split + 1) * n / P.n_split);
-  const int a = p0 < p1 ? u.useg.at(p0) : 0;
-  const int b = p0 < p1 ? u.useg.at(p1 - 1) + 1 : 0;
+  const int a = p0 < p1 ? walk_at<W>(u.useg, p0) : 0;
+  const int b = p0 < p1 ? walk_at<W>(u.useg, p1 - 1) + 1 : 0;
   u.useg.clip(a, b);
   u.seg[0].clip(a, b);
   u.seg[1].clip(a, b);
   return u;
 }
 
-__device__ __forceinline__ bool active(const Unit& u, int s, int j) { return u.seg[s].contains(j); }
+template <bool W>
+__device__ __forceinline__ bool active(const Unit& u, int s, int j) { return walk_has<W>(u.seg[s], j); }
 
 // ------------------------------------------------------------------ producer
-template <int D>
+template <int D, bool W>
 __device__ void producer(const FwdParams& P, const Unit& u, uint8_t* smem, Bars& bars, const WaitGuard& g) {
   using C = Cfg<D>;
   const Problem& p = P.prob;
@@ -195,16 +216,16 @@ __device__ void producer(const FwdParams& P, const Unit& u, uint8_t* smem, Bars&
   tma_prefetch_desc(&P.tm_v);
 #pragma unroll
   for (int s = 0; s < 2; s++) {
-    if (!u.seg[s].any()) continue;
+    if (walk_count<W>(u.seg[s]) == 0) continue;
     mbar_arrive_expect_tx(&bars.q_full[s], C::TILE);
     for (int pnl = 0; pnl < C::PANELS; pnl++)
       tma_load_3d(smem + C::OFF_Q + s * C::TILE + pnl * PANEL, &P.tm_q, &bars.q_full[s], pnl * 64, u.q0[s],
                   u.b * p.Hq + u.head[s]);
   }
   int issued = 0;
-  const int un = u.useg.count();
+  const int un = walk_count<W>(u.useg);
   for (int t = 0; t < un; t++) {
-    const int j = u.useg.at(t);
+    const int j = walk_at<W>(u.useg, t);
     for (int which = 0; which < 2; which++) {
       const int r = 2 * t + which;
       const int st = r % C::NST;
@@ -226,12 +247,12 @@ drain:
     for (int r = imax(0, issued - C::NST); r < issued; r++) mbar_wait_ignore_abort(&bars.kv_full[r % C::NST], (r / C::NST) & 1, g2);
 #pragma unroll
     for (int s = 0; s < 2; s++)
-      if (u.seg[s].any()) mbar_wait_ignore_abort(&bars.q_full[s], 0, g2);
+      if (walk_count<W>(u.seg[s]) > 0) mbar_wait_ignore_abort(&bars.q_full[s], 0, g2);
   }
 }
 
 // ------------------------------------------------------------------ MMA issuer
-template <int D>
+template <int D, bool W>
 __device__ void mma_issuer(const FwdParams& P, const Unit& u, uint8_t* smem, Bars& bars, uint32_t tmem,
                            const WaitGuard& g) {
   using C = Cfg<D>;
@@ -243,7 +264,7 @@ __device__ void mma_issuer(const FwdParams& P, const Unit& u, uint8_t* smem, Bar
   const uint64_t kv_kmaj = sw128_desc(smem_u32(smem + C::OFF_KV), 16, 1024);
   const uint64_t kv_mn = sw128_desc(smem_u32(smem + C::OFF_KV), PANEL, 1024);
   auto adv = [](uint64_t d, uint32_t bytes) { return d + (uint64_t)(bytes >> 4); };
-  const int un = u.useg.count();
+  const int un = walk_count<W>(u.useg);
   if (un == 0) return;
 
   // K of walk position t sits in ring slot 2t, V in 2t + 1.
@@ -262,34 +283,34 @@ __device__ void mma_issuer(const FwdParams& P, const Unit& u, uint8_t* smem, Bar
   };
   // Tiles of each slot's walk done so far, and the walk lengths.
   int done0 = 0, done1 = 0;
-  const int n0 = u.seg[0].count(), n1 = u.seg[1].count();
+  const int n0 = walk_count<W>(u.seg[0]), n1 = walk_count<W>(u.seg[1]);
 
   for (int s = 0; s < 2; s++)
-    if (u.seg[s].any() && !mbar_wait(&bars.q_full[s], 0, g, 10)) goto out;
+    if (walk_count<W>(u.seg[s]) > 0 && !mbar_wait(&bars.q_full[s], 0, g, 10)) goto out;
 
   {
     // Prologue: S for the first tile of the walk.
-    const int j0 = u.useg.at(0);
+    const int j0 = walk_at<W>(u.useg, 0);
     if (!mbar_wait(&bars.kv_full[stage_of(0, 0)], phase_of(0, 0), g, 11)) goto out;
     tc_fence_after();
 #pragma unroll
     for (int s = 0; s < 2; s++)
-      if (active(u, s, j0)) issue_s(s, 0);
+      if (active<W>(u, s, j0)) issue_s(s, 0);
     mma_commit(&bars.kv_empty[stage_of(0, 0)]);
   }
 
   for (int t = 0; t < un; t++) {
-    const int j = u.useg.at(t);
+    const int j = walk_at<W>(u.useg, t);
     if (!mbar_wait(&bars.kv_full[stage_of(t, 1)], phase_of(t, 1), g, 12)) goto out;
     const bool next = t + 1 < un;
-    const int jn = next ? u.useg.at(t + 1) : -1;
+    const int jn = next ? walk_at<W>(u.useg, t + 1) : -1;
     if (next) {
       if (!mbar_wait(&bars.kv_full[stage_of(t + 1, 0)], phase_of(t + 1, 0), g, 13)) goto out;
     }
     const uint64_t vd = adv(kv_mn, stage_of(t, 1) * C::TILE);
 #pragma unroll
     for (int s = 0; s < 2; s++) {
-      if (active(u, s, j)) {
+      if (active<W>(u, s, j)) {
         const int done = s ? done1 : done0;
         const int ns = s ? n1 : n0;
         if (!mbar_wait(&bars.p_full[s], done & 1, g, 14 + s)) goto out;
@@ -301,7 +322,7 @@ __device__ void mma_issuer(const FwdParams& P, const Unit& u, uint8_t* smem, Bar
         if (done == ns - 1) mma_commit(&bars.o_full[s]);
         if (s) done1++; else done0++;
       }
-      if (next && active(u, s, jn)) issue_s(s, t + 1);
+      if (next && active<W>(u, s, jn)) issue_s(s, t + 1);
     }
     mma_commit(&bars.kv_empty[stage_of(t, 1)]);
     if (next) mma_commit(&bars.kv_empty[stage_of(t + 1, 0)]);
@@ -315,7 +336,7 @@ out:
 // ------------------------------------------------------------------ softmax
 // One warpgroup per slot; thread `row` owns query row q0 + row and TMEM lane
 // `row` (warp w of the group may only touch lanes 32*(w%4) .. +31).
-template <int D>
+template <int D, bool W>
 __device__ void softmax_slot(const FwdParams& P, const Unit& u, int s, Bars& bars, uint32_t tmem,
                              const WaitGuard& g) {
   const Problem& p = P.prob;
@@ -324,7 +345,7 @@ __device__ void softmax_slot(const FwdParams& P, const Unit& u, int s, Bars& bar
   const int row = wl * 32 + lane;
   // Slot fields as scalars (a runtime index into Unit would put it in local memory).
   const Segs walk = s ? u.seg[1] : u.seg[0];  // this slot's key tiles, in order
-  const int n_walk = walk.count();
+  const int n_walk = walk_count<W>(walk);
   const int head_s = s ? u.head[1] : u.head[0];
   const int q_row = (s ? u.q0[1] : u.q0[0]) + row;
   int key_lo, key_hi;  // the row's band
@@ -332,7 +353,7 @@ __device__ void softmax_slot(const FwdParams& P, const Unit& u, int s, Bars& bar
   {
     const Problem ps = seq_problem(p, u.b);  // this sequence's lengths and masks
     row_key_range(ps, q_row, key_lo, key_hi);
-    if (has_global(ps) && q_row < ps.Lq) {
+    if (W && has_global(ps) && q_row < ps.Lq) {
       const int lim = ps.causal ? imin(ps.Lk, q_row + diag_off(ps) + 1) : ps.Lk;
       gh_hi = imin(ps.global_head, lim);
       gt_lo = tail_start(ps);
@@ -349,7 +370,7 @@ __device__ void softmax_slot(const FwdParams& P, const Unit& u, int s, Bars& bar
   float l = 0.f;        // running sum of exp2(c*S - m)
 
   for (int it = 0; it < n_walk; it++) {
-    const int j = walk.at(it);
+    const int j = walk_at<W>(walk, it);
     if (!mbar_wait(&bars.s_full[s], it & 1, g, 20 + s)) return;
     tc_fence_after();
     uint32_t x[BN];
@@ -361,7 +382,7 @@ __device__ void softmax_slot(const FwdParams& P, const Unit& u, int s, Bars& bar
     const int key0 = j * BN;
     const bool masked = key0 < key_lo || key0 + BN > key_hi;
     if (masked) {
-      if (gh_hi > 0 || gt_hi > gt_lo) {
+      if (W && (gh_hi > 0 || gt_hi > gt_lo)) {
         // Global keys on top of the band (rare: only global-token masks).
 #pragma unroll
         for (int cc = 0; cc < BN; cc++) {
@@ -510,7 +531,8 @@ __device__ void softmax_slot(const FwdParams& P, const Unit& u, int s, Bars& bar
 }
 
 // ------------------------------------------------------------------ kernel
-template <int D>
+// W: the problem has global tokens (the key-tile walk may have several ranges).
+template <int D, bool W>
 __global__ void __launch_bounds__(THREADS, 1) attn_fwd_kernel(const __grid_constant__ FwdParams P) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -518,7 +540,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_kernel(const __grid_const
   Bars& bars = *reinterpret_cast<Bars*>(smem + C::OFF_BAR);
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  const Unit u = decode_unit_split(P, blockIdx.x);
+  const Unit u = decode_unit_split<W>(P, blockIdx.x);
   const WaitGuard g{P.err, &bars.abort_flag, P.limit_ns, 0};
 
   if (threadIdx.x == 0) {
@@ -550,13 +572,13 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_kernel(const __grid_const
   if (warp < 4) {
     regs_dec<112>();
     if (warp == 0) {
-      if (lane == 0) producer<D>(P, u, smem, bars, g);
+      if (lane == 0) producer<D, W>(P, u, smem, bars, g);
     } else if (warp == 1) {
-      if (lane == 0) mma_issuer<D>(P, u, smem, bars, tmem, g);
+      if (lane == 0) mma_issuer<D, W>(P, u, smem, bars, tmem, g);
     }
   } else {
     regs_inc<192>();
-    softmax_slot<D>(P, u, (warp - 4) / 4, bars, tmem, g);
+    softmax_slot<D, W>(P, u, (warp - 4) / 4, bars, tmem, g);
   }
   tc_fence_before();
   __syncthreads();
@@ -640,18 +662,20 @@ void fwd_plan(const Problem& p, int* n_units, int* pair_heads) {
   }
 }
 
-template <int D>
+template <int D, bool W>
 static cudaError_t launch_fwd_d(const FwdParams& P, cudaStream_t stream) {
   constexpr int smem = fwd::Cfg<D>::SMEM;
-  cudaError_t e = cudaFuncSetAttribute(fwd::attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = cudaFuncSetAttribute(fwd::attn_fwd_kernel<D, W>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  fwd::attn_fwd_kernel<D><<<P.n_units * imax(1, P.n_split), fwd::THREADS, smem, stream>>>(P);
+  fwd::attn_fwd_kernel<D, W><<<P.n_units * imax(1, P.n_split), fwd::THREADS, smem, stream>>>(P);
   return cudaGetLastError();
 }
 
 cudaError_t launch_fwd(const FwdParams& P, cudaStream_t stream) {
   if (P.n_units <= 0) return cudaSuccess;
-  return P.prob.d == 128 ? launch_fwd_d<128>(P, stream) : launch_fwd_d<64>(P, stream);
+  if (has_global(P.prob))
+    return P.prob.d == 128 ? launch_fwd_d<128, true>(P, stream) : launch_fwd_d<64, true>(P, stream);
+  return P.prob.d == 128 ? launch_fwd_d<128, false>(P, stream) : launch_fwd_d<64, false>(P, stream);
 }
 
 }  // namespace tea
