@@ -41,7 +41,7 @@ KERNEL_SRC = os.path.join(ROOT, "tiled_exact_attention_02_b200", "csrc", "attn_b
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=800)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=10)
@@ -76,39 +76,74 @@ def profile_traffic():
 
 
 class ClockSampler:
-    """nvidia-smi clock/throttle sampling during the timed region."""
+    """nvidia-smi clock/throttle sampling during the timed region.
+
+    nvidia-smi needs a moment to start, so the sampler is started first and
+    waits for its first sample; `mark()` brackets the timed region on the host
+    clock and `stop()` keeps the samples whose timestamps fall inside it (the
+    first one after it when the region is shorter than the sampling period)."""
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, index):
         self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
-        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        self.t0 = self.t1 = None
         try:
-            self.p = subprocess.Popen(["nvidia-smi", f"--id={index}", f"--query-gpu={q}", "--format=csv,noheader,nounits",
-                                       "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+            self.p = subprocess.Popen(["nvidia-smi", f"--id={index}", f"--query-gpu={self.FIELDS}",
+                                       "--format=csv,noheader,nounits", "-lms", "100"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
         except OSError:
             self.p = None
+            return
+        deadline = time.time() + 5.0
+        while time.time() < deadline and not open(self.f.name).read().strip():
+            time.sleep(0.05)
+
+    def mark(self, start):
+        if start:
+            self.t0 = time.time()
+        else:
+            self.t1 = time.time()
+
+    @staticmethod
+    def _when(stamp):
+        from datetime import datetime
+        try:
+            return datetime.strptime(stamp.strip(), "%Y/%m/%d %H:%M:%S.%f").timestamp()
+        except ValueError:
+            return None
 
     def stop(self):
         if self.p is None:
             return None
+        time.sleep(0.15)  # let a sample land after the region when it was shorter than the period
         self.p.terminate()
         self.p.wait()
         self.f.flush()
-        rows = [r.split(",") for r in open(self.f.name).read().strip().splitlines() if r.strip()]
+        rows = [[c.strip() for c in r.split(",")] for r in open(self.f.name).read().strip().splitlines() if r.strip()]
         os.unlink(self.f.name)
+        rows = [r for r in rows if len(r) >= 10]
         if not rows:
             return None
-        sm = [float(r[1]) for r in rows if len(r) > 8]
+        timed = [r for r in rows if self.t0 is not None and self.t1 is not None
+                 and (self._when(r[0]) or 0.0) >= self.t0 and (self._when(r[0]) or 0.0) <= self.t1]
+        window = "timed region"
+        if not timed:
+            after = [r for r in rows if self.t0 is not None and (self._when(r[0]) or 0.0) >= self.t0]
+            timed = after[:1] or rows[-1:]
+            window = "first sample after the region started (region shorter than the 100 ms period)"
+        sm = [float(r[2]) for r in timed]
         reasons = set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for r in rows:
-            for n, v in zip(names, r[5:9]):
-                if v.strip() == "Active":
+        for r in timed:
+            for n, v in zip(names, r[6:10]):
+                if v == "Active":
                     reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": float(rows[0][2]) if len(rows[0]) > 2 else None,
-                "samples": len(sm), "reasons": sorted(reasons)}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(timed[0][3]),
+                "power_w": statistics.median(float(r[4]) for r in timed),
+                "samples": len(timed), "window": window, "reasons": sorted(reasons)}
 
 
 def dist_setup(n_gpus, backend="nccl"):
@@ -328,11 +363,13 @@ def main():
     clocks = ClockSampler(local)
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
+    clocks.mark(True)
     t_start.record(stream)
     for i in range(args.steps):
         step(events[i])
     t_end.record(stream)
     torch.cuda.synchronize()
+    clocks.mark(False)
     barrier(world)
     clk = clocks.stop()
     st, site = ta.device_error()

@@ -70,6 +70,33 @@ def test_fwd_edge_shapes(ta, B, Hq, Hkv, Lq, Lk, d, causal, window):
     check_lse(lse, rl, "LSE")
 
 
+# Short queries with a GQA group (G > 1, Lq < 128): the G heads of a kv group
+# share the tile rows (row r = query r % Lq of head r / Lq), one tile or two,
+# tiles inside one head and across heads, the group's last tile ragged.
+# (B, Hq, Hkv, Lq, Lk, d, causal, window)
+PACKED = [
+    (2, 8, 2, 16, 1000, 128, 2, 0),
+    (1, 12, 2, 40, 700, 64, 2, 0),
+    (1, 16, 2, 100, 900, 128, 1, 0),
+    (3, 32, 8, 1, 5000, 128, 2, 0),
+    (1, 4, 2, 64, 64, 128, 0, 16),
+    (1, 6, 3, 127, 127, 128, 1, 0),
+    (1, 24, 8, 5, 300, 64, 2, 32),
+    (2, 8, 1, 33, 33, 128, 0, 0),
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Lq,Lk,d,causal,window", PACKED)
+def test_fwd_packed_rows(ta, B, Hq, Hkv, Lq, Lk, d, causal, window):
+    """Heads of a kv group stacked in the tile rows, against the oracle."""
+    x = make_shape_inputs(B, Hq, Hkv, Lq, Lk, d, seed=Lq * 13 + Lk + d + Hq)
+    scale = d ** -0.5
+    o, lse = run_fwd(ta, x, causal, window, scale)
+    ro, rl = oracle.attn_fwd(x["q"], x["k"], x["v"], scale, causal, window)
+    check_o(o, ro, "O")
+    check_lse(lse, rl, "LSE")
+
+
 # (B, Hq, Hkv, Lq, Lk, d, causal, window, n_split); n_split None: the library's choice
 SPLIT = [
     (2, 8, 2, 1, 3000, 128, 2, 0, 8),
@@ -79,6 +106,8 @@ SPLIT = [
     (1, 2, 2, 200, 100, 128, 2, 0, 7),
     (1, 2, 2, 100, 900, 128, 0, 64, 4),
     (1, 2, 2, 50, 700, 128, 0, 0, 64),
+    (2, 16, 4, 8, 4000, 128, 2, 0, None),
+    (1, 12, 2, 40, 3000, 64, 2, 256, 6),
 ]
 
 
@@ -103,6 +132,7 @@ VARLEN = [
     (2, 4, 4, 200, 200, 64, 0, 0, [200, 77], [150, 200]),
     (2, 2, 1, 500, 500, 128, 1, 64, [500, 333], [500, 333]),
     (2, 2, 2, 300, 300, 128, 0, 50, [300, 128], [10, 300]),
+    (3, 8, 2, 16, 600, 128, 2, 0, [16, 5, 0], [600, 17, 300]),
 ]
 
 
@@ -130,6 +160,7 @@ GLOBAL = [
     (2, 2, 1, 300, 500, 64, 2, 50, 130, 20),
     (1, 2, 2, 257, 257, 128, 0, 8, 0, 3),
     (1, 2, 2, 400, 400, 128, 0, 0, 5, 5),
+    (1, 8, 2, 32, 900, 128, 2, 64, 4, 2),
 ]
 
 

@@ -167,13 +167,16 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, float*
   // With Lk == 0 nothing reads K/V; map Q's memory so the descriptors stay valid.
   const void* kp = Lk > 0 ? k : q;
   const void* vp = Lk > 0 ? v : q;
-  if ((st = make_map(enc, &P.tm_q, q, B * Hq, Lq, d)) != ATTN_OK) return st;
+  fwd_plan(P.prob, &P.n_units, &P.pair_heads, &P.packed);
+  // Packed rows read Q as [B*Hkv, G*Lq, d]: the G heads of a kv group are adjacent in memory.
+  if ((st = P.packed ? make_map(enc, &P.tm_q, q, B * Hkv, (Hq / Hkv) * Lq, d) : make_map(enc, &P.tm_q, q, B * Hq, Lq, d)) !=
+      ATTN_OK)
+    return st;
   if ((st = make_map(enc, &P.tm_k, kp, Lk > 0 ? B * Hkv : B * Hq, Lk > 0 ? Lk : Lq, d)) != ATTN_OK) return st;
   if ((st = make_map(enc, &P.tm_v, vp, Lk > 0 ? B * Hkv : B * Hq, Lk > 0 ? Lk : Lq, d)) != ATTN_OK) return st;
   P.o = o;
   P.lse = lse;
   P.scale_log2 = scale * 1.4426950408889634f;
-  fwd_plan(P.prob, &P.n_units, &P.pair_heads);
   P.n_split = n_split;
   if (n_split > 1) {
     const size_t rows = (size_t)B * Hq * Lq;
@@ -221,18 +224,24 @@ int attn_fwd_split_default(int B, int Hq, int Hkv, int Lq, int Lk, int d, int ca
   if (check_shape(B, Hq, Hkv, Lq, Lk, d, 1.f, causal, window) != ATTN_OK) return 1;
   if (B == 0 || Hq == 0 || Lq == 0 || Lk == 0) return 1;
   Problem p{B, Hq, Hkv, Lq, Lk, d, causal, window, 1.f};
-  int n_units, pair;
-  fwd_plan(p, &n_units, &pair);
+  int n_units, pair, packed;
+  fwd_plan(p, &n_units, &pair, &packed);
   int sms = 148;
   int dev;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // Enough slices that the grid covers every SM about twice, but no slice
-  // shorter than two key tiles.
+  // Pick the slice count with the least estimated time: waves of one CTA per
+  // SM, each as long as a slice's key tiles plus about two tiles of fixed
+  // cost (Q load, pipeline fill, epilogue); no slice shorter than two tiles.
   const int tiles = (Lk + 127) / 128;
-  int n = (2 * sms + n_units - 1) / n_units;
-  n = n < tiles / 2 ? n : tiles / 2;
-  n = n < kMaxSplit ? n : kMaxSplit;
-  return n < 1 ? 1 : n;
+  const int n_max = imin(kMaxSplit, imax(1, tiles / 2));
+  int best = 1;
+  double best_t = 0;
+  for (int n = 1; n <= n_max; n++) {
+    const double waves = (double)((n_units * (int64_t)n + sms - 1) / sms);
+    const double t = waves * ((double)tiles / n + 2.0);
+    if (n == 1 || t < best_t) best = n, best_t = t;
+  }
+  return best;
 }
 
 int attn_fwd_split(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Lq,

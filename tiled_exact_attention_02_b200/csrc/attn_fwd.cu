@@ -138,7 +138,42 @@ __device__ __forceinline__ bool walk_has(const Segs& s, int j) {
   else return j >= s.lo[1] && j < s.hi[1];
 }
 
+// Packed rows (short queries): row r of kv group (b, kvh) is query r % Lq of
+// head kvh*G + r / Lq, i.e. Q read as [B*Hkv, G*Lq, d]; each unit takes two
+// consecutive 128-row tiles of a group.  A tile inside one head sees the key
+// tiles of its own query rows, a tile across heads those of all Lq rows.
+__device__ __forceinline__ Unit decode_unit_packed(const FwdParams& P, int idx) {
+  const Problem& p = P.prob;
+  Unit u;
+  const int G = p.Hq / p.Hkv;
+  const int R = G * p.Lq;
+  const int nq = cdiv(cdiv(R, BM), 2);
+  const int grp = idx / nq;
+  u.b = grp / p.Hkv;
+  u.kvh = grp % p.Hkv;
+  const int qi = idx % nq;
+  const Problem ps = seq_problem(p, u.b);
+#pragma unroll
+  for (int s = 0; s < 2; s++) {
+    const int r0 = (2 * qi + s) * BM;
+    const int r1 = imin(r0 + BM, R);
+    u.head[s] = u.kvh * G;
+    u.q0[s] = r0;
+    if (r0 >= r1) {
+      u.seg[s] = Segs{};
+    } else if (r0 / p.Lq != (r1 - 1) / p.Lq) {
+      u.seg[s] = kv_tile_segs(ps, 0, p.Lq, BN);
+    } else {
+      u.seg[s] = kv_tile_segs(ps, r0 % p.Lq, (r1 - 1) % p.Lq + 1, BN);
+    }
+  }
+  u.useg = u.seg[0];
+  u.useg.unite(u.seg[1]);
+  return u;
+}
+
 __device__ __forceinline__ Unit decode_unit(const FwdParams& P, int idx) {
+  if (P.packed) return decode_unit_packed(P, idx);
   const Problem& p = P.prob;
   Unit u;
   const int G = p.Hq / p.Hkv;
@@ -220,7 +255,7 @@ __device__ void producer(const FwdParams& P, const Unit& u, uint8_t* smem, Bars&
     mbar_arrive_expect_tx(&bars.q_full[s], C::TILE);
     for (int pnl = 0; pnl < C::PANELS; pnl++)
       tma_load_3d(smem + C::OFF_Q + s * C::TILE + pnl * PANEL, &P.tm_q, &bars.q_full[s], pnl * 64, u.q0[s],
-                  u.b * p.Hq + u.head[s]);
+                  P.packed ? u.b * p.Hkv + u.kvh : u.b * p.Hq + u.head[s]);
   }
   int issued = 0;
   const int un = walk_count<W>(u.useg);
@@ -346,8 +381,16 @@ __device__ void softmax_slot(const FwdParams& P, const Unit& u, int s, Bars& bar
   // Slot fields as scalars (a runtime index into Unit would put it in local memory).
   const Segs walk = s ? u.seg[1] : u.seg[0];  // this slot's key tiles, in order
   const int n_walk = walk_count<W>(walk);
-  const int head_s = s ? u.head[1] : u.head[0];
-  const int q_row = (s ? u.q0[1] : u.q0[0]) + row;
+  int head_s = s ? u.head[1] : u.head[0];
+  int q_row = (s ? u.q0[1] : u.q0[0]) + row;
+  if (P.packed) {
+    // Packed rows: this row's head and query; rows past the group's last
+    // (the tile's zero-filled tail) get q_row = Lq, which sees nothing and is not written.
+    const int pr = q_row;
+    const int G = p.Hq / p.Hkv;
+    head_s += pr / p.Lq;
+    q_row = pr < G * p.Lq ? pr % p.Lq : p.Lq;
+  }
   int key_lo, key_hi;  // the row's band
   int gh_hi = 0, gt_lo = 0, gt_hi = 0;  // global keys it also sees: [0, gh_hi) and [gt_lo, gt_hi)
   {
@@ -650,10 +693,17 @@ cudaError_t launch_fwd_merge(const FwdParams& P, cudaStream_t stream) {
 }
 
 
-void fwd_plan(const Problem& p, int* n_units, int* pair_heads) {
+void fwd_plan(const Problem& p, int* n_units, int* pair_heads, int* packed) {
   const int G = p.Hq / p.Hkv;
   const int nqt = cdiv(p.Lq, fwd::BM);
-  if (G % 2 == 0) {
+  *packed = 0;
+  if (G > 1 && p.Lq < fwd::BM) {
+    // Fewer query rows than a tile: stack the G heads of a kv group in the
+    // tile rows, so the group's K/V stream once per 256 rows (two slots).
+    *packed = 1;
+    *pair_heads = 0;
+    *n_units = p.B * p.Hkv * cdiv(cdiv(G * p.Lq, fwd::BM), 2);
+  } else if (G % 2 == 0) {
     *pair_heads = 1;
     *n_units = p.B * (p.Hq / 2) * nqt;
   } else {

@@ -8,7 +8,7 @@
 namespace tea {
 
 struct FwdParams {
-  CUtensorMap tm_q;  // [B*Hq, Lq, d] bf16, box 64 x 128 x 1, 128-byte swizzle
+  CUtensorMap tm_q;  // [B*Hq, Lq, d] bf16, box 64 x 128 x 1, 128-byte swizzle ([B*Hkv, G*Lq, d] if packed)
   CUtensorMap tm_k;  // [B*Hkv, Lk, d]
   CUtensorMap tm_v;  // [B*Hkv, Lk, d]
   Problem prob;
@@ -16,6 +16,7 @@ struct FwdParams {
   float* lse;        // fp32 [B, Hq, Lq]
   float scale_log2;  // scale * log2(e)
   int pair_heads;    // 1: a CTA takes two heads of one GQA group at the same rows
+  int packed;        // 1: short queries; a tile's 128 rows run over the G heads of one kv group
   int n_units;       // work units (two query tiles each); the grid is n_units * n_split CTAs
   int n_split;       // key-range slices per unit (1: the CTA writes O and LSE itself)
   float* part_o;     // n_split > 1: fp32 [n_split][B*Hq][Lq][d], O of each slice normalised by its own sum
@@ -68,7 +69,7 @@ cudaError_t launch_bwd_post(const float* dq_acc, void* dq, int BH, int Lq, int l
                             cudaStream_t stream);
 
 // Number of CTAs of the forward grid and whether heads are paired.
-void fwd_plan(const Problem& p, int* n_units, int* pair_heads);
+void fwd_plan(const Problem& p, int* n_units, int* pair_heads, int* packed);
 cudaError_t launch_fwd(const FwdParams& P, cudaStream_t stream);
 // Combine n_split partial (O, LSE) of every row into bf16 O and fp32 LSE.
 cudaError_t launch_fwd_merge(const FwdParams& P, cudaStream_t stream);
