@@ -48,6 +48,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--all-configs", action="store_true",
                     help="time attn_fwd and the backward on every workload (one JSON line each); not the bench line")
+    ap.add_argument("--workload", default=None, help="with --all-configs: only this workload")
     return ap.parse_args()
 
 
@@ -267,6 +268,8 @@ def all_configs(args):
     import tiled_exact_attention_02_b200 as ta
     burst, sustained, hbm, peak_src = peaks()
     for name, w in WORKLOADS.items():
+        if args.workload is not None and name != args.workload:
+            continue
         x = make_inputs(w)
         dev = lambda bits: torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).cuda()
         q, k, v = (dev(x[n]) for n in ("q", "k", "v"))
@@ -387,23 +390,23 @@ def main():
     achieved = w.bwd_flops() / (main_ms * 1e-3) / 1e12
     fwd_tf = w.fwd_flops() / (per["attn_fwd"] * 1e-3) / 1e12
 
-    # End to end through the public API with host buffers: pinned host inputs
-    # copied in, the step run, and every output (O, LSE, dQ, dK, dV) copied out.
+    # End to end through the C ABI's host-buffer call: attn_step_host copies
+    # the pinned host inputs in, runs the step and copies every output (O,
+    # LSE, dQ, dK, dV) back, overlapping the copies with the kernels chunk by
+    # chunk.
     e2e = None
     if args.e2e_steps > 0:
-        hin = [t.cpu().pin_memory() for t in (q, k, v, do)]
-        outs = (o, lse, dq, dk, dv)
-        hout = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
-        h2d = sum(t.numel() * t.element_size() for t in hin)
-        d2h = sum(t.numel() * t.element_size() for t in hout)
-        dins = (q, k, v, do)
+        hq, hk, hv, hdo = (t.cpu().pin_memory() for t in (q, k, v, do))
+        pin = lambda t: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+        ho, hlse, hdq, hdk, hdv = (pin(t) for t in (o, lse, dq, dk, dv))
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
+        d2h = sum(t.numel() * t.element_size() for t in (ho, hlse, hdq, hdk, hdv))
+        hbuf = torch.empty(ta.step_host_buffer_size(w.B, w.Hq, w.Hkv, w.Lq, w.Lk, w.d, True), dtype=torch.uint8,
+                           device=dev)
 
         def e2e_step():
-            for dst, src in zip(dins, hin):
-                dst.copy_(src, non_blocking=True)
-            step()
-            for dst, src in zip(hout, outs):
-                dst.copy_(src, non_blocking=True)
+            ta.step_host(hq, hk, hv, ho, hlse, hbuf, do=hdo, dq=hdq, dk=hdk, dv=hdv, causal=w.causal,
+                         window=w.window, scale=w.scale, stream=stream)
 
         for _ in range(2):
             e2e_step()

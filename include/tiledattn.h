@@ -255,6 +255,39 @@ ATTN_API int attn_bwd_noalloc(const void* q, const void* k, const void* v, const
                               const void* dO, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Lq, int Lk,
                               int d, float scale, int causal, int window, void* stream);
 
+/*
+ * The attention step with HOST buffers: copies Q, K, V (and dO) in, runs
+ * attn_fwd (and attn_bwd), and copies O and LSE (and dQ, dK, dV) out, all
+ * ordered on `stream` like every other call (asynchronous; synchronise the
+ * stream before reading the host outputs).  The pages' interface works on
+ * tensors already on the device; this is the same computation for a caller
+ * whose data lives in host memory.
+ *
+ *  - q, k, v, dO, o, lse, dq, dk, dv: HOST pointers, same shapes and layouts
+ *    as attn_fwd / attn_bwd.  Page-locked (pinned) host memory lets the copies
+ *    run concurrently with the kernels; pageable memory gives the same
+ *    results with the copies serialised.
+ *  - dO == NULL: forward only (dq, dk, dv are ignored and may be NULL).
+ *  - dev_buf: caller-owned device memory, 256-byte aligned, at least
+ *    attn_step_host_buffer_size(...) bytes (with_backward = dO != NULL); it
+ *    stages every tensor and the backward workspace.  The library allocates
+ *    no device memory; it creates and releases three streams and a few events
+ *    per call.
+ *  - The problem is cut into chunks of whole kv-head groups of one sequence
+ *    (about eight chunks): chunk c's inputs are copied in on one internal
+ *    stream while chunk c-1 computes on a second and chunk c-2's outputs are
+ *    copied out on a third.  Results are bit-identical to attn_fwd / attn_bwd
+ *    on the whole problem.
+ *  - Errors: shape, mask and scale checks as attn_fwd (before anything is
+ *    enqueued); NULL host pointers or a short / misaligned dev_buf:
+ *    ATTN_ERR_INVALID_ARG; a failing CUDA call: ATTN_ERR_CUDA (work already
+ *    enqueued still runs; outputs are then undefined).
+ */
+ATTN_API size_t attn_step_host_buffer_size(int B, int Hq, int Hkv, int Lq, int Lk, int d, int with_backward);
+ATTN_API int attn_step_host(const void* q, const void* k, const void* v, const void* dO, void* o, float* lse,
+                            void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale,
+                            int causal, int window, void* dev_buf, size_t dev_buf_bytes, void* stream);
+
 /* Static, human-readable name of a status code. */
 ATTN_API const char* attn_status_string(int status);
 

@@ -158,3 +158,37 @@ def test_fwd_ex_and_bwd_ex_validate_the_mask(ta):
     m.global_tail = -2
     assert ta.lib.attn_bwd_ex(*([P] * 9), 1, 2, 2, 8, 8, 64, 0.125, ctypes.byref(m), P, 1 << 20, None) == 1
     assert ta.lib.attn_bwd_ex(*([P] * 9), 1, 2, 2, 8, 8, 64, 0.125, None, P, 1 << 20, None) == 1
+
+
+def _host_size(ta, B=2, Hq=8, Hkv=2, Lq=300, Lk=500, d=128, bwd=1):
+    return ta.lib.attn_step_host_buffer_size(B, Hq, Hkv, Lq, Lk, d, bwd)
+
+
+def test_step_host_buffer_size(ta):
+    a = lambda x: (x + 255) // 256 * 256
+    B, Hq, Hkv, Lq, Lk, d = 2, 8, 2, 300, 500, 128
+    nq, nk = B * Hq * Lq * d * 2, B * Hkv * Lk * d * 2
+    # One kv head per chunk here (B * Hkv = 4 groups): LSE staged in 4 chunk slots of G * Lq floats each.
+    fwd_only = a(nq) + 2 * a(nk) + a(nq) + a(4 * a(Hq // Hkv * Lq * 4))
+    assert _host_size(ta, bwd=0) == fwd_only
+    # Backward adds dO, dQ, dK, dV and one chunk's workspace.
+    ws = ta.lib.attn_bwd_workspace_size(1, Hq // Hkv, 1, Lq, Lk, d)
+    assert _host_size(ta, bwd=1) == fwd_only + 2 * a(nq) + 2 * a(nk) + a(ws)
+    assert _host_size(ta, d=96) == 0
+    assert _host_size(ta, Hq=3) == 0
+    assert _host_size(ta, B=0) == 0
+
+
+def _host(ta, buf=P << 4, nbytes=1 << 40, do=P, q=P, B=1, Hq=2, Hkv=2, Lq=8, Lk=8, d=64, scale=0.125, causal=0,
+          window=0):
+    return ta.lib.attn_step_host(q, P, P, do, P, P, P, P, P, B, Hq, Hkv, Lq, Lk, d, scale, causal, window, buf,
+                                 nbytes, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(d=96), 2), (dict(Hq=3), 1), (dict(causal=3), 1), (dict(scale=0.0), 1), (dict(window=-1), 1),
+    (dict(q=0), 1), (dict(buf=0), 1), (dict(buf=(P << 4) + 16), 1), (dict(nbytes=100), 1),
+    (dict(B=0), 0), (dict(Lq=0), 0),
+])
+def test_step_host_rejects_before_any_copy(ta, kw, status):
+    assert _host(ta, **kw) == status

@@ -260,6 +260,29 @@ def test_fwd_full_size_sampled_heads(ta, name, heads):
     assert np.all(np.isfinite(o))
 
 
+@pytest.mark.parametrize("split", [False, True])
+def test_fwd_decode_full_size(ta, split):
+    """gqa_decode_32768 at full size (packed rows; with split=True the split-KV
+    launch with the library's default slice count, as timed): sampled heads
+    against the oracle."""
+    w = WORKLOADS["gqa_decode_32768"]
+    x = make_inputs(w)
+    q, k, v = (to_dev(x[n]) for n in "qkv")
+    if split:
+        o, lse = ta.attention_split(q, k, v, w.causal, w.window, w.scale, None)
+    else:
+        o, lse = ta.attention(q, k, v, w.causal, w.window, w.scale)
+    st, site = ta.device_error()
+    assert st == 0, f"device error {st} at site {site}"
+    o, lse = to_f64(o), to_f64(lse)
+    heads = [(0, 0), (3, 31), (1, 13), (2, 6)]
+    ro, rl = oracle.attn_fwd(x["q"], x["k"], x["v"], w.scale, w.causal, w.window, heads=heads)
+    for b, h in heads:
+        check_o(o[b, h], ro[b, h], f"decode O[{b},{h}]")
+        check_lse(lse[b, h], rl[b, h], f"decode LSE[{b},{h}]")
+    assert np.all(np.isfinite(o))
+
+
 def test_bounded_wait_reports_timeout(ta):
     """A wait that nothing completes gives up and reports ATTN_ERR_TIMEOUT;
     the context stays usable afterwards."""

@@ -73,6 +73,10 @@ def _load() -> ctypes.CDLL:
     lib.attn_bwd_main.restype = i
     lib.attn_bwd_finalize.argtypes = [vp, i, i, i, i, f, vp, sz, vp]
     lib.attn_bwd_finalize.restype = i
+    lib.attn_step_host_buffer_size.argtypes = [i, i, i, i, i, i, i]
+    lib.attn_step_host_buffer_size.restype = sz
+    lib.attn_step_host.argtypes = [vp] * 9 + [i] * 6 + [f, i, i, vp, sz, vp]
+    lib.attn_step_host.restype = i
     lib.attn_last_cuda_error.argtypes = []
     lib.attn_last_cuda_error.restype = ctypes.c_char_p
     lib.attn_status_string.argtypes = [i]
@@ -226,6 +230,33 @@ def bwd_phases(q, k, v, o, lse, do, dq, dk, dv, workspace, causal: bool = False,
     hook(2)
     _check(lib.attn_bwd_finalize(dq.data_ptr(), B, Hq, Lq, d, scale, ws, wsb, sp), "attn_bwd_finalize")
     hook(3)
+
+
+def step_host_buffer_size(B, Hq, Hkv, Lq, Lk, d, with_backward: bool = True) -> int:
+    return int(lib.attn_step_host_buffer_size(B, Hq, Hkv, Lq, Lk, d, int(bool(with_backward))))
+
+
+def step_host(q, k, v, o, lse, buf, do=None, dq=None, dk=None, dv=None, causal: bool = False, window: int = 0,
+              scale: float | None = None, stream=None) -> None:
+    """attn_step_host: q, k, v (do) and the outputs o, lse (dq, dk, dv) are
+    contiguous CPU tensors (pinned for overlapped copies); `buf` is a CUDA
+    uint8 tensor of at least step_host_buffer_size bytes.  Asynchronous on
+    `stream`: synchronise it before reading the outputs."""
+    import torch
+    B, Hq, Hkv, Lq, Lk, d = _shapes(q, k)
+    host = [("q", q), ("k", k), ("v", v), ("o", o)] + ([("do", do), ("dq", dq), ("dk", dk), ("dv", dv)]
+                                                     if do is not None else [])
+    for name, t in host:
+        if t is None or t.is_cuda or not t.is_contiguous() or t.dtype != torch.bfloat16:
+            raise ValueError(f"{name} must be a contiguous bf16 CPU tensor")
+    if lse.is_cuda or not lse.is_contiguous() or lse.dtype != torch.float32:
+        raise ValueError("lse must be a contiguous float32 CPU tensor")
+    _require(buf, "buf", torch.uint8)
+    sc = d ** -0.5 if scale is None else scale
+    ptr = lambda t: None if t is None else t.data_ptr()
+    _check(lib.attn_step_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), ptr(do), o.data_ptr(), lse.data_ptr(),
+                              ptr(dq), ptr(dk), ptr(dv), B, Hq, Hkv, Lq, Lk, d, sc, _causal_code(causal),
+                              int(window), buf.data_ptr(), buf.numel(), _stream_ptr(stream)), "attn_step_host")
 
 
 def device_error(stream=None) -> tuple[int, int]:

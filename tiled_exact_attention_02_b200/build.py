@@ -11,7 +11,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libtiledattn.so")
-SOURCES = ["api.cu", "attn_fwd.cu", "attn_bwd.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "attn_fwd.cu", "attn_bwd.cu", "noalloc.cu", "host_step.cu"]
 HEADERS = ["sm100.cuh", "attn_common.cuh", "attn_kernels.h", "../../include/tiledattn.h"]
 
 

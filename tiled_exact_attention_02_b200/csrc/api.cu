@@ -124,6 +124,13 @@ __global__ void selftest_wait_kernel(int* err, uint64_t limit_ns) {
 }
 
 }  // namespace
+
+int validate_problem(int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale, int causal, int window) {
+  return check_shape(B, Hq, Hkv, Lq, Lk, d, scale, causal, window);
+}
+
+int record_cuda_error(const char* step, cudaError_t e) { return cuda_fail(step, e); }
+
 }  // namespace tea
 
 using namespace tea;
@@ -167,7 +174,7 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, float*
   // With Lk == 0 nothing reads K/V; map Q's memory so the descriptors stay valid.
   const void* kp = Lk > 0 ? k : q;
   const void* vp = Lk > 0 ? v : q;
-  fwd_plan(P.prob, &P.n_units, &P.pair_heads, &P.packed);
+  fwd_plan(P.prob, &P.n_units, &P.pair_heads, &P.packed, &P.alternate);
   // Packed rows read Q as [B*Hkv, G*Lq, d]: the G heads of a kv group are adjacent in memory.
   if ((st = P.packed ? make_map(enc, &P.tm_q, q, B * Hkv, (Hq / Hkv) * Lq, d) : make_map(enc, &P.tm_q, q, B * Hq, Lq, d)) !=
       ATTN_OK)
@@ -224,8 +231,8 @@ int attn_fwd_split_default(int B, int Hq, int Hkv, int Lq, int Lk, int d, int ca
   if (check_shape(B, Hq, Hkv, Lq, Lk, d, 1.f, causal, window) != ATTN_OK) return 1;
   if (B == 0 || Hq == 0 || Lq == 0 || Lk == 0) return 1;
   Problem p{B, Hq, Hkv, Lq, Lk, d, causal, window, 1.f};
-  int n_units, pair, packed;
-  fwd_plan(p, &n_units, &pair, &packed);
+  int n_units, pair, packed, alternate;
+  fwd_plan(p, &n_units, &pair, &packed, &alternate);
   int sms = 148;
   int dev;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

@@ -98,6 +98,7 @@ struct Bars {
   uint64_t s_full[2];
   uint64_t p_full[2];
   uint64_t o_full[2];
+  uint64_t merge;       // alternating slots: slot 1's row max and sum are in shared memory [4 warps]
   uint64_t drain;
   uint64_t kv_full[8];
   uint64_t kv_empty[8];
@@ -117,6 +118,7 @@ struct Unit {
   Segs seg[2];       // key tiles of each slot, in walk order (band, plus global head/tail tiles)
   Segs useg;         // their union: the tiles the CTA streams
   int split;         // key-range slice of a split problem (0 otherwise)
+  int alt;           // 1: both slots hold the same rows and take alternate key tiles of one range
 };
 
 // Walk accessors.  W = false (no global tokens): the walk is the band alone,
@@ -172,8 +174,25 @@ __device__ __forceinline__ Unit decode_unit_packed(const FwdParams& P, int idx) 
   return u;
 }
 
+// A unit whose second slot would hold no rows instead gives both slots the
+// first slot's rows; slot s then takes the key tiles at even (s = 0) or odd
+// (s = 1) positions of the walk, and the two partial softmaxes are merged in
+// the epilogue.  The two chains of softmax and MMAs then run side by side.
+__device__ __forceinline__ void make_alternating(Unit& u) {
+  u.alt = 1;
+  u.q0[1] = u.q0[0];
+  u.head[1] = u.head[0];
+  u.seg[1] = u.seg[0];
+  u.useg = u.seg[0];
+}
+
 __device__ __forceinline__ Unit decode_unit(const FwdParams& P, int idx) {
-  if (P.packed) return decode_unit_packed(P, idx);
+  if (P.packed) {
+    Unit u = decode_unit_packed(P, idx);
+    u.alt = 0;
+    if (P.alternate) make_alternating(u);
+    return u;
+  }
   const Problem& p = P.prob;
   Unit u;
   const int G = p.Hq / p.Hkv;
@@ -210,6 +229,8 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& P, int idx) {
   u.seg[1] = kv_tile_segs(ps, u.q0[1], u.q0[1] + BM, BN);
   u.useg = u.seg[0];
   u.useg.unite(u.seg[1]);
+  u.alt = 0;
+  if (P.alternate) make_alternating(u);
   return u;
 }
 
@@ -238,8 +259,22 @@ __device__ __forceinline__ Unit decode_unit_split(const FwdParams& P, int idx) {
   return u;
 }
 
+// Slot walks: with alternating slots (never with global tokens) slot s takes
+// positions s, s + 2, ... of the one contiguous range.
 template <bool W>
-__device__ __forceinline__ bool active(const Unit& u, int s, int j) { return walk_has<W>(u.seg[s], j); }
+__device__ __forceinline__ bool active(const Unit& u, int s, int j) {
+  if (!W && u.alt) return walk_has<W>(u.seg[s], j) && ((j - u.seg[s].lo[1]) & 1) == s;
+  return walk_has<W>(u.seg[s], j);
+}
+template <bool W>
+__device__ __forceinline__ int slot_count(const Unit& u, const Segs& sg, int s) {
+  const int n = walk_count<W>(sg);
+  return (!W && u.alt) ? (n + 1 - s) / 2 : n;
+}
+template <bool W>
+__device__ __forceinline__ int slot_at(const Unit& u, const Segs& sg, int s, int i) {
+  return (!W && u.alt) ? sg.lo[1] + 2 * i + s : walk_at<W>(sg, i);
+}
 
 // ------------------------------------------------------------------ producer
 template <int D, bool W>
@@ -251,7 +286,7 @@ __device__ void producer(const FwdParams& P, const Unit& u, uint8_t* smem, Bars&
   tma_prefetch_desc(&P.tm_v);
 #pragma unroll
   for (int s = 0; s < 2; s++) {
-    if (walk_count<W>(u.seg[s]) == 0) continue;
+    if (walk_count<W>(u.seg[s]) == 0 || (s == 1 && u.alt)) continue;  // alternating slots share slot 0's Q
     mbar_arrive_expect_tx(&bars.q_full[s], C::TILE);
     for (int pnl = 0; pnl < C::PANELS; pnl++)
       tma_load_3d(smem + C::OFF_Q + s * C::TILE + pnl * PANEL, &P.tm_q, &bars.q_full[s], pnl * 64, u.q0[s],
@@ -282,7 +317,7 @@ drain:
     for (int r = imax(0, issued - C::NST); r < issued; r++) mbar_wait_ignore_abort(&bars.kv_full[r % C::NST], (r / C::NST) & 1, g2);
 #pragma unroll
     for (int s = 0; s < 2; s++)
-      if (walk_count<W>(u.seg[s]) > 0) mbar_wait_ignore_abort(&bars.q_full[s], 0, g2);
+      if (walk_count<W>(u.seg[s]) > 0 && !(s == 1 && u.alt)) mbar_wait_ignore_abort(&bars.q_full[s], 0, g2);
   }
 }
 
@@ -368,11 +403,69 @@ out:
   mbar_wait_ignore_abort(&bars.drain, 0, g);
 }
 
+// ------------------------------------------------------------------ MMA issuer, alternating slots
+// Walk position t belongs to slot t & 1 and both slots read slot 0's Q.  The
+// S of a slot's next tile (position t + 2) is issued right after the P.V of
+// its current one, so while one slot's softmax runs the other slot's MMAs
+// have the tensor cores.
+template <int D>
+__device__ void mma_issuer_alt(const FwdParams& P, const Unit& u, uint8_t* smem, Bars& bars, uint32_t tmem,
+                               const WaitGuard& g) {
+  using C = Cfg<D>;
+  const uint32_t idesc_qk = idesc_bf16_f32(BM, BN, 0, 0);
+  const uint32_t idesc_pv = idesc_bf16_f32(BM, D, 0, 1);
+  const uint64_t q_kmaj = sw128_desc(smem_u32(smem + C::OFF_Q), 16, 1024);
+  const uint64_t kv_kmaj = sw128_desc(smem_u32(smem + C::OFF_KV), 16, 1024);
+  const uint64_t kv_mn = sw128_desc(smem_u32(smem + C::OFF_KV), PANEL, 1024);
+  auto adv = [](uint64_t d, uint32_t bytes) { return d + (uint64_t)(bytes >> 4); };
+  const int un = walk_count<false>(u.useg);
+  if (un == 0) return;
+  auto stage_of = [&](int t, int which) { return (2 * t + which) % C::NST; };
+  auto phase_of = [&](int t, int which) { return (uint32_t)(((2 * t + which) / C::NST) & 1); };
+  // S of slot s for walk position t (its K is in ring slot 2t); K released after.
+  auto issue_s = [&](int s, int t) -> bool {
+    if (!mbar_wait(&bars.kv_full[stage_of(t, 0)], phase_of(t, 0), g, 11)) return false;
+    tc_fence_after();
+    const uint64_t kd = adv(kv_kmaj, stage_of(t, 0) * C::TILE);
+#pragma unroll
+    for (int kk = 0; kk < D / 16; kk++) {
+      const uint32_t off = (kk / 4) * PANEL + (kk % 4) * 32;
+      mma_ss(tmem + s_col(s), adv(q_kmaj, off), adv(kd, off), idesc_qk, kk > 0);
+    }
+    mma_commit(&bars.s_full[s]);
+    mma_commit(&bars.kv_empty[stage_of(t, 0)]);
+    return true;
+  };
+
+  if (!mbar_wait(&bars.q_full[0], 0, g, 10)) goto out;
+  if (!issue_s(0, 0)) goto out;
+  if (un > 1 && !issue_s(1, 1)) goto out;
+  for (int t = 0; t < un; t++) {
+    const int s = t & 1;
+    if (!mbar_wait(&bars.kv_full[stage_of(t, 1)], phase_of(t, 1), g, 12)) goto out;
+    if (!mbar_wait(&bars.p_full[s], (t >> 1) & 1, g, 14 + s)) goto out;
+    tc_fence_after();
+    {
+      const uint64_t vd = adv(kv_mn, stage_of(t, 1) * C::TILE);
+      const uint32_t acc0 = t >= 2;
+#pragma unroll
+      for (int kk = 0; kk < BN / 16; kk++)
+        mma_ts(tmem + o_col(s), tmem + s_col(s) + kk * 8, adv(vd, kk * 2048), idesc_pv, kk > 0 ? 1u : acc0);
+    }
+    if (t + 2 >= un) mma_commit(&bars.o_full[s]);
+    mma_commit(&bars.kv_empty[stage_of(t, 1)]);
+    if (t + 2 < un && !issue_s(s, t + 2)) goto out;
+  }
+out:
+  mma_commit(&bars.drain);
+  mbar_wait_ignore_abort(&bars.drain, 0, g);
+}
+
 // ------------------------------------------------------------------ softmax
 // One warpgroup per slot; thread `row` owns query row q0 + row and TMEM lane
 // `row` (warp w of the group may only touch lanes 32*(w%4) .. +31).
 template <int D, bool W>
-__device__ void softmax_slot(const FwdParams& P, const Unit& u, int s, Bars& bars, uint32_t tmem,
+__device__ void softmax_slot(const FwdParams& P, const Unit& u, int s, uint8_t* smem, Bars& bars, uint32_t tmem,
                              const WaitGuard& g) {
   const Problem& p = P.prob;
   const int wl = (threadIdx.x / 32) % 4;
@@ -380,7 +473,7 @@ __device__ void softmax_slot(const FwdParams& P, const Unit& u, int s, Bars& bar
   const int row = wl * 32 + lane;
   // Slot fields as scalars (a runtime index into Unit would put it in local memory).
   const Segs walk = s ? u.seg[1] : u.seg[0];  // this slot's key tiles, in order
-  const int n_walk = walk_count<W>(walk);
+  const int n_walk = slot_count<W>(u, walk, s);
   int head_s = s ? u.head[1] : u.head[0];
   int q_row = (s ? u.q0[1] : u.q0[0]) + row;
   if (P.packed) {
@@ -413,7 +506,7 @@ __device__ void softmax_slot(const FwdParams& P, const Unit& u, int s, Bars& bar
   float l = 0.f;        // running sum of exp2(c*S - m)
 
   for (int it = 0; it < n_walk; it++) {
-    const int j = walk_at<W>(walk, it);
+    const int j = slot_at<W>(u, walk, s, it);
     if (!mbar_wait(&bars.s_full[s], it & 1, g, 20 + s)) return;
     tc_fence_after();
     uint32_t x[BN];
@@ -521,30 +614,71 @@ __device__ void softmax_slot(const FwdParams& P, const Unit& u, int s, Bars& bar
     if (!mbar_wait(&bars.o_full[s], 0, g, 22 + s)) return;
     tc_fence_after();
   }
+  // Alternating slots: slot 1 hands its row max and sum to slot 0 through
+  // shared memory (slot 1's Q tile, unused in this mode) and slot 0 merges
+  // the two partial softmaxes: with M = max(m0, m1), O = O0 2^(m0-M) +
+  // O1 2^(m1-M) and l = l0 2^(m0-M) + l1 2^(m1-M), exact up to rounding.
+  float a_own = 1.f, a_oth = 0.f;
+  bool oth = false;  // slot 1's O takes part
+  const uint32_t t_o1 = tmem + lane_base + o_col(1);
+  if (!W && u.alt) {
+    float2* ml = reinterpret_cast<float2*>(smem + Cfg<D>::OFF_Q + Cfg<D>::TILE);
+    if (s == 1) {
+      ml[row] = make_float2(m, l);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.merge);
+      return;
+    }
+    const int n1 = slot_count<W>(u, u.seg[1], 1);
+    if (!mbar_wait(&bars.merge, 0, g, 26)) return;
+    if (n1 > 0) {
+      if (!mbar_wait(&bars.o_full[1], 0, g, 27)) return;
+      tc_fence_after();
+    }
+    const float2 o1 = ml[row];
+    const float M = fmaxf(m, o1.x);
+    a_own = m == -INFINITY ? 0.f : ex2_approx(m - M);
+    a_oth = (n1 == 0 || o1.x == -INFINITY) ? 0.f : ex2_approx(o1.x - M);
+    oth = n1 > 0;
+    l = l * a_own + o1.y * a_oth;
+    m = M;
+  }
   const bool write = q_row < p.Lq;
   const float inv_l = l > 0.f ? 1.f / l : 0.f;
+  const float sc_own = a_own * inv_l, sc_oth = a_oth * inv_l;
   const size_t row_off = ((size_t)(u.b * p.Hq + head_s) * p.Lq + q_row);
   const float lse_row = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
+  // Columns 16q .. 16q+15 of the row's normalised O (both slots' parts when merging).
+  auto load_o = [&](int q, float (&f)[16]) {
+    uint32_t o[16];
+    if (has) {
+      tmem_ld16(t_o + 16 * q, o);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 16; e++) f[e] = __uint_as_float(o[e]) * sc_own;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 16; e++) f[e] = 0.f;
+    }
+    if (oth) {
+      tmem_ld16(t_o1 + 16 * q, o);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 16; e++) f[e] = fmaf(__uint_as_float(o[e]), sc_oth, f[e]);
+    }
+  };
   if (P.n_split > 1) {
     // One key-range slice of a split problem: fp32 O normalised by this
     // slice's own sum, and the slice's LSE; the merge kernel combines them.
     const size_t part_row = (size_t)u.split * ((size_t)p.B * p.Hq * p.Lq) + row_off;
     float4* outp = reinterpret_cast<float4*>(P.part_o + part_row * D);
 #pragma unroll
-    for (int q = 0; q < D / 32; q++) {
-      uint32_t o[32];
-      if (has) {
-        tmem_ld32p(t_o + 32 * q, o);
-        tmem_wait_ld();
-      } else {
-#pragma unroll
-        for (int e = 0; e < 32; e++) o[e] = 0u;
-      }
+    for (int q = 0; q < D / 16; q++) {
+      float f[16];
+      load_o(q, f);
       if (write) {
 #pragma unroll
-        for (int v = 0; v < 8; v++)
-          outp[q * 8 + v] = make_float4(__uint_as_float(o[4 * v]) * inv_l, __uint_as_float(o[4 * v + 1]) * inv_l,
-                                        __uint_as_float(o[4 * v + 2]) * inv_l, __uint_as_float(o[4 * v + 3]) * inv_l);
+        for (int v = 0; v < 4; v++) outp[q * 4 + v] = make_float4(f[4 * v], f[4 * v + 1], f[4 * v + 2], f[4 * v + 3]);
       }
     }
     if (write) P.part_lse[part_row] = lse_row;
@@ -552,22 +686,15 @@ __device__ void softmax_slot(const FwdParams& P, const Unit& u, int s, Bars& bar
   }
   uint4* out = reinterpret_cast<uint4*>(static_cast<uint16_t*>(P.o) + row_off * D);
 #pragma unroll
-  for (int q = 0; q < D / 32; q++) {
-    uint32_t o[32];
-    if (has) {
-      tmem_ld32p(t_o + 32 * q, o);
-      tmem_wait_ld();
-    } else {
+  for (int q = 0; q < D / 16; q++) {
+    float f[16];
+    load_o(q, f);
+    uint32_t w[8];
 #pragma unroll
-      for (int e = 0; e < 32; e++) o[e] = 0u;
-    }
-    uint32_t w[16];
-#pragma unroll
-    for (int e = 0; e < 16; e++)
-      w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
+    for (int e = 0; e < 8; e++) w[e] = pack_bf16x2(f[2 * e], f[2 * e + 1]);
     if (write) {
 #pragma unroll
-      for (int v = 0; v < 4; v++) out[q * 4 + v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+      for (int v = 0; v < 2; v++) out[q * 2 + v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
     }
   }
   if (write) P.lse[row_off] = lse_row;
@@ -575,7 +702,9 @@ __device__ void softmax_slot(const FwdParams& P, const Unit& u, int s, Bars& bar
 
 // ------------------------------------------------------------------ kernel
 // W: the problem has global tokens (the key-tile walk may have several ranges).
-template <int D, bool W>
+// A: alternating slots (launched only for plans that use them, so the other
+// variants carry none of that code).
+template <int D, bool W, bool A>
 __global__ void __launch_bounds__(THREADS, 1) attn_fwd_kernel(const __grid_constant__ FwdParams P) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -583,7 +712,8 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_kernel(const __grid_const
   Bars& bars = *reinterpret_cast<Bars*>(smem + C::OFF_BAR);
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  const Unit u = decode_unit_split<W>(P, blockIdx.x);
+  Unit u = decode_unit_split<W>(P, blockIdx.x);
+  if (!A || W) u.alt = 0;
   const WaitGuard g{P.err, &bars.abort_flag, P.limit_ns, 0};
 
   if (threadIdx.x == 0) {
@@ -594,6 +724,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_kernel(const __grid_const
       mbar_init(&bars.p_full[s], 4);
       mbar_init(&bars.o_full[s], 1);
     }
+    mbar_init(&bars.merge, 4);
     mbar_init(&bars.drain, 1);
     for (int st = 0; st < C::NST; st++) {
       mbar_init(&bars.kv_full[st], 1);
@@ -617,11 +748,16 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_kernel(const __grid_const
     if (warp == 0) {
       if (lane == 0) producer<D, W>(P, u, smem, bars, g);
     } else if (warp == 1) {
-      if (lane == 0) mma_issuer<D, W>(P, u, smem, bars, tmem, g);
+      if (lane == 0) {
+        if (!W && u.alt)
+          mma_issuer_alt<D>(P, u, smem, bars, tmem, g);
+        else
+          mma_issuer<D, W>(P, u, smem, bars, tmem, g);
+      }
     }
   } else {
     regs_inc<192>();
-    softmax_slot<D, W>(P, u, (warp - 4) / 4, bars, tmem, g);
+    softmax_slot<D, W>(P, u, (warp - 4) / 4, smem, bars, tmem, g);
   }
   tc_fence_before();
   __syncthreads();
@@ -693,39 +829,50 @@ cudaError_t launch_fwd_merge(const FwdParams& P, cudaStream_t stream) {
 }
 
 
-void fwd_plan(const Problem& p, int* n_units, int* pair_heads, int* packed) {
+void fwd_plan(const Problem& p, int* n_units, int* pair_heads, int* packed, int* alternate) {
   const int G = p.Hq / p.Hkv;
   const int nqt = cdiv(p.Lq, fwd::BM);
   *packed = 0;
+  *alternate = 0;
   if (G > 1 && p.Lq < fwd::BM) {
     // Fewer query rows than a tile: stack the G heads of a kv group in the
     // tile rows, so the group's K/V stream once per 256 rows (two slots).
     *packed = 1;
     *pair_heads = 0;
     *n_units = p.B * p.Hkv * cdiv(cdiv(G * p.Lq, fwd::BM), 2);
+    *alternate = cdiv(G * p.Lq, fwd::BM) == 1;
   } else if (G % 2 == 0) {
     *pair_heads = 1;
     *n_units = p.B * (p.Hq / 2) * nqt;
   } else {
     *pair_heads = 0;
     *n_units = p.B * p.Hq * cdiv(nqt, 2);
+    *alternate = nqt == 1;
   }
+  // One slot of rows per unit: the second slot takes alternate key tiles of
+  // the same rows (one contiguous key range, so not with global tokens).
+  if (has_global(p)) *alternate = 0;
 }
 
-template <int D, bool W>
+template <int D, bool W, bool A>
 static cudaError_t launch_fwd_d(const FwdParams& P, cudaStream_t stream) {
   constexpr int smem = fwd::Cfg<D>::SMEM;
-  cudaError_t e = cudaFuncSetAttribute(fwd::attn_fwd_kernel<D, W>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e =
+      cudaFuncSetAttribute(fwd::attn_fwd_kernel<D, W, A>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  fwd::attn_fwd_kernel<D, W><<<P.n_units * imax(1, P.n_split), fwd::THREADS, smem, stream>>>(P);
+  fwd::attn_fwd_kernel<D, W, A><<<P.n_units * imax(1, P.n_split), fwd::THREADS, smem, stream>>>(P);
   return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t launch_fwd_dd(const FwdParams& P, cudaStream_t stream) {
+  if (has_global(P.prob)) return launch_fwd_d<D, true, false>(P, stream);
+  return P.alternate ? launch_fwd_d<D, false, true>(P, stream) : launch_fwd_d<D, false, false>(P, stream);
 }
 
 cudaError_t launch_fwd(const FwdParams& P, cudaStream_t stream) {
   if (P.n_units <= 0) return cudaSuccess;
-  if (has_global(P.prob))
-    return P.prob.d == 128 ? launch_fwd_d<128, true>(P, stream) : launch_fwd_d<64, true>(P, stream);
-  return P.prob.d == 128 ? launch_fwd_d<128, false>(P, stream) : launch_fwd_d<64, false>(P, stream);
+  return P.prob.d == 128 ? launch_fwd_dd<128>(P, stream) : launch_fwd_dd<64>(P, stream);
 }
 
 }  // namespace tea

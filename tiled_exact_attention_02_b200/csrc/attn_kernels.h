@@ -17,6 +17,7 @@ struct FwdParams {
   float scale_log2;  // scale * log2(e)
   int pair_heads;    // 1: a CTA takes two heads of one GQA group at the same rows
   int packed;        // 1: short queries; a tile's 128 rows run over the G heads of one kv group
+  int alternate;     // 1: each unit has one slot of rows; both slots take them, on alternate key tiles
   int n_units;       // work units (two query tiles each); the grid is n_units * n_split CTAs
   int n_split;       // key-range slices per unit (1: the CTA writes O and LSE itself)
   float* part_o;     // n_split > 1: fp32 [n_split][B*Hq][Lq][d], O of each slice normalised by its own sum
@@ -69,7 +70,11 @@ cudaError_t launch_bwd_post(const float* dq_acc, void* dq, int BH, int Lq, int l
                             cudaStream_t stream);
 
 // Number of CTAs of the forward grid and whether heads are paired.
-void fwd_plan(const Problem& p, int* n_units, int* pair_heads, int* packed);
+void fwd_plan(const Problem& p, int* n_units, int* pair_heads, int* packed, int* alternate);
+// The C ABI's shape, mask and scale checks (ATTN_OK or the status to return).
+int validate_problem(int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale, int causal, int window);
+// Records `step` and the error's text for attn_last_cuda_error; returns ATTN_ERR_CUDA.
+int record_cuda_error(const char* step, cudaError_t e);
 cudaError_t launch_fwd(const FwdParams& P, cudaStream_t stream);
 // Combine n_split partial (O, LSE) of every row into bf16 O and fp32 LSE.
 cudaError_t launch_fwd_merge(const FwdParams& P, cudaStream_t stream);
