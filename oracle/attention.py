@@ -14,6 +14,10 @@ Sources (page title and section):
       causal band  i - w < j <= i  (w keys, the query itself included), and,
       without a causal mask, as the two-sided band  i - w < j < i + w  (the
       "前后" (before and after) wording of the same section).
+  * "大模型高效注意力机制全解析" §4.1.2 (block-sparse attention): the mask is
+      built block by block: for each query block start i (step b) and each
+      j from max(0, i - b) to min(L, i + b) - 1, the b x b block at (i, j) is
+      set.  `sparse_block_mask` builds it exactly that way.
   * "缩放定律与高效注意力" §3.3: the backward pass needs only O and the per-row
       logsumexp; the gradient formulas themselves are the textbook softmax
       gradient (the pages do not print them).
@@ -46,11 +50,35 @@ def diag_offset(causal, Lq: int, Lk: int) -> int:
     return Lk - Lq if causal == 2 else 0
 
 
-def _visible(i, j, causal, window: int, off: int = 0, glob=(0, 0, 0)) -> np.ndarray:
+def sparse_block_mask(rows, lo: int, hi: int, b: int, Lq: int, Lk: int) -> np.ndarray:
+    """The block-sparse mask of "大模型高效注意力机制全解析" §4.1.2 for query rows
+    `rows` and key columns [lo, hi): the page's construction on an [Lq, Lk]
+    matrix (query block starts i = 0, b, 2b, ... below Lq; for each, every j
+    in [max(0, i - b), min(Lk, i + b)) sets the block rows i..i+b-1, keys
+    j..j+b-1, clipped to the matrix), restricted to the rows asked for."""
+    rows = np.asarray(rows)
+    out = np.zeros((rows.size, hi - lo), dtype=bool)
+    if rows.size == 0:
+        return out
+    r_min, r_max = int(rows.min()), int(rows.max())
+    for i in range(0, Lq, b):
+        if i + b <= r_min or i > r_max:
+            continue  # this query block holds none of the rows
+        sel = (rows >= i) & (rows < i + b)
+        for j in range(max(0, i - b), min(Lk, i + b)):
+            c0, c1 = max(j, lo), min(j + b, Lk, hi)
+            if c0 < c1:
+                out[np.ix_(sel, np.arange(c0 - lo, c1 - lo))] = True
+    return out
+
+
+def _visible(i, j, causal, window: int, off: int = 0, glob=(0, 0, 0), blk=None) -> np.ndarray:
     """Elementwise visibility of key j to query i (broadcasting arrays);
     `off` is diag_offset(causal, Lq, Lk); glob = (global_head, global_tail, Lk):
     the first global_head and the last global_tail key positions are visible
-    to every query (still subject to the causal mask)."""
+    to every query (still subject to the causal mask); blk: an optional
+    block-sparse mask of the same shape, intersected with the causal and window
+    masks before the global keys are added."""
     vis = np.ones(np.broadcast(i, j).shape, dtype=bool)
     if causal:
         vis &= j <= i + off
@@ -58,6 +86,8 @@ def _visible(i, j, causal, window: int, off: int = 0, glob=(0, 0, 0)) -> np.ndar
         vis &= j > i + off - window
         if not causal:
             vis &= j < i + window
+    if blk is not None:
+        vis &= blk
     gh, gt, lk = glob
     if gh > 0 or gt > 0:
         g = (j < gh) | (j >= lk - gt)
@@ -67,7 +97,8 @@ def _visible(i, j, causal, window: int, off: int = 0, glob=(0, 0, 0)) -> np.ndar
     return vis
 
 
-def visible_mask(Lq: int, Lk: int, causal, window: int, global_head: int = 0, global_tail: int = 0) -> np.ndarray:
+def visible_mask(Lq: int, Lk: int, causal, window: int, global_head: int = 0, global_tail: int = 0,
+                 sparse_block: int = 0) -> np.ndarray:
     """Boolean [Lq, Lk]: True where key j is visible to query i.
 
     Causal: j <= i (causal = 2: j <= i + Lk - Lq).  Window w > 0: the w keys
@@ -75,8 +106,9 @@ def visible_mask(Lq: int, Lk: int, causal, window: int, global_head: int = 0, gl
     sliding window); without causal the band reaches w - 1 keys to either
     side, i - w < j < i + w (the two-sided "前后" reading of the same section).
     """
+    blk = sparse_block_mask(np.arange(Lq), 0, Lk, sparse_block, Lq, Lk) if sparse_block > 0 else None
     return _visible(np.arange(Lq)[:, None], np.arange(Lk)[None, :], causal, window, diag_offset(causal, Lq, Lk),
-                    (global_head, global_tail, Lk))
+                    (global_head, global_tail, Lk), blk)
 
 
 def visible_band(r0: int, r1: int, Lk: int, causal, window: int, off: int = 0, glob=(0, 0, 0)) -> tuple[int, int]:
@@ -116,7 +148,7 @@ def attention_weights(q, k, scale: float, vis: np.ndarray):
     return A, lse
 
 
-def _head_fwd(qh, kh, vh, scale, causal, window, rows=None, gl=(0, 0)):
+def _head_fwd(qh, kh, vh, scale, causal, window, rows=None, gl=(0, 0), sb=0):
     """O and LSE for the rows `rows` (default: all) of one head."""
     Lq, Lk = qh.shape[0], kh.shape[0]
     off = diag_offset(causal, Lq, Lk)
@@ -134,7 +166,7 @@ def _head_fwd(qh, kh, vh, scale, causal, window, rows=None, gl=(0, 0)):
         r0, r1 = int(blk.min()), int(blk.max()) + 1
         glob = (gl[0], gl[1], Lk)
         lo, hi = visible_band(r0, r1, Lk, causal, window, off, glob)
-        vis = _band_mask(blk, lo, hi, causal, window, off, glob)
+        vis = _band_mask(blk, lo, hi, causal, window, off, glob, sb, Lq, Lk)
         A, l = attention_weights(qh[blk], kh[lo:hi], scale, vis)
         O[start:stop] = A @ vh[lo:hi]
         lse[start:stop] = l
@@ -142,8 +174,9 @@ def _head_fwd(qh, kh, vh, scale, causal, window, rows=None, gl=(0, 0)):
     return O, lse
 
 
-def _band_mask(rows, lo, hi, causal, window, off, glob=(0, 0, 0)):
-    return _visible(np.asarray(rows)[:, None], np.arange(lo, hi)[None, :], causal, window, off, glob)
+def _band_mask(rows, lo, hi, causal, window, off, glob=(0, 0, 0), sb=0, Lq=0, Lk=0):
+    blk = sparse_block_mask(rows, lo, hi, sb, Lq, Lk) if sb > 0 else None
+    return _visible(np.asarray(rows)[:, None], np.arange(lo, hi)[None, :], causal, window, off, glob, blk)
 
 
 def _group(Hq: int, Hkv: int) -> int:
@@ -162,7 +195,7 @@ def _lengths(seqlens, b: int, full: int) -> int:
 
 
 def attn_fwd(q, k, v, scale: float, causal: bool = False, window: int = 0, heads=None, seqlens_q=None,
-             seqlens_k=None, global_head: int = 0, global_tail: int = 0):
+             seqlens_k=None, global_head: int = 0, global_tail: int = 0, sparse_block: int = 0):
     """O [B,Hq,Lq,d] and LSE [B,Hq,Lq] in float64.
 
     q: [B,Hq,Lq,d]; k, v: [B,Hkv,Lk,d] (float or bf16 bits as uint16).
@@ -173,6 +206,9 @@ def attn_fwd(q, k, v, scale: float, causal: bool = False, window: int = 0, heads
     sequence b is its own attention problem over its first seqlens_q[b]
     queries and seqlens_k[b] keys (a bottom-right causal diagonal is placed by
     those lengths); padded query rows get O = 0 and LSE = -inf.
+    sparse_block: b > 0 adds the block-sparse mask of "大模型高效注意力机制全解析"
+    §4.1.2 with b x b blocks (each sequence of a padded batch builds it over
+    its own lengths).
     """
     q, k, v = _f64(q), _f64(k), _f64(v)
     B, Hq, Lq, d = q.shape
@@ -186,7 +222,7 @@ def attn_fwd(q, k, v, scale: float, causal: bool = False, window: int = 0, heads
         O[b, h] = 0.0
         lse[b, h] = -np.inf
         O[b, h, :nq], lse[b, h, :nq] = _head_fwd(q[b, h, :nq], k[b, g, :nk], v[b, g, :nk], scale, causal, window,
-                                                 gl=(global_head, global_tail))
+                                                 gl=(global_head, global_tail), sb=sparse_block)
     return O, lse
 
 
@@ -214,14 +250,14 @@ def attn_fwd_rows(q, k, v, scale, causal, window, b, h, rows):
     return O, lse
 
 
-def _rows_bwd(qh, kh, vh, doh, scale, causal, window, r0, r1, gl=(0, 0)):
+def _rows_bwd(qh, kh, vh, doh, scale, causal, window, r0, r1, gl=(0, 0), sb=0):
     """Rows [r0, r1) of one head: their O and LSE, their dQ rows, and their
     contributions to dK and dV over the visible key band [lo, hi)."""
     Lq, Lk = qh.shape[0], kh.shape[0]
     off = diag_offset(causal, Lq, Lk)
     glob = (gl[0], gl[1], Lk)
     lo, hi = visible_band(r0, r1, Lk, causal, window, off, glob)
-    vis = _band_mask(np.arange(r0, r1), lo, hi, causal, window, off, glob)
+    vis = _band_mask(np.arange(r0, r1), lo, hi, causal, window, off, glob, sb, Lq, Lk)
     A, lse = attention_weights(qh[r0:r1], kh[lo:hi], scale, vis)
     O = A @ vh[lo:hi]
     dO = doh[r0:r1]
@@ -234,7 +270,7 @@ def _rows_bwd(qh, kh, vh, doh, scale, causal, window, r0, r1, gl=(0, 0)):
     return lo, hi, O, lse, dq, dk, dv
 
 
-def _head_bwd(qh, kh, vh, doh, scale, causal, window, gl=(0, 0)):
+def _head_bwd(qh, kh, vh, doh, scale, causal, window, gl=(0, 0), sb=0):
     """dQ, dK, dV for one (query head, kv head) pair; textbook softmax gradient."""
     Lq, Lk = qh.shape[0], kh.shape[0]
     dq = np.zeros_like(qh)
@@ -243,7 +279,7 @@ def _head_bwd(qh, kh, vh, doh, scale, causal, window, gl=(0, 0)):
     step = max(1, _ROW_BLOCK_ELEMS // max(1, Lk))
     for r0 in range(0, Lq, step):
         r1 = min(Lq, r0 + step)
-        lo, hi, _, _, dqb, dkb, dvb = _rows_bwd(qh, kh, vh, doh, scale, causal, window, r0, r1, gl)
+        lo, hi, _, _, dqb, dkb, dvb = _rows_bwd(qh, kh, vh, doh, scale, causal, window, r0, r1, gl, sb)
         dq[r0:r1] = dqb
         dk[lo:hi] += dkb
         dv[lo:hi] += dvb
@@ -264,14 +300,14 @@ def attn_row_block(q, k, v, do, scale, causal, window, b, h, r0, r1):
 
 
 def attn_bwd(q, k, v, do, scale: float, causal: bool = False, window: int = 0, heads=None, seqlens_q=None,
-             seqlens_k=None, global_head: int = 0, global_tail: int = 0):
+             seqlens_k=None, global_head: int = 0, global_tail: int = 0, sparse_block: int = 0):
     """dQ [B,Hq,Lq,d], dK and dV [B,Hkv,Lk,d] in float64.
 
     dK/dV of a K/V head are summed over the query heads that share it.
     heads: optional list of (b, hkv): only those K/V heads (and all query
     heads of their groups) are evaluated; the rest is left NaN.
-    seqlens_q / seqlens_k, global_head / global_tail: as attn_fwd; padded rows
-    and keys get zero gradients.
+    seqlens_q / seqlens_k, global_head / global_tail, sparse_block: as
+    attn_fwd; padded rows and keys get zero gradients.
     """
     q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
     B, Hq, Lq, d = q.shape
@@ -288,7 +324,7 @@ def attn_bwd(q, k, v, do, scale: float, causal: bool = False, window: int = 0, h
         for h in (h for h in range(Hq) if _kv_head(h, Hq, Hkv) == g):
             dq[b, h] = 0.0
             dqh, dkh, dvh = _head_bwd(q[b, h, :nq], k[b, g, :nk], v[b, g, :nk], do[b, h, :nq], scale, causal, window,
-                                      (global_head, global_tail))
+                                      (global_head, global_tail), sparse_block)
             dq[b, h, :nq] = dqh
             dk[b, g, :nk] += dkh
             dv[b, g, :nk] += dvh

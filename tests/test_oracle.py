@@ -269,6 +269,85 @@ def test_global_tokens_backward_finite_differences():
         np.testing.assert_allclose(G, num, atol=1e-6, rtol=0)
 
 
+# ---------------------------------------------------------------- block-sparse mask
+def _block_rule(Lq, Lk, b):
+    """Closed form of the block-sparse construction, written independently of
+    the oracle's loops: query i (block start s = b * floor(i / b)) sees keys
+    max(0, s - b) <= j < min(Lk, s + 2b - 1)."""
+    i = torch.arange(Lq)[:, None]
+    j = torch.arange(Lk)[None, :]
+    s = (i // b) * b
+    return (j >= (s - b).clamp(min=0)) & (j < (s + 2 * b - 1).clamp(max=Lk))
+
+
+@pytest.mark.parametrize("Lq,Lk,b,causal,w", [(40, 40, 8, False, 0), (40, 40, 5, True, 0), (33, 50, 7, False, 0),
+                                              (50, 33, 6, 2, 0), (40, 40, 8, False, 6), (30, 30, 3, True, 4)])
+def test_block_sparse_matches_torch_sdpa(Lq, Lk, b, causal, w):
+    """Block-sparse mask of "大模型高效注意力机制全解析" §4.1.2 (with causal / window
+    masks on top) against torch SDPA with the mask from the closed-form rule."""
+    q, k, v = _rand(1, 2, Lq, 5), _rand(1, 2, Lk, 5), _rand(1, 2, Lk, 5)
+    O, _ = oracle.attn_fwd(q, k, v, 0.45, causal, w, sparse_block=b)
+    i = torch.arange(Lq)[:, None]
+    j = torch.arange(Lk)[None, :]
+    off = Lk - Lq if causal == 2 else 0
+    mask = _block_rule(Lq, Lk, b)
+    if causal:
+        mask &= j <= i + off
+        if w:
+            mask &= j > i + off - w
+    elif w:
+        mask &= (i - j).abs() < w
+    ref = torch.nn.functional.scaled_dot_product_attention(*(torch.from_numpy(x) for x in (q, k, v)),
+                                                           attn_mask=mask, scale=0.45)
+    rows = mask.any(1).numpy()  # SDPA gives NaN on rows with no visible key
+    np.testing.assert_allclose(O[0, :, rows], ref.numpy()[0, :, rows], atol=1e-12)
+    assert np.all(O[0, :, ~rows] == 0.0)
+
+
+def test_block_sparse_pages_example_counts():
+    """The page's example (seq_len 1024, block 64): interior query blocks see
+    3b - 1 keys, the first block 2b - 1, the last 2b; the total follows."""
+    m = oracle.visible_mask(1024, 1024, False, 0, sparse_block=64)
+    per_row = m.sum(1)
+    assert set(per_row[:64]) == {127} and set(per_row[64:960]) == {191} and set(per_row[960:]) == {128}
+    assert m.sum() == 64 * (127 + 14 * 191 + 128)
+
+
+def test_block_sparse_degenerate_sizes():
+    """b >= L: every query sees every key (plain attention); b = 1: query i
+    sees keys i - 1 and i, the same as a causal window of two keys."""
+    q, k, v = _rand(1, 2, 17, 4), _rand(1, 2, 17, 4), _rand(1, 2, 17, 4)
+    O, lse = oracle.attn_fwd(q, k, v, 0.6, False, 0, sparse_block=17)
+    O0, lse0 = oracle.attn_fwd(q, k, v, 0.6, False, 0)
+    np.testing.assert_array_equal(O, O0)
+    np.testing.assert_array_equal(lse, lse0)
+    O, lse = oracle.attn_fwd(q, k, v, 0.6, False, 0, sparse_block=1)
+    O2, lse2 = oracle.attn_fwd(q, k, v, 0.6, True, 2)
+    np.testing.assert_allclose(O, O2, atol=1e-15)
+    np.testing.assert_allclose(lse, lse2, atol=1e-15)
+
+
+def test_block_sparse_backward_finite_differences():
+    """Gradient under the block-sparse mask against central differences."""
+    rng = np.random.default_rng(12)
+    q, k, v, R = (rng.standard_normal((1, 2, 11, 3)) for _ in range(4))
+    dq, dk, dv = oracle.attn_bwd(q, k, v, R, 0.5, False, 0, sparse_block=3)
+    eps = 1e-5
+    for X, G in ((q, dq), (k, dk), (v, dv)):
+        num = np.zeros_like(X)
+        it = np.nditer(X, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            old = X[idx]
+            X[idx] = old + eps
+            fp = float(np.sum(oracle.attn_fwd(q, k, v, 0.5, False, 0, sparse_block=3)[0] * R))
+            X[idx] = old - eps
+            fm = float(np.sum(oracle.attn_fwd(q, k, v, 0.5, False, 0, sparse_block=3)[0] * R))
+            X[idx] = old
+            num[idx] = (fp - fm) / (2 * eps)
+        np.testing.assert_allclose(G, num, atol=1e-6, rtol=0)
+
+
 def test_value_shift_and_score_shift_invariance():
     """V + 1 c^T gives O + 1 c^T; a per-row constant added to the logits changes nothing."""
     L, d = 19, 4
@@ -535,7 +614,8 @@ def _pins_pass():
               lambda: test_zero_query_gives_mean_of_visible(True, 5),
               lambda: test_gqa_equals_mha_with_repeated_kv(4, 2),
               lambda: test_backward_matches_finite_differences(2, 1, 8, True, 3),
-              lambda: test_matches_torch_sdpa_float64(4, 2, True, 0)]
+              lambda: test_matches_torch_sdpa_float64(4, 2, True, 0),
+              lambda: test_block_sparse_matches_torch_sdpa(33, 50, 7, False, 0)]
     for c in checks:
         try:
             c()
@@ -548,7 +628,7 @@ def test_pins_pass_unmodified():
     assert _pins_pass()
 
 
-@pytest.mark.parametrize("slip", ["transpose", "no_mask", "dS_sign", "dk_no_scale", "gqa_map"])
+@pytest.mark.parametrize("slip", ["transpose", "no_mask", "dS_sign", "dk_no_scale", "gqa_map", "block_edge"])
 def test_pins_catch_planted_slips(monkeypatch, slip):
     """Plant a plausible mistake in the oracle (CPU only) and check a pin fails."""
     if slip == "transpose":
@@ -565,7 +645,21 @@ def test_pins_catch_planted_slips(monkeypatch, slip):
         monkeypatch.setattr(oa, "_head_bwd", _bwd_with(None, dk_scale=False))
     elif slip == "gqa_map":
         monkeypatch.setattr(oa, "_kv_head", lambda h, Hq, Hkv: h % Hkv)
+    elif slip == "block_edge":
+        # Each query block one key block too narrow on the right (j up to i + b - 2).
+        orig = oa.sparse_block_mask
+        monkeypatch.setattr(oa, "sparse_block_mask",
+                            lambda rows, lo, hi, b, Lq, Lk: orig(rows, lo, hi, b, Lq, Lk)
+                            & _drop_last_block_key(rows, lo, hi, b, Lk))
     assert not _pins_pass()
+
+
+def _drop_last_block_key(rows, lo, hi, b, Lk):
+    """Keep every key except the last one the block-sparse construction reaches."""
+    rows = np.asarray(rows)
+    s = (rows // b) * b
+    last = np.minimum(Lk, s + 2 * b - 1) - 1
+    return np.arange(lo, hi)[None, :] != last[:, None]
 
 
 def _transposed_weights(orig, q, k, s, vis):
@@ -584,9 +678,9 @@ def _transposed_weights(orig, q, k, s, vis):
 
 
 def _bwd_with(ds_fn, dk_scale=True):
-    def head_bwd(qh, kh, vh, doh, scale, causal, window, gl=(0, 0)):
+    def head_bwd(qh, kh, vh, doh, scale, causal, window, gl=(0, 0), sb=0):
         Lq, Lk = qh.shape[0], kh.shape[0]
-        vis = oracle.visible_mask(Lq, Lk, causal, window, *gl)
+        vis = oracle.visible_mask(Lq, Lk, causal, window, *gl, sparse_block=sb)
         A, _ = oa.attention_weights(qh, kh, scale, vis)
         O = A @ vh
         dP = doh @ vh.T
