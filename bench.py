@@ -292,22 +292,27 @@ def all_configs(args):
             return statistics.median(ts)
 
         n = max(5, min(args.steps, 50))
-        f_ms = timed(lambda: ta.fwd(q, k, v, o, lse, w.causal, w.window, w.scale), n)
+        sb = w.sparse_block
+        f_ms = timed(lambda: ta.fwd(q, k, v, o, lse, w.causal, w.window, w.scale, sparse_block=sb), n)
         ns = ta.lib.attn_fwd_split_default(w.B, w.Hq, w.Hkv, w.Lq, w.Lk, w.d, ta._causal_code(w.causal), w.window)
         split = None
-        if ns > 1:
+        if ns > 1 and not sb:
             sws = torch.empty(max(256, ta.lib.attn_fwd_split_workspace_size(w.B, w.Hq, w.Hkv, w.Lq, w.Lk, w.d, ns)),
                               dtype=torch.uint8, device="cuda")
             s_ms = timed(lambda: ta.fwd_split(q, k, v, o, lse, ns, sws, w.causal, w.window, w.scale), n)
             split = {"n_split": ns, "fwd_ms": s_ms, "fwd_tflops": w.fwd_flops() / s_ms / 1e9}
-        b_ms = timed(lambda: ta.bwd_phases(q, k, v, o, lse, do, dq, dk, dv, ws, w.causal, w.window, w.scale), n)
+        if sb:
+            b_ms = timed(lambda: ta.bwd(q, k, v, o, lse, do, dq, dk, dv, ws, w.causal, w.window, w.scale,
+                                        sparse_block=sb), n)
+        else:
+            b_ms = timed(lambda: ta.bwd_phases(q, k, v, o, lse, do, dq, dk, dv, ws, w.causal, w.window, w.scale), n)
         st, site = ta.device_error()
         if st != 0:
             raise SystemExit(f"device error {st} at site {site} on {name}")
         fwd_bytes = (q.numel() + k.numel() + v.numel() + o.numel()) * 2 + lse.numel() * 4
         print(json.dumps({
             "workload": name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.Lq, "d": w.d, "causal": w.causal,
-            "window": w.window, "fwd_ms": f_ms, "fwd_tflops": w.fwd_flops() / f_ms / 1e9,
+            "window": w.window, "sparse_block": sb, "fwd_ms": f_ms, "fwd_tflops": w.fwd_flops() / f_ms / 1e9,
             "fwd_frac_spec_2250": w.fwd_flops() / f_ms / 1e9 / 2250.0,
             "fwd_algorithmic_GBs": fwd_bytes / f_ms / 1e6, "hbm_peak_GBs": hbm,
             "fwd_split": None if split is None else dict(split, fwd_algorithmic_GBs=fwd_bytes / split["fwd_ms"] / 1e6),

@@ -96,6 +96,14 @@ ATTN_API int attn_fwd(const void* q, const void* k, const void* v, void* o, floa
  *                          global_tokens [0, -1]: the first and last tokens
  *                          globally visible); 0 for none
  *  seqlens_q, seqlens_k    as attn_fwd_varlen (device int32 [B] or NULL)
+ *  sparse_block            b >= 0: the block-sparse mask of
+ *                          "大模型高效注意力机制全解析" §4.1.2 with b x b
+ *                          blocks (0 for none): the query block starting at
+ *                          s = b * floor(i / b) sees the key blocks starting
+ *                          at every j in [s - b, s + b), i.e. keys
+ *                          [max(0, s - b), min(Lk, s + 2b - 1)); intersected
+ *                          with the causal and window masks (global keys stay
+ *                          visible on top).  b <= 2^28.
  */
 typedef struct {
   int causal;
@@ -104,6 +112,7 @@ typedef struct {
   int global_tail;
   const int* seqlens_q;
   const int* seqlens_k;
+  int sparse_block;
 } attn_mask;
 
 /*

@@ -19,6 +19,9 @@ Mistral example on the same page):
   gqa_decode_32768  B=4, Hq=32/Hkv=8, Lq=16 over Lk=32768, d=128, bottom-right
                     causal (new queries over a long cache, the KV-cache
                     setting of "高效注意力" §3)
+  mha_sparse64_4096 B=2, Hq=Hkv=32,  L=4096,  d=128, block-sparse mask with
+                    64 x 64 blocks (the block size of the example in
+                    "大模型高效注意力机制全解析" §4.1.2), no causal mask
 """
 
 from dataclasses import dataclass, field
@@ -41,6 +44,7 @@ class Workload:
     q_mult: float = 1.0      # applied after bf16 rounding (a power of two: exact)
     backward: bool = False
     seed: int = 42
+    sparse_block: int = 0    # block-sparse mask block size (0: none)
 
     @property
     def scale(self) -> float:
@@ -56,6 +60,10 @@ class Workload:
             else:
                 hi = min(i + self.window, self.Lk) if self.window > 0 else self.Lk
             lo = max(0, i + off - self.window + 1) if self.window > 0 else 0
+            if self.sparse_block > 0:
+                s = i // self.sparse_block * self.sparse_block
+                lo = max(lo, s - self.sparse_block)
+                hi = min(hi, s + 2 * self.sparse_block - 1)
             total += max(0, hi - lo)
         return total
 
@@ -78,6 +86,7 @@ WORKLOADS = {
         Workload("mha_causal_fwdbwd", 2, 32, 32, 4096, 4096, 128, True, backward=True, seed=46),
         # 16 new queries per sequence over a 32768-key cache (bottom-right causal)
         Workload("gqa_decode_32768", 4, 32, 8, 16, 32768, 128, 2, seed=47),
+        Workload("mha_sparse64_4096", 2, 32, 32, 4096, 4096, 128, 0, seed=48, sparse_block=64),
     ]
 }
 

@@ -148,7 +148,7 @@ def test_fwd_ex_and_bwd_ex_validate_the_mask(ta):
     """attn_fwd_ex / attn_bwd_ex: a NULL mask, negative global counts and a bad
     slice count are rejected before any launch."""
     import ctypes
-    m = ta.AttnMask(1, 0, -1, 0, None, None)
+    m = ta.AttnMask(1, 0, -1, 0, None, None, 0)
     args = (P, P, P, P, P, 1, 2, 2, 8, 8, 64, 0.125)
     assert ta.lib.attn_fwd_ex(*args, None, 1, None, 0, None) == 1
     assert ta.lib.attn_fwd_ex(*args, ctypes.byref(m), 1, None, 0, None) == 1
@@ -158,6 +158,19 @@ def test_fwd_ex_and_bwd_ex_validate_the_mask(ta):
     m.global_tail = -2
     assert ta.lib.attn_bwd_ex(*([P] * 9), 1, 2, 2, 8, 8, 64, 0.125, ctypes.byref(m), P, 1 << 20, None) == 1
     assert ta.lib.attn_bwd_ex(*([P] * 9), 1, 2, 2, 8, 8, 64, 0.125, None, P, 1 << 20, None) == 1
+    # Block-sparse block size: negative or above 2^28 is rejected.
+    for bad in (-1, (1 << 28) + 1):
+        m = ta.AttnMask(1, 0, 0, 0, None, None, bad)
+        assert ta.lib.attn_fwd_ex(*args, ctypes.byref(m), 1, None, 0, None) == 1
+        assert ta.lib.attn_bwd_ex(*([P] * 9), 1, 2, 2, 8, 8, 64, 0.125, ctypes.byref(m), P, 1 << 20, None) == 1
+
+
+def test_attn_mask_layout_matches_header(ta):
+    """The ctypes mirror of attn_mask has the header's field order and size."""
+    import ctypes
+    names = [f[0] for f in ta.AttnMask._fields_]
+    assert names == ["causal", "window", "global_head", "global_tail", "seqlens_q", "seqlens_k", "sparse_block"]
+    assert ctypes.sizeof(ta.AttnMask) == 40
 
 
 def _host_size(ta, B=2, Hq=8, Hkv=2, Lq=300, Lk=500, d=128, bwd=1):

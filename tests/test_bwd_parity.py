@@ -129,6 +129,34 @@ def test_bwd_global_tokens(ta, B, Hq, Hkv, Lq, Lk, d, causal, window, gh, gt):
     check_grad(to_f64(dv), rv, "dV")
 
 
+# Block-sparse mask ("大模型高效注意力机制全解析" §4.1.2), block size b, alone and under
+# causal / window masks, blocks smaller and larger than a tile, Lq != Lk.
+# (B, Hq, Hkv, Lq, Lk, d, causal, window, b)
+SPARSE = [
+    (1, 2, 2, 700, 700, 128, 0, 0, 64),
+    (1, 4, 2, 1000, 1000, 128, 1, 0, 128),
+    (2, 2, 1, 300, 500, 64, 2, 0, 50),
+    (1, 2, 2, 513, 513, 128, 0, 100, 200),
+    (1, 4, 4, 257, 257, 64, 1, 64, 1),
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Lq,Lk,d,causal,window,b", SPARSE)
+def test_bwd_sparse_block(ta, B, Hq, Hkv, Lq, Lk, d, causal, window, b):
+    """Gradients under the block-sparse mask, against the oracle."""
+    x = make_shape_inputs(B, Hq, Hkv, Lq, Lk, d, seed=Lq * 23 + Lk + d + b, with_do=True)
+    scale = d ** -0.5
+    q, k, v, do = (to_dev(x[n]) for n in ("q", "k", "v", "do"))
+    o, lse = ta.attention(q, k, v, causal, window, scale, sparse_block=b)
+    dq, dk, dv = ta.attention_backward(q, k, v, o, lse, do, causal, window, scale, sparse_block=b)
+    st, site = ta.device_error()
+    assert st == 0, f"device error {st} at site {site}"
+    rq, rk, rv = oracle.attn_bwd(x["q"], x["k"], x["v"], x["do"], scale, causal, window, sparse_block=b)
+    check_grad(to_f64(dq), rq, "dQ")
+    check_grad(to_f64(dk), rk, "dK")
+    check_grad(to_f64(dv), rv, "dV")
+
+
 def test_bwd_gqa_window_2048(ta):
     x = make_shape_inputs(1, 8, 2, 2048, 2048, 128, seed=17, with_do=True)
     dq, dk, dv = run_fwd_bwd(ta, x, True, 300, 128 ** -0.5)

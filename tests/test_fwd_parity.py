@@ -4,6 +4,8 @@ Same seeded bf16 inputs on both sides.  Tolerances: O max-abs 1e-2 and
 relative Frobenius 5e-3; LSE 1e-5 relative (absolute below |LSE| = 1).
 """
 
+import ctypes
+
 import numpy as np
 import pytest
 
@@ -22,9 +24,9 @@ def ta():
     return ta
 
 
-def run_fwd(ta, x, causal, window, scale):
+def run_fwd(ta, x, causal, window, scale, sparse_block=0):
     q, k, v = (to_dev(x[n]) for n in "qkv")
-    o, lse = ta.attention(q, k, v, causal, window, scale)
+    o, lse = ta.attention(q, k, v, causal, window, scale, sparse_block=sparse_block)
     st, site = ta.device_error()
     assert st == 0, f"device error {st} at site {site}"
     return to_f64(o), to_f64(lse)
@@ -164,6 +166,45 @@ GLOBAL = [
 ]
 
 
+# Block-sparse mask ("大模型高效注意力机制全解析" §4.1.2), block size b: blocks below,
+# at and above the tile size, with causal (both alignments) and window masks,
+# packed short queries, split-KV and global keys on top.
+# (B, Hq, Hkv, Lq, Lk, d, causal, window, b, n_split, gh, gt)
+SPARSE = [
+    (1, 2, 2, 1024, 1024, 128, 0, 0, 64, 1, 0, 0),
+    (2, 4, 2, 700, 700, 128, 1, 0, 128, 1, 0, 0),
+    (1, 2, 1, 300, 500, 64, 2, 0, 50, 1, 0, 0),
+    (1, 2, 2, 513, 513, 128, 0, 100, 200, 1, 0, 0),
+    (1, 3, 3, 257, 257, 64, 1, 64, 1, 1, 0, 0),
+    (2, 8, 2, 16, 2000, 128, 2, 0, 300, 1, 0, 0),
+    (1, 2, 2, 100, 3000, 128, 0, 0, 256, 4, 0, 0),
+    (1, 2, 2, 600, 600, 128, 0, 0, 64, 1, 2, 3),
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Lq,Lk,d,causal,window,b,ns,gh,gt", SPARSE)
+def test_fwd_sparse_block(ta, B, Hq, Hkv, Lq, Lk, d, causal, window, b, ns, gh, gt):
+    """Block-sparse forward through attn_fwd_ex against the oracle."""
+    import torch
+    x = make_shape_inputs(B, Hq, Hkv, Lq, Lk, d, seed=Lq * 29 + Lk + d + b)
+    scale = d ** -0.5
+    q, k, v = (to_dev(x[n]) for n in "qkv")
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device="cuda")
+    ws = torch.empty(max(256, ta.lib.attn_fwd_split_workspace_size(B, Hq, Hkv, Lq, Lk, d, ns)), dtype=torch.uint8,
+                     device="cuda")
+    m = ta.AttnMask(ta._causal_code(causal), window, gh, gt, None, None, b)
+    st = ta.lib.attn_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, Hq, Hkv, Lq,
+                            Lk, d, scale, ctypes.byref(m), ns, ws.data_ptr(), ws.numel(), None)
+    assert st == 0
+    st, site = ta.device_error()
+    assert st == 0, f"device error {st} at site {site}"
+    ro, rl = oracle.attn_fwd(x["q"], x["k"], x["v"], scale, causal, window, global_head=gh, global_tail=gt,
+                             sparse_block=b)
+    check_o(to_f64(o), ro, "O")
+    check_lse(to_f64(lse), rl, "LSE")
+
+
 @pytest.mark.parametrize("B,Hq,Hkv,Lq,Lk,d,causal,window,gh,gt", GLOBAL)
 def test_fwd_global_tokens(ta, B, Hq, Hkv, Lq, Lk, d, causal, window, gh, gt):
     """Global head/tail key positions on top of the window, against the oracle."""
@@ -191,7 +232,7 @@ def test_fwd_global_tokens_split_and_varlen(ta):
     lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device="cuda")
     tq = torch.tensor(lq, dtype=torch.int32, device="cuda")
     tk = torch.tensor(lk, dtype=torch.int32, device="cuda")
-    m = ta.AttnMask(2, w, gh, gt, tq.data_ptr(), tk.data_ptr())
+    m = ta.AttnMask(2, w, gh, gt, tq.data_ptr(), tk.data_ptr(), 0)
     ws = torch.empty(ta.lib.attn_fwd_split_workspace_size(B, Hq, Hkv, Lq, Lk, d, ns), dtype=torch.uint8, device="cuda")
     st = ta.lib.attn_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, Hq, Hkv, Lq,
                             Lk, d, scale, ctypes.byref(m), ns, ws.data_ptr(), ws.numel(),
@@ -246,14 +287,16 @@ def test_fwd_single_head_128(ta):
     ("mha_causal_4096", [(0, 0), (1, 31), (0, 17)]),
     ("gqa_causal_8192", [(0, 0), (3, 31), (2, 9)]),
     ("gqa_window_32768", [(0, 0), (0, 21)]),
+    ("mha_sparse64_4096", [(0, 0), (1, 31)]),
 ])
 def test_fwd_full_size_sampled_heads(ta, name, heads):
     """Full-size workloads in the benchmark's launch configuration; whole heads
     (independent units) are compared against the oracle."""
     w = WORKLOADS[name]
     x = make_inputs(w)
-    o, lse = run_fwd(ta, x, w.causal, w.window, w.scale)
-    ro, rl = oracle.attn_fwd(x["q"], x["k"], x["v"], w.scale, w.causal, w.window, heads=heads)
+    o, lse = run_fwd(ta, x, w.causal, w.window, w.scale, w.sparse_block)
+    ro, rl = oracle.attn_fwd(x["q"], x["k"], x["v"], w.scale, w.causal, w.window, heads=heads,
+                             sparse_block=w.sparse_block)
     for b, h in heads:
         check_o(o[b, h], ro[b, h], f"{name} O[{b},{h}]")
         check_lse(lse[b, h], rl[b, h], f"{name} LSE[{b},{h}]")

@@ -35,7 +35,8 @@ class AttnError(RuntimeError):
 class AttnMask(ctypes.Structure):
     """The C ABI's attn_mask."""
     _fields_ = [("causal", ctypes.c_int), ("window", ctypes.c_int), ("global_head", ctypes.c_int),
-                ("global_tail", ctypes.c_int), ("seqlens_q", ctypes.c_void_p), ("seqlens_k", ctypes.c_void_p)]
+                ("global_tail", ctypes.c_int), ("seqlens_q", ctypes.c_void_p), ("seqlens_k", ctypes.c_void_p),
+                ("sparse_block", ctypes.c_int)]
 
 
 def _load() -> ctypes.CDLL:
@@ -148,7 +149,7 @@ def _lens(seqlens, B, name):
 
 
 def fwd(q, k, v, o, lse, causal: bool = False, window: int = 0, scale: float | None = None, stream=None,
-        seqlens_q=None, seqlens_k=None, global_head: int = 0, global_tail: int = 0):
+        seqlens_q=None, seqlens_k=None, global_head: int = 0, global_tail: int = 0, sparse_block: int = 0):
     """attn_fwd on torch tensors (bf16 q/k/v/o, fp32 lse), asynchronous on
     `stream`; with seqlens_q / seqlens_k (int32 CUDA [B]) attn_fwd_varlen."""
     import torch
@@ -160,8 +161,8 @@ def fwd(q, k, v, o, lse, causal: bool = False, window: int = 0, scale: float | N
         raise ValueError("v/o/lse shape mismatch")
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     lq, lk = _lens(seqlens_q, B, "seqlens_q"), _lens(seqlens_k, B, "seqlens_k")
-    if global_head or global_tail:
-        m = AttnMask(_causal_code(causal), int(window), int(global_head), int(global_tail), lq, lk)
+    if global_head or global_tail or sparse_block:
+        m = AttnMask(_causal_code(causal), int(window), int(global_head), int(global_tail), lq, lk, int(sparse_block))
         st = lib.attn_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
                              B, Hq, Hkv, Lq, Lk, d, scale, ctypes.byref(m), 1, None, 0, _stream_ptr(stream))
         _check(st, "attn_fwd_ex")
@@ -182,7 +183,7 @@ def bwd_workspace_size(B, Hq, Hkv, Lq, Lk, d) -> int:
 
 def bwd(q, k, v, o, lse, do, dq, dk, dv, workspace, causal: bool = False, window: int = 0,
         scale: float | None = None, stream=None, seqlens_q=None, seqlens_k=None, global_head: int = 0,
-        global_tail: int = 0):
+        global_tail: int = 0, sparse_block: int = 0):
     """attn_bwd on torch tensors; `workspace` is a uint8 CUDA tensor; with
     seqlens_q / seqlens_k attn_bwd_varlen."""
     import torch
@@ -194,8 +195,8 @@ def bwd(q, k, v, o, lse, do, dq, dk, dv, workspace, causal: bool = False, window
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     lq, lk = _lens(seqlens_q, B, "seqlens_q"), _lens(seqlens_k, B, "seqlens_k")
     wsp, wsb = workspace.data_ptr(), workspace.numel() * workspace.element_size()
-    if global_head or global_tail:
-        m = AttnMask(_causal_code(causal), int(window), int(global_head), int(global_tail), lq, lk)
+    if global_head or global_tail or sparse_block:
+        m = AttnMask(_causal_code(causal), int(window), int(global_head), int(global_tail), lq, lk, int(sparse_block))
         st = lib.attn_bwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
                              dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv, Lq, Lk, d, scale,
                              ctypes.byref(m), wsp, wsb, _stream_ptr(stream))
@@ -267,14 +268,14 @@ def device_error(stream=None) -> tuple[int, int]:
 
 
 def attention(q, k, v, causal: bool = False, window: int = 0, scale: float | None = None, seqlens_q=None,
-              seqlens_k=None, global_head: int = 0, global_tail: int = 0):
+              seqlens_k=None, global_head: int = 0, global_tail: int = 0, sparse_block: int = 0):
     """Allocate O and LSE with torch and run the forward pass."""
     import torch
     B, Hq, Hkv, Lq, Lk, d = _shapes(q, k)
     o = torch.empty_like(q)
     lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
     fwd(q, k, v, o, lse, causal, window, scale, seqlens_q=seqlens_q, seqlens_k=seqlens_k, global_head=global_head,
-        global_tail=global_tail)
+        global_tail=global_tail, sparse_block=sparse_block)
     return o, lse
 
 
@@ -308,14 +309,15 @@ def attention_split(q, k, v, causal: bool = False, window: int = 0, scale: float
 
 
 def attention_backward(q, k, v, o, lse, do, causal: bool = False, window: int = 0, scale: float | None = None,
-                       seqlens_q=None, seqlens_k=None, global_head: int = 0, global_tail: int = 0):
+                       seqlens_q=None, seqlens_k=None, global_head: int = 0, global_tail: int = 0,
+                       sparse_block: int = 0):
     """Allocate dQ/dK/dV and the workspace with torch and run the backward pass."""
     import torch
     B, Hq, Hkv, Lq, Lk, d = _shapes(q, k)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     ws = torch.empty(max(1, bwd_workspace_size(B, Hq, Hkv, Lq, Lk, d)), dtype=torch.uint8, device=q.device)
     bwd(q, k, v, o, lse, do, dq, dk, dv, ws, causal, window, scale, seqlens_q=seqlens_q, seqlens_k=seqlens_k,
-        global_head=global_head, global_tail=global_tail)
+        global_head=global_head, global_tail=global_tail, sparse_block=sparse_block)
     return dq, dk, dv
 
 

@@ -153,10 +153,10 @@ const char* attn_status_string(int status) {
 // slices written to `workspace` and merged.
 static int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, const int* lens_q,
                     const int* lens_k, int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale, int causal,
-                    int window, int gh, int gt, int n_split, void* workspace, void* stream) {
+                    int window, int gh, int gt, int sb, int n_split, void* workspace, void* stream) {
   int st = check_shape(B, Hq, Hkv, Lq, Lk, d, scale, causal, window);
   if (st != ATTN_OK) return st;
-  if (gh < 0 || gt < 0) return ATTN_ERR_INVALID_ARG;
+  if (gh < 0 || gt < 0 || sb < 0 || sb > (1 << 28)) return ATTN_ERR_INVALID_ARG;
   if (B == 0 || Hq == 0 || Lq == 0) return ATTN_OK;
   if (!q || !o || !lse || !aligned16(q) || !aligned16(o) || !aligned16(lse)) return ATTN_ERR_INVALID_ARG;
   if (Lk > 0 && (!k || !v || !aligned16(k) || !aligned16(v))) return ATTN_ERR_INVALID_ARG;
@@ -171,6 +171,7 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, float*
   P.prob.len_k = lens_k;
   P.prob.global_head = gh;
   P.prob.global_tail = gt;
+  P.prob.sparse_block = sb;
   // With Lk == 0 nothing reads K/V; map Q's memory so the descriptors stay valid.
   const void* kp = Lk > 0 ? k : q;
   const void* vp = Lk > 0 ? v : q;
@@ -205,14 +206,14 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, float*
 
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Lq,
              int Lk, int d, float scale, int causal, int window, void* stream) {
-  return fwd_impl(q, k, v, o, lse, nullptr, nullptr, B, Hq, Hkv, Lq, Lk, d, scale, causal, window, 0, 0, 1, nullptr,
+  return fwd_impl(q, k, v, o, lse, nullptr, nullptr, B, Hq, Hkv, Lq, Lk, d, scale, causal, window, 0, 0, 0, 1, nullptr,
                   stream);
 }
 
 int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int* seqlens_q,
                     const int* seqlens_k, int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale, int causal,
                     int window, void* stream) {
-  return fwd_impl(q, k, v, o, lse, seqlens_q, seqlens_k, B, Hq, Hkv, Lq, Lk, d, scale, causal, window, 0, 0, 1,
+  return fwd_impl(q, k, v, o, lse, seqlens_q, seqlens_k, B, Hq, Hkv, Lq, Lk, d, scale, causal, window, 0, 0, 0, 1,
                   nullptr, stream);
 }
 
@@ -262,7 +263,7 @@ int attn_fwd_split(const void* q, const void* k, const void* v, void* o, float* 
   const size_t need = attn_fwd_split_workspace_size(B, Hq, Hkv, Lq, Lk, d, n_split);
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need)
     return ATTN_ERR_INVALID_ARG;
-  return fwd_impl(q, k, v, o, lse, nullptr, nullptr, B, Hq, Hkv, Lq, Lk, d, scale, causal, window, 0, 0, n_split,
+  return fwd_impl(q, k, v, o, lse, nullptr, nullptr, B, Hq, Hkv, Lq, Lk, d, scale, causal, window, 0, 0, 0, n_split,
                   workspace, stream);
 }
 
@@ -302,10 +303,10 @@ int attn_bwd_preprocess(const void* o, const void* dO, int B, int Hq, int Lq, in
 
 static int bwd_main_impl(const void* q, const void* k, const void* v, const float* lse, const void* dO, void* dk,
                          void* dv, const int* lens_q, const int* lens_k, int B, int Hq, int Hkv, int Lq, int Lk, int d,
-                         float scale, int causal, int window, int gh, int gt, void* workspace,
+                         float scale, int causal, int window, int gh, int gt, int sb, void* workspace,
                          size_t workspace_bytes, void* stream) {
   int st = check_shape(B, Hq, Hkv, Lq, Lk, d, scale, causal, window);
-  if (st == ATTN_OK && (gh < 0 || gt < 0)) st = ATTN_ERR_INVALID_ARG;
+  if (st == ATTN_OK && (gh < 0 || gt < 0 || sb < 0 || sb > (1 << 28))) st = ATTN_ERR_INVALID_ARG;
   if (st != ATTN_OK) return st;
   if (B == 0 || Hq == 0 || Lk == 0) return ATTN_OK;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -331,6 +332,7 @@ static int bwd_main_impl(const void* q, const void* k, const void* v, const floa
   P.prob.len_k = lens_k;
   P.prob.global_head = gh;
   P.prob.global_tail = gt;
+  P.prob.sparse_block = sb;
   const int bm = bwd_block_m(d);
   if ((st = make_map(enc, &P.tm_q, q, B * Hq, Lq, d, bm)) != ATTN_OK) return st;
   if ((st = make_map(enc, &P.tm_do, dO, B * Hq, Lq, d, bm)) != ATTN_OK) return st;
@@ -367,7 +369,7 @@ int attn_bwd_main(const void* q, const void* k, const void* v, const float* lse,
                   int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale, int causal, int window, void* workspace,
                   size_t workspace_bytes, void* stream) {
   return bwd_main_impl(q, k, v, lse, dO, dk, dv, nullptr, nullptr, B, Hq, Hkv, Lq, Lk, d, scale, causal, window, 0,
-                       0, workspace, workspace_bytes, stream);
+                       0, 0, workspace, workspace_bytes, stream);
 }
 
 int attn_bwd_main_varlen(const void* q, const void* k, const void* v, const float* lse, const void* dO, void* dk,
@@ -375,7 +377,7 @@ int attn_bwd_main_varlen(const void* q, const void* k, const void* v, const floa
                          int d, float scale, int causal, int window, void* workspace, size_t workspace_bytes,
                          void* stream) {
   return bwd_main_impl(q, k, v, lse, dO, dk, dv, seqlens_q, seqlens_k, B, Hq, Hkv, Lq, Lk, d, scale, causal, window,
-                       0, 0, workspace, workspace_bytes, stream);
+                       0, 0, 0, workspace, workspace_bytes, stream);
 }
 
 int attn_bwd_finalize(void* dq, int B, int Hq, int Lq, int d, float scale, void* workspace, size_t workspace_bytes,
@@ -392,16 +394,16 @@ int attn_bwd_finalize(void* dq, int B, int Hq, int Lq, int d, float scale, void*
 
 static int bwd_impl(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
                     void* dq, void* dk, void* dv, const int* lens_q, const int* lens_k, int B, int Hq, int Hkv, int Lq,
-                    int Lk, int d, float scale, int causal, int window, int gh, int gt, void* workspace,
+                    int Lk, int d, float scale, int causal, int window, int gh, int gt, int sb, void* workspace,
                     size_t workspace_bytes, void* stream) {
   int st = check_shape(B, Hq, Hkv, Lq, Lk, d, scale, causal, window);
   if (st != ATTN_OK) return st;
-  if (gh < 0 || gt < 0) return ATTN_ERR_INVALID_ARG;
+  if (gh < 0 || gt < 0 || sb < 0 || sb > (1 << 28)) return ATTN_ERR_INVALID_ARG;
   if (B == 0 || Hq == 0) return ATTN_OK;
   if (Lq == 0 || Lk == 0) {
     if (Lq == 0)  // dK = dV = 0
       return bwd_main_impl(q, k, v, lse, dO, dk, dv, lens_q, lens_k, B, Hq, Hkv, Lq, Lk, d, scale, causal, window,
-                           gh, gt, workspace, workspace_bytes, stream);
+                           gh, gt, sb, workspace, workspace_bytes, stream);
     // No key: every row is fully masked, dQ = 0.
     if (!dq || !aligned16(dq)) return ATTN_ERR_INVALID_ARG;
     const cudaError_t e = cudaMemsetAsync(dq, 0, (size_t)B * Hq * Lq * d * 2, static_cast<cudaStream_t>(stream));
@@ -415,7 +417,7 @@ static int bwd_impl(const void* q, const void* k, const void* v, const void* o, 
   if ((st = split_workspace(B, Hq, Lq, d, workspace, workspace_bytes, &dvec, &dq_acc)) != ATTN_OK) return st;
   if ((st = attn_bwd_preprocess(o, dO, B, Hq, Lq, d, workspace, workspace_bytes, stream)) != ATTN_OK) return st;
   if ((st = bwd_main_impl(q, k, v, lse, dO, dk, dv, lens_q, lens_k, B, Hq, Hkv, Lq, Lk, d, scale, causal, window,
-                          gh, gt, workspace, workspace_bytes, stream)) != ATTN_OK)
+                          gh, gt, sb, workspace, workspace_bytes, stream)) != ATTN_OK)
     return st;
   return attn_bwd_finalize(dq, B, Hq, Lq, d, scale, workspace, workspace_bytes, stream);
 }
@@ -424,7 +426,7 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
              void* dk, void* dv, int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale, int causal, int window,
              void* workspace, size_t workspace_bytes, void* stream) {
   return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, nullptr, nullptr, B, Hq, Hkv, Lq, Lk, d, scale, causal, window, 0,
-                  0, workspace, workspace_bytes, stream);
+                  0, 0, workspace, workspace_bytes, stream);
 }
 
 int attn_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
@@ -432,7 +434,7 @@ int attn_bwd_varlen(const void* q, const void* k, const void* v, const void* o, 
                     int Lq, int Lk, int d, float scale, int causal, int window, void* workspace,
                     size_t workspace_bytes, void* stream) {
   return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, seqlens_q, seqlens_k, B, Hq, Hkv, Lq, Lk, d, scale, causal, window,
-                  0, 0, workspace, workspace_bytes, stream);
+                  0, 0, 0, workspace, workspace_bytes, stream);
 }
 
 const char* attn_last_cuda_error(void) { return g_last_err; }
@@ -450,7 +452,7 @@ int attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse
       return ATTN_ERR_INVALID_ARG;
   }
   return fwd_impl(q, k, v, o, lse, mask->seqlens_q, mask->seqlens_k, B, Hq, Hkv, Lq, Lk, d, scale, mask->causal,
-                  mask->window, mask->global_head, mask->global_tail, n_split, workspace, stream);
+                  mask->window, mask->global_head, mask->global_tail, mask->sparse_block, n_split, workspace, stream);
 }
 
 int attn_bwd_ex(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO, void* dq,
@@ -458,7 +460,8 @@ int attn_bwd_ex(const void* q, const void* k, const void* v, const void* o, cons
                 void* workspace, size_t workspace_bytes, void* stream) {
   if (!mask) return ATTN_ERR_INVALID_ARG;
   return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, mask->seqlens_q, mask->seqlens_k, B, Hq, Hkv, Lq, Lk, d, scale,
-                  mask->causal, mask->window, mask->global_head, mask->global_tail, workspace, workspace_bytes, stream);
+                  mask->causal, mask->window, mask->global_head, mask->global_tail, mask->sparse_block, workspace,
+                  workspace_bytes, stream);
 }
 
 int attn_get_device_error(void* stream, int* site) {

@@ -325,6 +325,12 @@ __device__ void grad_rows(const BwdParams& P, const Unit& u, uint8_t* smem, Bars
     const int off = diag_off(ps);
     vis_lo = ps.causal ? imax(0, key - off) : (ps.window > 0 ? imax(0, key - ps.window + 1) : 0);
     vis_hi = ps.window > 0 ? imin(ps.Lq, key - off + ps.window) : ps.Lq;
+    if (ps.sparse_block > 0) {
+      int slo, shi;
+      sparse_key_rows(ps, key, key + 1, slo, shi);
+      vis_lo = imax(vis_lo, slo);
+      vis_hi = imin(vis_hi, shi);
+    }
     // A global key is seen by every query (at or past it under a causal mask).
     if (key < ps.global_head || key >= tail_start(ps)) {
       vis_lo = ps.causal ? imax(0, key - off) : 0;

@@ -35,6 +35,9 @@ struct Problem {
   // to the causal mask.
   int global_head = 0;
   int global_tail = 0;
+  // Block-sparse mask ("大模型高效注意力机制全解析" §4.1.2), block size b
+  // (0: none): intersected with the causal and window masks.
+  int sparse_block = 0;
 };
 
 // The problem of sequence b: Lq and Lk replaced by its own lengths (for the
@@ -62,6 +65,27 @@ __host__ __device__ inline bool global_visible(const Problem& p, int i, int j) {
   if (i >= p.Lq || j >= p.Lk) return false;
   if (!(j < p.global_head || j >= tail_start(p))) return false;
   return !p.causal || j <= i + diag_off(p);
+}
+
+// Block-sparse mask with b x b blocks: the page's construction sets, for the
+// query block starting at s and every key start j in [s - b, s + b), the
+// block of keys [j, j + b); their union is the key range
+// [max(0, s - b), min(Lk, s + 2b - 1)), the same for every row of the block.
+__host__ __device__ inline int sparse_key_lo(const Problem& p, int i) {
+  const int b = p.sparse_block;
+  return imax(0, i / b * b - b);
+}
+__host__ __device__ inline int sparse_key_hi(const Problem& p, int i) {
+  const int b = p.sparse_block;
+  return imin(p.Lk, i / b * b + 2 * b - 1);
+}
+// Query rows [lo, hi) whose block-sparse key range meets keys [k0, k1)
+// (k0 < k1): block starts s with s + 2b - 1 > k0 and s - b < k1.
+__host__ __device__ inline void sparse_key_rows(const Problem& p, int k0, int k1, int& lo, int& hi) {
+  const int b = p.sparse_block;
+  const int t = k0 - 2 * b + 2;  // smallest admissible block start, before rounding up to a block
+  lo = t <= 0 ? 0 : cdiv(t, b) * b;
+  hi = (cdiv(k1, b) + 1) * b;
 }
 
 // The key tiles a query tile walks, as three ranges in walk order: the global
@@ -146,6 +170,10 @@ __host__ __device__ inline void row_key_range(const Problem& p, int i, int& key_
   const int off = diag_off(p);
   key_hi = p.causal ? imin(p.Lk, i + off + 1) : (p.window > 0 ? imin(p.Lk, i + p.window) : p.Lk);
   key_lo = p.window > 0 ? imax(0, i + off - p.window + 1) : 0;
+  if (p.sparse_block > 0) {
+    key_lo = imax(key_lo, sparse_key_lo(p, i));
+    key_hi = imin(key_hi, sparse_key_hi(p, i));
+  }
 }
 
 // Key tiles [lo, hi) (tiles of bn keys) holding any key visible to any query
@@ -156,8 +184,13 @@ __host__ __device__ inline void kv_tile_range(const Problem& p, int q0, int q1, 
   if (q0 >= q1) return;
   const int off = diag_off(p);
   // The last row reaches furthest forward, the first row furthest back.
-  const int key_hi = p.causal ? imin(p.Lk, q1 + off) : (p.window > 0 ? imin(p.Lk, q1 - 1 + p.window) : p.Lk);
-  const int key_lo = p.window > 0 ? imax(0, q0 + off - p.window + 1) : 0;
+  int key_hi = p.causal ? imin(p.Lk, q1 + off) : (p.window > 0 ? imin(p.Lk, q1 - 1 + p.window) : p.Lk);
+  int key_lo = p.window > 0 ? imax(0, q0 + off - p.window + 1) : 0;
+  if (p.sparse_block > 0) {
+    // Both ends of every mask's key range only grow with the row.
+    key_lo = imax(key_lo, sparse_key_lo(p, q0));
+    key_hi = imin(key_hi, sparse_key_hi(p, q1 - 1));
+  }
   if (key_lo >= key_hi) return;
   lo = key_lo / bn;
   hi = cdiv(key_hi, bn);
@@ -192,6 +225,12 @@ __host__ __device__ inline void q_row_range(const Problem& p, int k0, int k1, in
   int lo = p.causal ? imax(0, k0 - off) : (p.window > 0 ? imax(0, k0 - p.window + 1) : 0);
   // j > i + off - w  =>  i < j - off + w
   int hi = p.window > 0 ? imin(p.Lq, (k1 - 1) - off + p.window) : p.Lq;
+  if (p.sparse_block > 0) {
+    int slo, shi;
+    sparse_key_rows(p, k0, k1, slo, shi);
+    lo = imax(lo, slo);
+    hi = imin(hi, shi);
+  }
   // A global key in the tile is seen by every row (every row at or past it
   // under a causal mask); the band's rows lie inside that range.
   if (has_global(p)) {
