@@ -684,7 +684,11 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const uint16_t* __restrict
 }
 
 // dQ[bh, q, :] = scale * acc[bh, :, q], rounded to bf16.  One CTA transposes a
-// 64-query x d tile through shared memory: reads run along q, writes along d.
+// 64-query x d tile through shared memory: reads run along q (16 bytes per
+// thread: lq_pad is a multiple of 4 and the accumulator is 256-byte aligned,
+// so every 4-query group below lq_pad is one aligned float4), writes along d.
+// Accumulator columns in [Lq, lq_pad) were zeroed by the preprocess and are
+// read but never written out.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_post_kernel(const float* __restrict__ acc, uint16_t* __restrict__ dq, int Lq,
                                                        int lq_pad, float scale) {
@@ -692,9 +696,15 @@ __global__ void __launch_bounds__(256) bwd_post_kernel(const float* __restrict__
   const int bh = blockIdx.y;
   const int q0 = blockIdx.x * 64;
   const float* src = acc + (size_t)bh * D * lq_pad;
-  for (int idx = threadIdx.x; idx < D * 64; idx += 256) {
-    const int dd = idx / 64, qq = idx % 64;
-    tile[dd][qq] = q0 + qq < Lq ? src[(size_t)dd * lq_pad + q0 + qq] : 0.f;
+  for (int idx = threadIdx.x; idx < D * 16; idx += 256) {
+    const int dd = idx / 16, qv = idx % 16;
+    const int q = q0 + 4 * qv;
+    float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (q < lq_pad) f = *reinterpret_cast<const float4*>(src + (size_t)dd * lq_pad + q);
+    tile[dd][4 * qv] = f.x;
+    tile[dd][4 * qv + 1] = f.y;
+    tile[dd][4 * qv + 2] = f.z;
+    tile[dd][4 * qv + 3] = f.w;
   }
   __syncthreads();
   constexpr int CH = D / 8;  // 16-byte output chunks per row
