@@ -136,6 +136,8 @@ def attention_weights(q, k, scale: float, vis: np.ndarray):
     Returns (A, lse): A[i, j] = exp(S_ij) / sum_vis exp(S_ij) on visible
     entries and exactly 0 elsewhere; lse[i] = log sum_vis exp(S_ij).
     """
+    if k.shape[0] == 0:  # no key at all (a sequence of a padded batch with no keys): every row is fully masked
+        return np.zeros((q.shape[0], 0)), np.full(q.shape[0], -np.inf)
     S = scale * (q @ k.T)
     S = np.where(vis, S, -np.inf)
     m = S.max(axis=1, keepdims=True)

@@ -303,6 +303,46 @@ def test_fwd_full_size_sampled_heads(ta, name, heads):
     assert np.all(np.isfinite(o))
 
 
+# More units than SMs (several waves of CTAs): plain, alternating slots (G = 1
+# with short queries, and packed GQA rows with sequences of no queries or no
+# keys between full ones), split-KV, global keys, d = 64.
+# (B, Hq, Hkv, Lq, Lk, d, causal, window, n_split, gh, gt, seqlens_q, seqlens_k)
+MANY_UNITS = [
+    (4, 32, 32, 300, 300, 128, 1, 0, 1, 0, 0, None, None),
+    (8, 40, 40, 100, 700, 64, 2, 0, 1, 0, 0, None, None),
+    (24, 32, 8, 16, 600, 128, 2, 0, 1, 0, 0, [16, 0, 5, 16, 0, 0, 9, 16] * 3, [600, 17, 300, 0, 600, 40, 9, 128] * 3),
+    (2, 64, 8, 16, 5000, 128, 2, 0, 20, 0, 0, None, None),
+    (4, 32, 8, 300, 300, 128, 0, 64, 1, 2, 2, None, None),
+    (3, 48, 48, 257, 257, 64, 1, 100, 1, 0, 0, None, None),
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Lq,Lk,d,causal,window,ns,gh,gt,lq,lk", MANY_UNITS)
+def test_fwd_many_units(ta, B, Hq, Hkv, Lq, Lk, d, causal, window, ns, gh, gt, lq, lk):
+    """Problems with more units than SMs, through attn_fwd_ex, against the oracle."""
+    import torch
+    x = make_shape_inputs(B, Hq, Hkv, Lq, Lk, d, seed=B * 31 + Hq + Lq + Lk + d)
+    scale = d ** -0.5
+    q, k, v = (to_dev(x[n]) for n in "qkv")
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device="cuda")
+    ws = torch.empty(max(256, ta.lib.attn_fwd_split_workspace_size(B, Hq, Hkv, Lq, Lk, d, ns)), dtype=torch.uint8,
+                     device="cuda")
+    tq = torch.tensor(lq, dtype=torch.int32, device="cuda") if lq else None
+    tk = torch.tensor(lk, dtype=torch.int32, device="cuda") if lk else None
+    m = ta.AttnMask(ta._causal_code(causal), window, gh, gt, tq.data_ptr() if lq else None,
+                    tk.data_ptr() if lk else None, 0)
+    st = ta.lib.attn_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, Hq, Hkv, Lq,
+                            Lk, d, scale, ctypes.byref(m), ns, ws.data_ptr(), ws.numel(), None)
+    assert st == 0
+    st, site = ta.device_error()
+    assert st == 0, f"device error {st} at site {site}"
+    ro, rl = oracle.attn_fwd(x["q"], x["k"], x["v"], scale, causal, window, global_head=gh, global_tail=gt,
+                             seqlens_q=lq, seqlens_k=lk)
+    check_o(to_f64(o), ro, "O")
+    check_lse(to_f64(lse), rl, "LSE")
+
+
 @pytest.mark.parametrize("split", [False, True])
 def test_fwd_decode_full_size(ta, split):
     """gqa_decode_32768 at full size (packed rows; with split=True the split-KV

@@ -208,6 +208,20 @@ def test_padded_batch_equals_separate_sequences():
         np.testing.assert_array_equal(l2, lse)
 
 
+def test_padded_batch_sequence_without_keys():
+    """A sequence with queries but no keys (seqlens_k = 0): every one of its
+    rows is fully masked, so O = 0 and LSE = -inf (no NaN); the other
+    sequences are unaffected."""
+    q, k, v = _rand(2, 2, 6, 4), _rand(2, 2, 9, 4), _rand(2, 2, 9, 4)
+    O, lse = oracle.attn_fwd(q, k, v, 0.5, 2, 0, seqlens_q=[6, 4], seqlens_k=[9, 0])
+    assert np.all(O[1] == 0.0) and np.all(np.isneginf(lse[1]))
+    O0, lse0 = oracle.attn_fwd(q[:1], k[:1], v[:1], 0.5, 2, 0)
+    np.testing.assert_array_equal(O[0], O0[0])
+    np.testing.assert_array_equal(lse[0], lse0[0])
+    dq, dk, dv = oracle.attn_bwd(q, k, v, _rand(2, 2, 6, 4), 0.5, 2, 0, seqlens_q=[6, 4], seqlens_k=[9, 0])
+    assert np.all(dq[1] == 0.0) and np.all(dk[1] == 0.0) and np.all(dv[1] == 0.0)
+
+
 def test_padded_batch_matches_torch_sdpa_key_padding_mask():
     """Per-sequence key lengths against torch SDPA with a key-padding mask built here."""
     B, H, L, d = 2, 2, 10, 4
