@@ -111,6 +111,9 @@ def test_fwd_split_default_is_in_range(ta):
     assert 1 <= d(8, 32, 8, 1, 32768, 128, 2, 0) <= 64
     assert d(2, 32, 32, 4096, 4096, 128, 1, 0) == 1     # a full grid does not
     assert d(1, 2, 2, 1, 100, 64, 2, 0) == 1            # a single key tile does not
+    # 16 queries per head over 32768 keys, G = 4: 32 packed units of 256 key tiles.  With 148 SMs (the
+    # default without a device) 9 slices (288 CTAs, two waves) give the least modelled time.
+    assert d(4, 32, 8, 16, 32768, 128, 2, 0) == 9
 
 
 def _split(ta, n_split=4, ws=P, wsb=1 << 20, **kw):

@@ -318,6 +318,26 @@ def test_block_sparse_matches_torch_sdpa(Lq, Lk, b, causal, w):
     assert np.all(O[0, :, ~rows] == 0.0)
 
 
+def test_block_sparse_with_global_keys_matches_torch_sdpa():
+    """Block-sparse mask and global keys together: the global keys are added on
+    top of the block-sparse (and causal) band, as they are on top of a window."""
+    Lq = Lk = 36
+    b, gh, gt = 6, 2, 3
+    q, k, v = _rand(1, 2, Lq, 5), _rand(1, 2, Lk, 5), _rand(1, 2, Lk, 5)
+    for causal in (False, True):
+        O, _ = oracle.attn_fwd(q, k, v, 0.4, causal, 0, global_head=gh, global_tail=gt, sparse_block=b)
+        i = torch.arange(Lq)[:, None]
+        j = torch.arange(Lk)[None, :]
+        band = _block_rule(Lq, Lk, b)
+        glob = ((j < gh) | (j >= Lk - gt)).expand(Lq, Lk)
+        if causal:
+            band = band & (j <= i)
+            glob = glob & (j <= i)
+        ref = torch.nn.functional.scaled_dot_product_attention(*(torch.from_numpy(x) for x in (q, k, v)),
+                                                               attn_mask=band | glob, scale=0.4)
+        np.testing.assert_allclose(O, ref.numpy(), atol=1e-12)
+
+
 def test_block_sparse_pages_example_counts():
     """The page's example (seq_len 1024, block 64): interior query blocks see
     3b - 1 keys, the first block 2b - 1, the last 2b; the total follows."""
