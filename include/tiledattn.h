@@ -268,8 +268,10 @@ ATTN_API int attn_bwd_noalloc(const void* q, const void* k, const void* v, const
  * The attention step with HOST buffers: copies Q, K, V (and dO) in, runs
  * attn_fwd (and attn_bwd), and copies O and LSE (and dQ, dK, dV) out, all
  * ordered on `stream` like every other call (asynchronous; synchronise the
- * stream before reading the host outputs).  The pages' interface works on
- * tensors already on the device; this is the same computation for a caller
+ * stream before reading the host outputs).  The computation is that of
+ * attn_fwd / attn_bwd (the scaled-dot-product attention call of
+ * "缩放定律与高效注意力" §3.5, and its recompute backward of §3.3); the pages
+ * call it on tensors already on the device, this entry point serves a caller
  * whose data lives in host memory.
  *
  *  - q, k, v, dO, o, lse, dq, dk, dv: HOST pointers, same shapes and layouts
