@@ -45,6 +45,10 @@
  *    attn_get_device_error() reports; its outputs are then undefined.
  *  - Empty problems (B, Hq, Lq = 0) are valid and launch nothing.  Lk = 0 is
  *    valid: every row sees no key.
+ *  - The library looks up the device addresses of its own device-side objects
+ *    (the error word, the attn_bwd_noalloc scratch array) once per device and
+ *    keeps them: do not use it on a device across cudaDeviceReset(), which
+ *    may move them.
  */
 #ifndef TILEDATTN_H
 #define TILEDATTN_H
@@ -291,8 +295,10 @@ ATTN_API int attn_bwd_noalloc(const void* q, const void* k, const void* v, const
  *    on the whole problem.
  *  - Errors: shape, mask and scale checks as attn_fwd (before anything is
  *    enqueued); NULL host pointers or a short / misaligned dev_buf:
- *    ATTN_ERR_INVALID_ARG; a failing CUDA call: ATTN_ERR_CUDA (work already
- *    enqueued still runs; outputs are then undefined).
+ *    ATTN_ERR_INVALID_ARG; a failing CUDA call: ATTN_ERR_CUDA.  Before an
+ *    error is returned after chunks were already queued, the call waits for
+ *    that work to finish, so no copy still reads or writes the caller's host
+ *    buffers or dev_buf once it has returned; the outputs are then undefined.
  */
 ATTN_API size_t attn_step_host_buffer_size(int B, int Hq, int Hkv, int Lq, int Lk, int d, int with_backward);
 ATTN_API int attn_step_host(const void* q, const void* k, const void* v, const void* dO, void* o, float* lse,
@@ -325,6 +331,16 @@ ATTN_API int attn_get_device_error(void* stream, int* site);
  * status.  No counterpart on the pages: it exists to test failure handling.
  */
 ATTN_API int attn_selftest_wait_timeout(int64_t limit_ns, void* stream);
+
+/*
+ * Self-test of attn_step_host's error path: the next attn_step_host call (on
+ * any thread) behaves as if the copy in of chunk `chunk` had failed, after
+ * the earlier chunks' copies and kernels were queued, and returns
+ * ATTN_ERR_CUDA.  chunk = -1 cancels; chunk < -1 is ATTN_ERR_INVALID_ARG.
+ * The failure is made on the host; nothing faults on the GPU.  No counterpart
+ * on the pages: it exists to test failure handling.
+ */
+ATTN_API int attn_selftest_step_host_fail_at(int chunk);
 
 #ifdef __cplusplus
 }

@@ -53,3 +53,18 @@ def test_short_region_takes_the_first_sample_after_its_start():
 
 def test_no_samples_gives_none():
     assert _sampler([], time.time(), time.time() + 1).stop() is None
+
+
+def test_roofline_peak_matches_the_timed_region():
+    import bench
+    burst, sustained = 1674.3, 1409.4
+    # A short region at full clock: the burst GEMM figure.
+    p, kind = bench.roofline_peak(burst, sustained, 24.0, {"reasons": [], "sm_mhz": 1965.0})
+    assert p == burst and kind.startswith("burst")
+    # A short region that saw the power cap is still a burst measurement.
+    assert bench.roofline_peak(burst, sustained, 300.0, {"reasons": ["sw_power_cap"]})[0] == burst
+    # Only a region of a second or more under the power cap pairs with the sustained figure.
+    p, kind = bench.roofline_peak(burst, sustained, 1300.0, {"reasons": ["sw_power_cap"]})
+    assert p == sustained and kind.startswith("sustained")
+    assert bench.roofline_peak(burst, sustained, 1300.0, {"reasons": []})[0] == burst
+    assert bench.roofline_peak(burst, sustained, 1300.0, None)[0] == burst

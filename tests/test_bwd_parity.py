@@ -168,17 +168,45 @@ def test_bwd_gqa_window_2048(ta):
 
 def test_bwd_full_size_sampled_heads(ta):
     """The fwd+bwd workload at full size (benchmark launch configuration);
-    whole K/V heads (independent units) compared against the oracle."""
+    whole K/V heads (independent units) from both sequences compared against
+    the oracle, row by row."""
     w = WORKLOADS["mha_causal_fwdbwd"]
     x = make_inputs(w)
     dq, dk, dv = run_fwd_bwd(ta, x, w.causal, w.window, w.scale)
-    heads = [(0, 0), (1, 31)]
+    heads = [(0, 0), (0, 17), (1, 5), (1, 31)]
     rq, rk, rv = oracle.attn_bwd(x["q"], x["k"], x["v"], x["do"], w.scale, w.causal, w.window, heads=heads)
     for b, h in heads:
         check_grad(dq[b, h], rq[b, h], f"dQ[{b},{h}]")
         check_grad(dk[b, h], rk[b, h], f"dK[{b},{h}]")
         check_grad(dv[b, h], rv[b, h], f"dV[{b},{h}]")
     assert np.all(np.isfinite(dq)) and np.all(np.isfinite(dk)) and np.all(np.isfinite(dv))
+
+
+@pytest.mark.parametrize("name,heads", [("gqa_causal_8192", [(0, 0), (3, 7)]), ("gqa_window_32768", [(0, 5)])])
+def test_bwd_gqa_full_size_sampled_heads(ta, name, heads):
+    """Backward of the full-size GQA workloads (causal with Q x 2, and the
+    32768-token causal window of 4096) with a dO drawn after Q, K, V: whole
+    K/V heads, i.e. the kv head's dK/dV summed over its 4 query heads and
+    those heads' dQ, against the oracle row by row."""
+    import dataclasses
+    import torch
+    w = dataclasses.replace(WORKLOADS[name], backward=True)
+    x = make_inputs(w)
+    q, k, v, do = (to_dev(x[n]) for n in ("q", "k", "v", "do"))
+    o, lse = ta.attention(q, k, v, w.causal, w.window, w.scale)
+    dq, dk, dv = ta.attention_backward(q, k, v, o, lse, do, w.causal, w.window, w.scale)
+    st, site = ta.device_error()
+    assert st == 0, f"device error {st} at site {site}"
+    for t in (dq, dk, dv):
+        assert bool(torch.isfinite(t.float()).all())
+    del q, k, v, o, lse, do
+    G = w.Hq // w.Hkv
+    rq, rk, rv = oracle.attn_bwd(x["q"], x["k"], x["v"], x["do"], w.scale, w.causal, w.window, heads=heads)
+    for b, g in heads:
+        check_grad(to_f64(dk[b, g]), rk[b, g], f"dK[{b},{g}]")
+        check_grad(to_f64(dv[b, g]), rv[b, g], f"dV[{b},{g}]")
+        for h in range(g * G, (g + 1) * G):
+            check_grad(to_f64(dq[b, h]), rq[b, h], f"dQ[{b},{h}]")
 
 
 def test_autograd_wrapper(ta):

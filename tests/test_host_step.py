@@ -13,7 +13,7 @@ import pytest
 
 import oracle
 from synth import make_shape_inputs
-from tests._util import check_lse, check_o, rel_fro, to_dev, to_f64
+from tests._util import check_grad, check_lse, check_o, rel_fro, row_errors, to_dev, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -82,6 +82,7 @@ def test_step_host_matches_device_path(ta, B, Hq, Hkv, Lq, Lk, d, causal, window
     assert torch.equal(g["dk"], dk.cpu()), "dK differs from attn_bwd"
     assert torch.equal(g["dv"], dv.cpu()), "dV differs from attn_bwd"
     assert rel_fro(to_f64(g["dq"]), to_f64(dq)) <= 1e-3, "dQ differs from attn_bwd"
+    assert np.max(row_errors(to_f64(g["dq"]), to_f64(dq)), initial=0.0) <= 1e-2, "a dQ row differs from attn_bwd"
 
 
 def test_step_host_forward_only_against_oracle(ta):
@@ -101,4 +102,35 @@ def test_step_host_backward_against_oracle(ta):
     _, _, g = _run_host(ta, x, causal, window, scale, True, True)
     rdq, rdk, rdv = oracle.attn_bwd(x["q"], x["k"], x["v"], x["do"], scale, causal, window)
     for name, got, ref in (("dQ", g["dq"], rdq), ("dK", g["dk"], rdk), ("dV", g["dv"], rdv)):
-        assert rel_fro(to_f64(got), ref) <= 2e-2, f"{name} relative Frobenius error"
+        check_grad(to_f64(got), ref, name)
+
+
+def test_step_host_error_after_queued_chunks_leaves_buffers_quiet(ta):
+    """A failure at a late chunk (made on the host by the self-test hook) is
+    returned only after the chunks already queued have finished: host outputs
+    overwritten right after the call are not touched by a late copy."""
+    import torch
+    B, Hq, Hkv, Lq, Lk, d = 2, 8, 8, 512, 512, 128  # 16 kv groups -> 8 chunks
+    x = make_shape_inputs(B, Hq, Hkv, Lq, Lk, d, seed=99, with_do=True)
+    q, k, v, do = (_host(x[n], True) for n in ("q", "k", "v", "do"))
+    pin = lambda t: torch.zeros(t.shape, dtype=t.dtype, pin_memory=True)
+    o, dq, dk, dv = pin(q), pin(q), pin(k), pin(v)
+    lse = torch.zeros((B, Hq, Lq), dtype=torch.float32, pin_memory=True)
+    buf = torch.empty(ta.step_host_buffer_size(B, Hq, Hkv, Lq, Lk, d, True), dtype=torch.uint8, device="cuda")
+    assert ta.lib.attn_selftest_step_host_fail_at(6) == ta.ATTN_OK
+    with pytest.raises(ta.AttnError) as ei:
+        ta.step_host(q, k, v, o, lse, buf, do=do, dq=dq, dk=dk, dv=dv, causal=True, scale=d ** -0.5)
+    assert ei.value.status == ta.ATTN_ERR_CUDA and "self-test" in str(ei.value)
+    marker = torch.tensor(-7.0, dtype=torch.bfloat16)
+    for t in (o, dq, dk, dv):
+        t.fill_(marker)
+    lse.fill_(-7.0)
+    torch.cuda.synchronize()
+    for t in (o, dq, dk, dv):
+        assert bool((t == marker).all())
+    assert bool((lse == -7.0).all())
+    # The hook fires once: the next call runs normally.
+    ta.step_host(q, k, v, o, lse, buf, do=do, dq=dq, dk=dk, dv=dv, causal=True, scale=d ** -0.5)
+    torch.cuda.synchronize()
+    assert ta.device_error()[0] == ta.ATTN_OK
+    assert not bool((o == marker).any())

@@ -42,7 +42,7 @@ class AttnMask(ctypes.Structure):
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"{LIB_PATH} is not built; run `python -m tiled_exact_attention_02_b200.build`")
+            f"{LIB_PATH} is not built; run `python tiled_exact_attention_02_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     lib.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, vp]
@@ -86,6 +86,8 @@ def _load() -> ctypes.CDLL:
     lib.attn_get_device_error.restype = i
     lib.attn_selftest_wait_timeout.argtypes = [ctypes.c_int64, vp]
     lib.attn_selftest_wait_timeout.restype = i
+    lib.attn_selftest_step_host_fail_at.argtypes = [i]
+    lib.attn_selftest_step_host_fail_at.restype = i
     return lib
 
 

@@ -1,6 +1,8 @@
 """Build the CUDA library libtiledattn.so in-tree (sm_100a only).
 
-Usage: python -m tiled_exact_attention_02_b200.build  (or build() from Python).
+Usage: python tiled_exact_attention_02_b200/build.py [--force] [-v]  (or
+__graft_entry__.build()).  Run it as a file: importing the package loads
+the library this script builds.
 """
 
 import os

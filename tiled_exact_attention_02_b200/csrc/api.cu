@@ -20,7 +20,6 @@ __device__ int g_dev_err;
 
 namespace {
 
-constexpr int kMaxDevices = 64;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s without progress
 
 std::mutex g_mu;

@@ -762,11 +762,14 @@ cudaError_t launch_bwd_post(const float* dq_acc, void* dq, int BH, int Lq, int l
 template <int D>
 static cudaError_t launch_bwd_d(const BwdParams& P, cudaStream_t stream) {
   constexpr int smem = bwd::Cfg<D>::SMEM;
-  cudaError_t e = cudaFuncSetAttribute(bwd::attn_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
-  // setmaxnreg redistributes the registers the block was launched with: the
-  // split above is only valid at exactly LAUNCH_REGS per thread.
-  e = check_launch_regs(reinterpret_cast<const void*>(bwd::attn_bwd_kernel<D>), bwd::LAUNCH_REGS);
+  static std::atomic<unsigned char> ready[kMaxDevices];
+  const cudaError_t e = once_per_device(ready, [] {
+    cudaError_t r = cudaFuncSetAttribute(bwd::attn_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (r != cudaSuccess) return r;
+    // setmaxnreg redistributes the registers the block was launched with: the
+    // split above is only valid at exactly LAUNCH_REGS per thread.
+    return check_launch_regs(reinterpret_cast<const void*>(bwd::attn_bwd_kernel<D>), bwd::LAUNCH_REGS);
+  });
   if (e != cudaSuccess) return e;
   bwd::attn_bwd_kernel<D><<<P.n_units, bwd::THREADS, smem, stream>>>(P);
   return cudaGetLastError();

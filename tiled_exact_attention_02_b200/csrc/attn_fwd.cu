@@ -857,8 +857,10 @@ void fwd_plan(const Problem& p, int* n_units, int* pair_heads, int* packed, int*
 template <int D, bool W, bool A>
 static cudaError_t launch_fwd_d(const FwdParams& P, cudaStream_t stream) {
   constexpr int smem = fwd::Cfg<D>::SMEM;
-  cudaError_t e =
-      cudaFuncSetAttribute(fwd::attn_fwd_kernel<D, W, A>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  static std::atomic<unsigned char> ready[kMaxDevices];
+  cudaError_t e = once_per_device(ready, [] {
+    return cudaFuncSetAttribute(fwd::attn_fwd_kernel<D, W, A>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  });
   if (e != cudaSuccess) return e;
   fwd::attn_fwd_kernel<D, W, A><<<P.n_units * imax(1, P.n_split), fwd::THREADS, smem, stream>>>(P);
   return cudaGetLastError();

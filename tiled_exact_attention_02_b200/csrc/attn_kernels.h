@@ -2,6 +2,7 @@
 #pragma once
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <atomic>
 #include <cstdint>
 #include "attn_common.cuh"
 
@@ -54,6 +55,23 @@ inline cudaError_t check_launch_regs(const void* kernel, int expected) {
   cudaError_t e = cudaFuncGetAttributes(&a, kernel);
   if (e != cudaSuccess) return e;
   return a.numRegs == expected ? cudaSuccess : cudaErrorInvalidConfiguration;
+}
+
+// Per-device one-time set-up of a kernel (its dynamic shared-memory limit, the
+// register-count check): `fn` runs until it first succeeds on the current
+// device, later launches on that device skip it.  Concurrent first calls may
+// both run it, which is harmless.
+constexpr int kMaxDevices = 64;
+template <typename Fn>
+inline cudaError_t once_per_device(std::atomic<unsigned char> (&done)[kMaxDevices], Fn&& fn) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return fn();
+  if (done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  e = fn();
+  if (e == cudaSuccess) done[dev].store(1, std::memory_order_release);
+  return e;
 }
 
 // Query rows per backward step for head dimension d.

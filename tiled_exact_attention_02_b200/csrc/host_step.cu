@@ -15,6 +15,7 @@
 // every other entry point.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 #include <vector>
 
@@ -27,9 +28,18 @@ constexpr int kTargetChunks = 8;
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
+// Chunk index at which the next attn_step_host call pretends that its copy
+// in failed (-1: none), set by attn_selftest_step_host_fail_at; it exercises
+// the error path after earlier chunks are already queued, without a GPU fault.
+std::atomic<int> g_fail_at{-1};
+
 // Byte offsets of every staged tensor inside the device buffer.  LSE is
 // staged per chunk (a chunk's rows start at any multiple of 4 bytes inside
-// the whole LSE, and the kernels want 16-byte aligned pointers).
+// the whole LSE, and the kernels want 16-byte aligned pointers).  The backward
+// workspace `ws` (D and the fp32 dQ accumulator) is one region shared by all
+// chunks: that is only safe because every chunk's kernels run in order on the
+// single compute stream, so chunk c's attn_bwd starts after chunk c-1's has
+// finished with it.
 struct Staging {
   size_t q, k, v, dO, o, lse, lse_chunk, dq, dk, dv, ws, ws_bytes, total;
 };
@@ -77,10 +87,19 @@ Staging staging(int B, int Hq, int Hkv, int Lq, int Lk, int d, bool bwd) {
 
 // Streams and events of one call; released on every return path.  A stream
 // or event destroyed with work still pending is released once that work ends.
+// If the call fails after work was queued (`quiesce` still set), the
+// destructor first waits for the three internal streams, so that no copy of
+// an earlier chunk still reads or writes the caller's buffers when the error
+// is returned.
 struct CallResources {
   cudaStream_t s_in = nullptr, s_comp = nullptr, s_out = nullptr;
   std::vector<cudaEvent_t> events;
+  bool quiesce = false;
   ~CallResources() {
+    if (quiesce) {
+      for (cudaStream_t s : {s_in, s_comp, s_out})
+        if (s) cudaStreamSynchronize(s);
+    }
     for (cudaEvent_t e : events) cudaEventDestroy(e);
     if (s_in) cudaStreamDestroy(s_in);
     if (s_comp) cudaStreamDestroy(s_comp);
@@ -130,6 +149,9 @@ int attn_step_host(const void* q, const void* k, const void* v, const void* dO, 
       (e = cudaStreamWaitEvent(R.s_out, start, 0)) != cudaSuccess)
     return tea::record_cuda_error("attn_step_host start", e);
 
+  // From here on, an error return waits for what was queued (see CallResources).
+  R.quiesce = true;
+  const int fail_at = g_fail_at.exchange(-1);
   int chunk = 0;
   for (int b = 0; b < B; b++) {
     for (int kv0 = 0; kv0 < Hkv; kv0 += kc, chunk++) {
@@ -146,6 +168,7 @@ int attn_step_host(const void* q, const void* k, const void* v, const void* dO, 
         return cudaMemcpyAsync(static_cast<uint8_t*>(dst) + off, base + src + off, bytes, cudaMemcpyDeviceToHost,
                                R.s_out);
       };
+      if (chunk == fail_at) return tea::record_cuda_error("attn_step_host copy in (self-test)", cudaErrorUnknown);
       if ((e = in(S.q, q, qe, qb)) != cudaSuccess ||
           (kb > 0 && ((e = in(S.k, k, ke, kb)) != cudaSuccess || (e = in(S.v, v, ke, kb)) != cudaSuccess)) ||
           (bwd && (e = in(S.dO, dO, qe, qb)) != cudaSuccess))
@@ -184,6 +207,13 @@ int attn_step_host(const void* q, const void* k, const void* v, const void* dO, 
   if ((e = R.event(&end)) != cudaSuccess || (e = cudaEventRecord(end, R.s_out)) != cudaSuccess ||
       (e = cudaStreamWaitEvent(caller, end, 0)) != cudaSuccess)
     return tea::record_cuda_error("attn_step_host end", e);
+  R.quiesce = false;  // the caller's stream now orders everything after the call's work
+  return ATTN_OK;
+}
+
+int attn_selftest_step_host_fail_at(int chunk) {
+  if (chunk < -1) return ATTN_ERR_INVALID_ARG;
+  g_fail_at.store(chunk);
   return ATTN_OK;
 }
 
