@@ -269,6 +269,58 @@ ATTN_API int attn_bwd_noalloc(const void* q, const void* k, const void* v, const
                               int d, float scale, int causal, int window, void* stream);
 
 /*
+ * Building blocks of ring (context-parallel) attention ("缩放定律与高效注意力"
+ * §5.1, the table of three directions: for longer contexts, RingAttention
+ * and LongFlashAttention run sequence parallelism on top of FlashAttention).
+ * The sequence is cut into blocks held by different devices; each device
+ * computes its queries against one K/V block at a time while the blocks are
+ * passed around a ring, and the partial results are merged exactly with the
+ * online-softmax rescale of "高效注意力：FlashAttention 与线性注意力", 原理与
+ * 机制 (running max / sum, rescaled by e^{m_old - m_new}), applied to whole
+ * key blocks through their logsumexp.  The exchange itself is the caller's
+ * (the Python package drives it over torch.distributed); these calls are the
+ * per-block compute.
+ *
+ * attn_fwd_accumulate: attention of q against the key block k, v (masks as
+ * attn_fwd, relative to the two blocks' own row indices: causal = 1 is the
+ * diagonal block of equal-length blocks, causal = 0 a block that lies wholly
+ * before the queries), merged into running accumulators:
+ *  o_acc    fp32 [B, Hq, Lq, d]  in/out: O over the key blocks so far,
+ *                                normalised by its own softmax sum
+ *  lse_acc  fp32 [B, Hq, Lq]     in/out: their natural-log logsumexp
+ *                                (-inf: no visible key yet)
+ *  init     1: the accumulators are written, not read (first block of these
+ *           rows); 0: merged: with M = max(LSE_a, LSE_b), w = exp(LSE - M),
+ *           O = (w_a O_a + w_b O_b) / (w_a + w_b), LSE = M + log(w_a + w_b).
+ * Other arguments, layouts and errors as attn_fwd.  Calls on the same
+ * accumulators must be ordered (one stream).
+ *
+ * attn_fwd_accumulate_finalize: o = bf16(o_acc) (round to nearest even),
+ * lse = lse_acc; o bf16 [B, Hq, Lq, d], lse fp32 [B, Hq, Lq].
+ *
+ * attn_bwd_accumulate: the backward of one key block with the FINAL (merged)
+ * lse of the queries and the workspace of attn_bwd_preprocess (D from the
+ * final O, and the fp32 dQ accumulator, to which this block's dQ is added;
+ * attn_bwd_finalize turns it into dQ after the last block).  This block's
+ * dK (scaled) and dV are added into fp32 accumulators dk_acc, dv_acc
+ * [B, Hkv, Lk, d] (init = 1: stored instead of added).  Other arguments as
+ * attn_bwd_main.
+ *
+ * attn_accumulator_to_bf16: out[i] = bf16(acc[i]) for n elements (dK / dV
+ * accumulators after the last block).  16-byte aligned pointers.
+ */
+ATTN_API int attn_fwd_accumulate(const void* q, const void* k, const void* v, float* o_acc, float* lse_acc, int B,
+                                 int Hq, int Hkv, int Lq, int Lk, int d, float scale, int causal, int window, int init,
+                                 void* stream);
+ATTN_API int attn_fwd_accumulate_finalize(const float* o_acc, const float* lse_acc, void* o, float* lse, int B, int Hq,
+                                          int Lq, int d, void* stream);
+ATTN_API int attn_bwd_accumulate(const void* q, const void* k, const void* v, const float* lse, const void* dO,
+                                 float* dk_acc, float* dv_acc, int B, int Hq, int Hkv, int Lq, int Lk, int d,
+                                 float scale, int causal, int window, int init, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+ATTN_API int attn_accumulator_to_bf16(const float* acc, void* out, size_t n, void* stream);
+
+/*
  * The attention step with HOST buffers: copies Q, K, V (and dO) in, runs
  * attn_fwd (and attn_bwd), and copies O and LSE (and dQ, dK, dV) out, all
  * ordered on `stream` like every other call (asynchronous; synchronise the

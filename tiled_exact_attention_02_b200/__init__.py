@@ -86,6 +86,14 @@ def _load() -> ctypes.CDLL:
     lib.attn_get_device_error.restype = i
     lib.attn_selftest_wait_timeout.argtypes = [ctypes.c_int64, vp]
     lib.attn_selftest_wait_timeout.restype = i
+    lib.attn_fwd_accumulate.argtypes = [vp] * 5 + [i] * 6 + [f, i, i, i, vp]
+    lib.attn_fwd_accumulate.restype = i
+    lib.attn_fwd_accumulate_finalize.argtypes = [vp] * 4 + [i] * 4 + [vp]
+    lib.attn_fwd_accumulate_finalize.restype = i
+    lib.attn_bwd_accumulate.argtypes = [vp] * 7 + [i] * 6 + [f, i, i, i, vp, sz, vp]
+    lib.attn_bwd_accumulate.restype = i
+    lib.attn_accumulator_to_bf16.argtypes = [vp, vp, sz, vp]
+    lib.attn_accumulator_to_bf16.restype = i
     lib.attn_selftest_step_host_fail_at.argtypes = [i]
     lib.attn_selftest_step_host_fail_at.restype = i
     return lib

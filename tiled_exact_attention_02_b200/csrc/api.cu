@@ -150,13 +150,22 @@ const char* attn_status_string(int status) {
 // Forward for every entry point: lens_q / lens_k optional per-sequence
 // lengths (device int32 [B]); n_split > 1 cuts each unit's key range into
 // slices written to `workspace` and merged.
+// acc_o != NULL: accumulate mode (attn_fwd_accumulate): the result is merged
+// into the fp32 accumulators acc_o / acc_lse (acc_init: written into them)
+// and o / lse are not used.
 static int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, const int* lens_q,
                     const int* lens_k, int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale, int causal,
-                    int window, int gh, int gt, int sb, int n_split, void* workspace, void* stream) {
+                    int window, int gh, int gt, int sb, int n_split, void* workspace, void* stream,
+                    float* acc_o = nullptr, float* acc_lse = nullptr, int acc_init = 0) {
   int st = check_shape(B, Hq, Hkv, Lq, Lk, d, scale, causal, window);
   if (st != ATTN_OK) return st;
   if (gh < 0 || gt < 0 || sb < 0 || sb > (1 << 28)) return ATTN_ERR_INVALID_ARG;
   if (B == 0 || Hq == 0 || Lq == 0) return ATTN_OK;
+  if (acc_o) {
+    if (!acc_lse || !aligned16(acc_o) || !aligned16(acc_lse) || n_split != 1) return ATTN_ERR_INVALID_ARG;
+    o = acc_o;  // placeholders for the checks below; the kernel writes only the accumulators
+    lse = acc_lse;
+  }
   if (!q || !o || !lse || !aligned16(q) || !aligned16(o) || !aligned16(lse)) return ATTN_ERR_INVALID_ARG;
   if (Lk > 0 && (!k || !v || !aligned16(k) || !aligned16(v))) return ATTN_ERR_INVALID_ARG;
   if ((lens_q && (reinterpret_cast<uintptr_t>(lens_q) & 3u)) || (lens_k && (reinterpret_cast<uintptr_t>(lens_k) & 3u)))
@@ -185,6 +194,14 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, float*
   P.lse = lse;
   P.scale_log2 = scale * 1.4426950408889634f;
   P.n_split = n_split;
+  if (acc_o) {
+    P.acc_mode = 1;
+    P.acc_init = acc_init != 0;
+    P.part_o = acc_o;
+    P.part_lse = acc_lse;
+    P.o = nullptr;
+    P.lse = nullptr;
+  }
   if (n_split > 1) {
     const size_t rows = (size_t)B * Hq * Lq;
     P.part_o = static_cast<float*>(workspace);
@@ -300,19 +317,29 @@ int attn_bwd_preprocess(const void* o, const void* dO, int B, int Hq, int Lq, in
   return e == cudaSuccess ? ATTN_OK : cuda_fail("attn_bwd_preprocess launch", e);
 }
 
+// dk_acc != NULL: accumulate mode (attn_bwd_accumulate): dK and dV are added
+// into the fp32 accumulators dk_acc / dv_acc (dkv_init: stored into them),
+// and dk / dv are not used.
 static int bwd_main_impl(const void* q, const void* k, const void* v, const float* lse, const void* dO, void* dk,
                          void* dv, const int* lens_q, const int* lens_k, int B, int Hq, int Hkv, int Lq, int Lk, int d,
                          float scale, int causal, int window, int gh, int gt, int sb, void* workspace,
-                         size_t workspace_bytes, void* stream) {
+                         size_t workspace_bytes, void* stream, float* dk_acc = nullptr, float* dv_acc = nullptr,
+                         int dkv_init = 0) {
   int st = check_shape(B, Hq, Hkv, Lq, Lk, d, scale, causal, window);
   if (st == ATTN_OK && (gh < 0 || gt < 0 || sb < 0 || sb > (1 << 28))) st = ATTN_ERR_INVALID_ARG;
   if (st != ATTN_OK) return st;
   if (B == 0 || Hq == 0 || Lk == 0) return ATTN_OK;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dk_acc) {
+    if (!dv_acc || !aligned16(dk_acc) || !aligned16(dv_acc)) return ATTN_ERR_INVALID_ARG;
+    dk = dk_acc;  // placeholders for the checks below; the kernel writes only the accumulators
+    dv = dv_acc;
+  }
   if (!k || !v || !dk || !dv || !aligned16(k) || !aligned16(v) || !aligned16(dk) || !aligned16(dv))
     return ATTN_ERR_INVALID_ARG;
-  if (Lq == 0) {  // no query: dK = dV = 0
-    const size_t kv_bytes = (size_t)B * Hkv * Lk * d * 2;
+  if (Lq == 0) {  // no query: dK = dV = 0 (an accumulator is only cleared when initialised here)
+    if (dk_acc && !dkv_init) return ATTN_OK;
+    const size_t kv_bytes = (size_t)B * Hkv * Lk * d * (dk_acc ? 4 : 2);
     cudaError_t e = cudaMemsetAsync(dk, 0, kv_bytes, s);
     if (e == cudaSuccess) e = cudaMemsetAsync(dv, 0, kv_bytes, s);
     return e == cudaSuccess ? ATTN_OK : cuda_fail("cudaMemsetAsync dK/dV", e);
@@ -355,6 +382,11 @@ static int bwd_main_impl(const void* q, const void* k, const void* v, const floa
   }
   P.dk = dk;
   P.dv = dv;
+  if (dk_acc) {
+    P.dk_acc = dk_acc;
+    P.dv_acc = dv_acc;
+    P.dkv_init = dkv_init != 0;
+  }
   P.scale = scale;
   P.scale_log2 = scale * 1.4426950408889634f;
   P.n_units = B * Hkv * ((Lk + 127) / 128);
@@ -434,6 +466,50 @@ int attn_bwd_varlen(const void* q, const void* k, const void* v, const void* o, 
                     size_t workspace_bytes, void* stream) {
   return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, seqlens_q, seqlens_k, B, Hq, Hkv, Lq, Lk, d, scale, causal, window,
                   0, 0, 0, workspace, workspace_bytes, stream);
+}
+
+// ------------------------------------------------------------------ accumulate (ring attention)
+int attn_fwd_accumulate(const void* q, const void* k, const void* v, float* o_acc, float* lse_acc, int B, int Hq,
+                        int Hkv, int Lq, int Lk, int d, float scale, int causal, int window, int init, void* stream) {
+  if (!o_acc || !lse_acc) return ATTN_ERR_INVALID_ARG;
+  return fwd_impl(q, k, v, nullptr, nullptr, nullptr, nullptr, B, Hq, Hkv, Lq, Lk, d, scale, causal, window, 0, 0, 0,
+                  1, nullptr, stream, o_acc, lse_acc, init);
+}
+
+int attn_fwd_accumulate_finalize(const float* o_acc, const float* lse_acc, void* o, float* lse, int B, int Hq, int Lq,
+                                 int d, void* stream) {
+  const int st = check_shape(B, Hq, Hq > 0 ? 1 : 0, Lq, 1, d, 1.f, 0, 0);
+  if (st != ATTN_OK) return st;
+  if (B == 0 || Hq == 0 || Lq == 0) return ATTN_OK;
+  if (!o_acc || !lse_acc || !o || !lse || !aligned16(o_acc) || !aligned16(lse_acc) || !aligned16(o) ||
+      !aligned16(lse))
+    return ATTN_ERR_INVALID_ARG;
+  FwdParams P;
+  memset(&P, 0, sizeof(P));
+  P.prob = Problem{B, Hq, 1, Lq, 1, d, 0, 0, 1.f};
+  P.part_o = const_cast<float*>(o_acc);
+  P.part_lse = const_cast<float*>(lse_acc);
+  P.o = o;
+  P.lse = lse;
+  P.n_split = 1;  // one "slice": O = the accumulator rounded to bf16, LSE copied
+  const cudaError_t e = launch_fwd_merge(P, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ATTN_OK : cuda_fail("attn_fwd_accumulate_finalize launch", e);
+}
+
+int attn_bwd_accumulate(const void* q, const void* k, const void* v, const float* lse, const void* dO, float* dk_acc,
+                        float* dv_acc, int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale, int causal,
+                        int window, int init, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!dk_acc || !dv_acc) return ATTN_ERR_INVALID_ARG;
+  return bwd_main_impl(q, k, v, lse, dO, nullptr, nullptr, nullptr, nullptr, B, Hq, Hkv, Lq, Lk, d, scale, causal,
+                       window, 0, 0, 0, workspace, workspace_bytes, stream, dk_acc, dv_acc, init);
+}
+
+int attn_accumulator_to_bf16(const float* acc, void* out, size_t n, void* stream) {
+  if (n == 0) return ATTN_OK;
+  if (!acc || !out || !aligned16(acc) || !aligned16(out)) return ATTN_ERR_INVALID_ARG;
+  if (n > ((size_t)1 << 40)) return ATTN_ERR_UNSUPPORTED;
+  const cudaError_t e = launch_f32_to_bf16(acc, out, n, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ATTN_OK : cuda_fail("attn_accumulator_to_bf16 launch", e);
 }
 
 const char* attn_last_cuda_error(void) { return g_last_err; }

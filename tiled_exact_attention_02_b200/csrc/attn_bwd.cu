@@ -24,8 +24,9 @@
 // so that one thread per key turns a row of S^T into P^T and dS^T, and the
 // bf16 P^T and dS^T, written once to shared memory, serve both as the K-major
 // A operand of dV/dK and as the MN-major operand of dQ.
-// Warp roles (512 threads): warp 0 TMA, warps 1 and 2 MMA issuers, warps 4-7 and
-// 8-11 the per-key softmax gradient (each group takes half of a step's query
+// Warp roles (512 threads): warp 0 TMA, warps 1 and 2 MMA issuers, warp 3
+// forwards the landing of each Q/dO tile to the issuers, warps 4-7 and 8-11
+// the per-key softmax gradient (each group takes half of a step's query
 // columns), warps 12-15 the dQ drain.  Tensor memory at d = 128:
 // S^T | dP^T | dV | dK | dQ^T | P^T | dS^T = 512 columns.  Q/dO tiles stream
 // through a 3-stage ring.
@@ -83,8 +84,10 @@ struct Cfg {
 // Barriers.  The MMA issuer pays for every wait and commit with tensor-core
 // idle time (its issue queue is shallow), so each of its waits covers
 // everything the next MMA group needs:
-//   sq_ready[stage]  Q/dO of a step landed (TMA, 1 arrival + bytes) and the
-//                    previous step's S^T/dP^T were read out (8 gradient warps)
+//   q_land[stage]    Q/dO of a step landed (TMA bytes; 1 arrival by the producer)
+//   sq_ready[stage]  Q/dO of a step landed (1 arrival by the landing forwarder,
+//                    after q_land) and the previous step's S^T/dP^T were read
+//                    out (8 gradient warps)
 //   grad_ready[2]    P^T/dS^T of a step written (8 gradient warps) and the
 //                    previous step's dQ read out of TMEM (4 drain warps)
 //   sdp_full         S^T/dP^T of a step complete
@@ -93,7 +96,7 @@ struct Cfg {
 //   q_empty[stage]   the step's Q/dO stage may be reloaded
 struct Bars {
   uint64_t kv_full;
-  uint64_t sq_ready[4], q_empty[4];  // Q/dO ring (up to 4 stages)
+  uint64_t sq_ready[4], q_empty[4], q_land[4];  // Q/dO ring (up to 4 stages)
   uint64_t grad_ready[2];
   uint64_t sdp_full, step_done;
   uint64_t vec_full[2][2];  // [group][buffer]
@@ -102,6 +105,11 @@ struct Bars {
   uint64_t drain[2];
   uint32_t tmem_base;
   int abort_flag;
+};
+
+template <int D>
+struct BarsFit {
+  static_assert(sizeof(Bars) <= 256, "barrier block overflows its shared-memory slot");
 };
 
 struct Unit {
@@ -165,23 +173,36 @@ __device__ void producer(const BwdParams& P, const Unit& u, uint8_t* smem, Bars&
     if (!mbar_wait(&bars.q_empty[st], ((i / C::NQS) & 1) ^ 1, g, 1)) break;
     int h, q0;
     step_of<D>(u, i, h, q0);
-    mbar_arrive_expect_tx(&bars.sq_ready[st], 2 * C::Q_TILE);
+    mbar_arrive_expect_tx(&bars.q_land[st], 2 * C::Q_TILE);
     for (int pnl = 0; pnl < D / 64; pnl++) {
-      tma_load_3d(smem + C::OFF_Q + st * C::Q_TILE + pnl * C::Q_PANEL, &P.tm_q, &bars.sq_ready[st], pnl * 64, q0,
+      tma_load_3d(smem + C::OFF_Q + st * C::Q_TILE + pnl * C::Q_PANEL, &P.tm_q, &bars.q_land[st], pnl * 64, q0,
                   u.b * p.Hq + h);
-      tma_load_3d(smem + C::OFF_DO + st * C::Q_TILE + pnl * C::Q_PANEL, &P.tm_do, &bars.sq_ready[st], pnl * 64, q0,
+      tma_load_3d(smem + C::OFF_DO + st * C::Q_TILE + pnl * C::Q_PANEL, &P.tm_do, &bars.q_land[st], pnl * 64, q0,
                   u.b * p.Hq + h);
     }
     issued = i + 1;
   }
-  // Let every copy this warp started land before the CTA may exit.  K/V have
-  // their own barrier; the Q/dO copies share sq_ready with the gradient
-  // warps' arrivals, so after an abort give them a fixed 50 us to land.
+  // Let every copy this warp started land before the CTA may exit (also after
+  // an abort).  K/V have their own barrier.  A Q/dO load of step j is only
+  // issued once step j - NQS has finished with its stage, so only the last
+  // NQS loads can still be in flight, each the latest phase of its stage's
+  // q_land barrier.
   mbar_wait_ignore_abort(&bars.kv_full, 0, g);
-  if (*g.abort_flag && issued > 0) {
-    const uint64_t t0 = globaltimer_ns();
-    while (globaltimer_ns() - t0 < 50000) {
-    }
+  for (int j = imax(0, issued - C::NQS); j < issued; j++)
+    mbar_wait_ignore_abort(&bars.q_land[j % C::NQS], (j / C::NQS) & 1, g);
+}
+
+// Passes the landing of each step's Q/dO tiles (q_land) on to sq_ready, which
+// also collects the gradient warps' arrivals: the issuer of S^T/dP^T then
+// waits on one barrier per step, and the producer keeps a barrier that counts
+// only its own copies, for an exact drain after an abort.
+template <int D>
+__device__ void land_forwarder(const Unit& u, Bars& bars, const WaitGuard& g) {
+  using C = Cfg<D>;
+  for (int i = 0; i < u.n_steps; i++) {
+    const int st = i % C::NQS;
+    if (!mbar_wait(&bars.q_land[st], (i / C::NQS) & 1, g, 2)) return;
+    mbar_arrive(&bars.sq_ready[st]);
   }
 }
 
@@ -466,6 +487,32 @@ __device__ void grad_rows(const BwdParams& P, const Unit& u, uint8_t* smem, Bars
   uint4* out = reinterpret_cast<uint4*>(static_cast<uint16_t*>(grp ? P.dk : P.dv) + off);
   const float f = grp ? P.scale : 1.f;
   const uint32_t colx = grp ? C::T_DK : C::T_DV;
+  if (P.dk_acc) {
+    // Accumulate mode (ring attention): this key block's dK / dV added into
+    // fp32 accumulators; a key row belongs to one CTA, so no race.
+    float4* acc = reinterpret_cast<float4*>((grp ? P.dk_acc : P.dv_acc) + off);
+#pragma unroll
+    for (int q = 0; q < D / 32; q++) {
+      uint32_t o[32];
+      if (has) {
+        tmem_ld32p(tmem + lane_base + colx + 32 * q, o);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; e++) o[e] = 0u;
+      }
+      if (write) {
+#pragma unroll
+        for (int v = 0; v < 8; v++) {
+          float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (!P.dkv_init) a = acc[q * 8 + v];
+          acc[q * 8 + v] = make_float4(a.x + __uint_as_float(o[4 * v]) * f, a.y + __uint_as_float(o[4 * v + 1]) * f,
+                                       a.z + __uint_as_float(o[4 * v + 2]) * f, a.w + __uint_as_float(o[4 * v + 3]) * f);
+        }
+      }
+    }
+    return;
+  }
 #pragma unroll
   for (int q = 0; q < D / 32; q++) {
     uint32_t o[32];
@@ -586,6 +633,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kernel(const __grid_const
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   Bars& bars = *reinterpret_cast<Bars*>(smem + C::OFF_BAR);
+  (void)sizeof(BarsFit<D>);
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
   const Unit u = decode_unit<D>(P, blockIdx.x);
@@ -595,8 +643,9 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kernel(const __grid_const
     bars.abort_flag = 0;
     mbar_init(&bars.kv_full, 1);
     for (int s = 0; s < C::NQS; s++) {
-      mbar_init(&bars.sq_ready[s], 1 + 8);  // producer + 8 gradient warps
+      mbar_init(&bars.sq_ready[s], 1 + 8);  // landing forwarder + 8 gradient warps
       mbar_init(&bars.q_empty[s], 1);
+      mbar_init(&bars.q_land[s], 1);
     }
     for (int s = 0; s < 2; s++) {
       mbar_init(&bars.grad_ready[s], 8 + 4);  // 8 gradient warps + 4 drain warps
@@ -633,6 +682,8 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kernel(const __grid_const
       if (lane == 0) mma_issuer<D, 0>(P, u, smem, bars, tmem, g);
     } else if (warp == 2) {
       if (lane == 0) mma_issuer<D, 1>(P, u, smem, bars, tmem, g);
+    } else {
+      if (lane == 0) land_forwarder<D>(u, bars, g);
     }
   } else if (warp < 12) {
     regs_set<RG, LAUNCH_REGS>();
@@ -722,6 +773,24 @@ __global__ void __launch_bounds__(256) bwd_post_kernel(const float* __restrict__
   }
 }
 
+// out = bf16(acc), 8 elements (two float4 in, one uint4 out) per thread and
+// iteration; a tail of fewer than 8 elements is converted one by one.
+__global__ void __launch_bounds__(256) f32_to_bf16_kernel(const float* __restrict__ acc, uint16_t* __restrict__ out,
+                                                          int64_t n) {
+  const int64_t n8 = n / 8;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; x < n8; x += stride) {
+    const float4 a = reinterpret_cast<const float4*>(acc)[2 * x];
+    const float4 b = reinterpret_cast<const float4*>(acc)[2 * x + 1];
+    reinterpret_cast<uint4*>(out)[x] =
+        make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
+  }
+  if (blockIdx.x == 0 && threadIdx.x < n - n8 * 8) {
+    const int64_t i = n8 * 8 + threadIdx.x;
+    out[i] = (uint16_t)(pack_bf16x2(acc[i], 0.f) & 0xFFFFu);
+  }
+}
+
 }  // namespace bwd
 
 static int elementwise_grid(int64_t work_threads) {
@@ -756,6 +825,13 @@ cudaError_t launch_bwd_post(const float* dq_acc, void* dq, int BH, int Lq, int l
     bwd::bwd_post_kernel<128><<<grid, 256, 0, stream>>>(dq_acc, static_cast<uint16_t*>(dq), Lq, lq_pad, scale);
   else
     bwd::bwd_post_kernel<64><<<grid, 256, 0, stream>>>(dq_acc, static_cast<uint16_t*>(dq), Lq, lq_pad, scale);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_f32_to_bf16(const float* acc, void* out, size_t n, cudaStream_t stream) {
+  if (n == 0) return cudaSuccess;
+  const int grid = elementwise_grid((int64_t)(n / 8) > 0 ? (int64_t)(n / 8) : 1);
+  bwd::f32_to_bf16_kernel<<<grid, 256, 0, stream>>>(acc, static_cast<uint16_t*>(out), (int64_t)n);
   return cudaGetLastError();
 }
 

@@ -667,6 +667,38 @@ __device__ void softmax_slot(const FwdParams& P, const Unit& u, int s, uint8_t* 
       for (int e = 0; e < 16; e++) f[e] = fmaf(__uint_as_float(o[e]), sc_oth, f[e]);
     }
   };
+  if (P.acc_mode) {
+    // Running accumulators of earlier key blocks (ring attention): with the
+    // old (O_a, LSE_a) and this block's (O_b, LSE_b), both normalised by
+    // their own sums, M = max(LSE_a, LSE_b), w = exp(LSE - M):
+    //   O = (w_a O_a + w_b O_b) / (w_a + w_b),  LSE = M + log(w_a + w_b),
+    // the rescale of the online softmax applied to whole key blocks.  Each
+    // row belongs to one CTA, so the read-modify-write does not race.
+    float* accp = P.part_o + row_off * D;
+    const float l_old = (write && !P.acc_init) ? P.part_lse[row_off] : -INFINITY;
+    const float M = fmaxf(l_old, lse_row);
+    const float w_old = l_old == -INFINITY ? 0.f : expf(l_old - M);
+    const float w_new = lse_row == -INFINITY ? 0.f : expf(lse_row - M);
+    const float wsum = w_old + w_new;
+    const float c_old = wsum > 0.f ? w_old / wsum : 0.f, c_new = wsum > 0.f ? w_new / wsum : 0.f;
+#pragma unroll
+    for (int q = 0; q < D / 16; q++) {
+      float f[16];
+      load_o(q, f);
+      if (write) {
+        float4* a4 = reinterpret_cast<float4*>(accp + q * 16);
+#pragma unroll
+        for (int v = 0; v < 4; v++) {
+          float4 o4 = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (w_old > 0.f) o4 = a4[v];
+          a4[v] = make_float4(o4.x * c_old + f[4 * v] * c_new, o4.y * c_old + f[4 * v + 1] * c_new,
+                              o4.z * c_old + f[4 * v + 2] * c_new, o4.w * c_old + f[4 * v + 3] * c_new);
+        }
+      }
+    }
+    if (write) P.part_lse[row_off] = wsum > 0.f ? M + logf(wsum) : -INFINITY;
+    return;
+  }
   if (P.n_split > 1) {
     // One key-range slice of a split problem: fp32 O normalised by this
     // slice's own sum, and the slice's LSE; the merge kernel combines them.

@@ -23,6 +23,12 @@ struct FwdParams {
   int n_split;       // key-range slices per unit (1: the CTA writes O and LSE itself)
   float* part_o;     // n_split > 1: fp32 [n_split][B*Hq][Lq][d], O of each slice normalised by its own sum
   float* part_lse;   // n_split > 1: fp32 [n_split][B*Hq][Lq], natural-log LSE of each slice (-inf: empty)
+  // acc_mode (n_split == 1): part_o / part_lse are running fp32 accumulators
+  // [B*Hq][Lq][d] and [B*Hq][Lq] of earlier key blocks (O normalised by its own
+  // sum, natural-log LSE); the epilogue merges this launch's result into them
+  // (acc_init: overwrites them instead) and writes no bf16 O.
+  int acc_mode;
+  int acc_init;
   int* err;          // device error word
   uint64_t limit_ns; // bounded-wait limit
 };
@@ -40,6 +46,12 @@ struct BwdParams {
   CUtensorMap tm_dq;  // dq_acc as 2-D [B*Hq*d rows, Lq cols], box 32 x 128, 128-byte swizzle (d = 128)
   void* dk;           // bf16 [B, Hkv, Lk, d]
   void* dv;           // bf16 [B, Hkv, Lk, d]
+  // Accumulate mode (both non-null): dK (already scaled) and dV are added into
+  // these fp32 [B, Hkv, Lk, d] buffers instead of written to dk / dv
+  // (dkv_init: stored instead of added).
+  float* dk_acc;
+  float* dv_acc;
+  int dkv_init;
   float scale;
   float scale_log2;
   int n_units;        // CTAs: B * Hkv * key tiles
@@ -86,6 +98,8 @@ cudaError_t launch_bwd_pre(const void* o, const void* dO, float* dvec, float* dq
 cudaError_t launch_bwd(const BwdParams& P, cudaStream_t stream);
 cudaError_t launch_bwd_post(const float* dq_acc, void* dq, int BH, int Lq, int lq_pad, int d, float scale,
                             cudaStream_t stream);
+// out[i] = bf16(acc[i]) (round to nearest even), n elements.
+cudaError_t launch_f32_to_bf16(const float* acc, void* out, size_t n, cudaStream_t stream);
 
 // Number of CTAs of the forward grid and whether heads are paired.
 void fwd_plan(const Problem& p, int* n_units, int* pair_heads, int* packed, int* alternate);
