@@ -39,7 +39,7 @@ def check_lse(got, ref, what=""):
     assert not bad.any(), f"{what}: LSE error {np.max(np.abs(got[live]-ref[live])):.3e} at {np.argwhere(bad)[:3]}"
 
 
-ABS_FLOOR = 1e-4
+ABS_FLOOR = 1e-3
 
 
 def row_errors(got, ref, half_window: int = 64):
@@ -56,10 +56,12 @@ def row_errors(got, ref, half_window: int = 64):
     (dP - D) nearly cancels and a row of dQ or dK can be far smaller than its
     rounding error.  It is local because row norms drift along the sequence
     (under a causal mask the last keys' dK/dV rows are ~100x smaller than the
-    first ones').  An absolute floor of 1e-4 on the row norm covers rows that
-    are zero in exact arithmetic (a window of one key: P = 1 and dP_i = D_i, so
-    dS = 0 and the computed row is fp32 noise of ~1e-7); with N(0, 1) inputs
-    the gradient rows of interest are orders of magnitude larger."""
+    first ones').  An absolute floor of 1e-3 on the row norm covers rows that
+    are zero in exact arithmetic: with a window of one key, P = 1 and dP_i =
+    D_i, so dS = 0, but the two 128-term fp32 dot products behind dP_i and D_i
+    (values up to ~40, ulp ~4e-6) differ in their last bits, which leaves dQ
+    rows of ~1e-5.  With N(0, 1) inputs the gradient rows of interest are
+    1e-2 to 10 in norm."""
     g = np.asarray(got, dtype=np.float64)
     r = np.asarray(ref, dtype=np.float64)
     if r.ndim == 1:
