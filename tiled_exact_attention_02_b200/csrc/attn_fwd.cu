@@ -61,8 +61,24 @@ constexpr float EXP2_C4 = 0.009570102207362652f;  // 0x3c1ccbeb
 // One pair of columns in POLY_EVERY uses the polynomial (0: none).  Measured
 // on the causal 4096 workload: 4 -> 0.309 ms, 8 -> 0.302 ms, 0 -> 0.297 ms;
 // this softmax is bound by latency, not by the exponential unit.
-constexpr int POLY_EVERY = 0;
+#ifndef TEA_POLY_EVERY
+#define TEA_POLY_EVERY 0
+#endif
+constexpr int POLY_EVERY = TEA_POLY_EVERY;
 constexpr int POLY_MOD = POLY_EVERY > 0 ? POLY_EVERY : 1;
+// Softmax pipelining inside one key tile:
+//   PIPE_LD    the row max of the first 64 columns runs while the TMEM load
+//              of the last 64 is in flight;
+//   SPLIT_PST  the bf16 P of the first 64 keys is stored to TMEM while the
+//              exponentials of the last 64 are computed.
+#ifndef TEA_PIPE_LD
+#define TEA_PIPE_LD 0
+#endif
+#ifndef TEA_SPLIT_PST
+#define TEA_SPLIT_PST 0
+#endif
+constexpr bool PIPE_LD = TEA_PIPE_LD != 0;
+constexpr bool SPLIT_PST = TEA_SPLIT_PST != 0;
 
 __device__ __forceinline__ void exp2_poly2(float& r0, float& r1, float x0, float x1) {
   constexpr float MAGIC = 12582912.0f;  // 1.5 * 2^23
@@ -510,13 +526,40 @@ __device__ void softmax_slot(const FwdParams& P, const Unit& u, int s, uint8_t* 
     if (!mbar_wait(&bars.s_full[s], it & 1, g, 20 + s)) return;
     tc_fence_after();
     uint32_t x[BN];
-#pragma unroll
-    for (int q = 0; q < BN / 32; q++) tmem_ld32p(t_s + 32 * q, x + 32 * q);
-    tmem_wait_ld();
-
     // Element-wise mask only on tiles that straddle this row's visible range.
     const int key0 = j * BN;
     const bool masked = key0 < key_lo || key0 + BN > key_hi;
+    float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+    if (PIPE_LD && !masked) {
+      // Max of the first half while the second half is still being loaded.
+      tmem_ld32p(t_s, x);
+      tmem_ld32p(t_s + 32, x + 32);
+      tmem_wait_ld();
+      tmem_reg_fence32(x);
+      tmem_reg_fence32(x + 32);
+      tmem_ld32p(t_s + 64, x + 64);
+      tmem_ld32p(t_s + 96, x + 96);
+#pragma unroll
+      for (int cc = 0; cc < BN / 2; cc += 8) {
+        mx0 = max3(mx0, __uint_as_float(x[cc]), __uint_as_float(x[cc + 1]));
+        mx1 = max3(mx1, __uint_as_float(x[cc + 2]), __uint_as_float(x[cc + 3]));
+        mx2 = max3(mx2, __uint_as_float(x[cc + 4]), __uint_as_float(x[cc + 5]));
+        mx3 = max3(mx3, __uint_as_float(x[cc + 6]), __uint_as_float(x[cc + 7]));
+      }
+      tmem_wait_ld();
+      tmem_reg_fence32(x + 64);
+      tmem_reg_fence32(x + 96);
+#pragma unroll
+      for (int cc = BN / 2; cc < BN; cc += 8) {
+        mx0 = max3(mx0, __uint_as_float(x[cc]), __uint_as_float(x[cc + 1]));
+        mx1 = max3(mx1, __uint_as_float(x[cc + 2]), __uint_as_float(x[cc + 3]));
+        mx2 = max3(mx2, __uint_as_float(x[cc + 4]), __uint_as_float(x[cc + 5]));
+        mx3 = max3(mx3, __uint_as_float(x[cc + 6]), __uint_as_float(x[cc + 7]));
+      }
+    } else {
+#pragma unroll
+    for (int q = 0; q < BN / 32; q++) tmem_ld32p(t_s + 32 * q, x + 32 * q);
+    tmem_wait_ld();
     if (masked) {
       if (W && (gh_hi > 0 || gt_hi > gt_lo)) {
         // Global keys on top of the band (rare: only global-token masks).
@@ -535,13 +578,13 @@ __device__ void softmax_slot(const FwdParams& P, const Unit& u, int s, uint8_t* 
         }
       }
     }
-    float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
     for (int cc = 0; cc < BN; cc += 8) {
       mx0 = max3(mx0, __uint_as_float(x[cc]), __uint_as_float(x[cc + 1]));
       mx1 = max3(mx1, __uint_as_float(x[cc + 2]), __uint_as_float(x[cc + 3]));
       mx2 = max3(mx2, __uint_as_float(x[cc + 4]), __uint_as_float(x[cc + 5]));
       mx3 = max3(mx3, __uint_as_float(x[cc + 6]), __uint_as_float(x[cc + 7]));
+    }
     }
     const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
     const float m_cand = mx == -INFINITY ? -INFINITY : mx * c;
@@ -572,6 +615,26 @@ __device__ void softmax_slot(const FwdParams& P, const Unit& u, int s, uint8_t* 
         add2(s0, s1, s0, s1, p0, p1);
         x[cc] = pack_bf16x2(p0, p1);
       }
+    } else if (SPLIT_PST) {
+      // First 64 keys, then their P leaves for tensor memory while the last
+      // 64 keys' exponentials run.
+#pragma unroll
+      for (int cc = 0; cc < BN / 4; cc++) {
+        float a0, a1;
+        fma2(a0, a1, __uint_as_float(x[2 * cc]), __uint_as_float(x[2 * cc + 1]), c, c, -m_sub, -m_sub);
+        const float p0 = ex2_approx(a0), p1 = ex2_approx(a1);
+        add2(s0, s1, s0, s1, p0, p1);
+        x[cc] = pack_bf16x2(p0, p1);
+      }
+      tmem_st32(t_s, x);
+#pragma unroll
+      for (int cc = BN / 4; cc < BN / 2; cc++) {
+        float a0, a1;
+        fma2(a0, a1, __uint_as_float(x[2 * cc]), __uint_as_float(x[2 * cc + 1]), c, c, -m_sub, -m_sub);
+        const float p0 = ex2_approx(a0), p1 = ex2_approx(a1);
+        add2(s0, s1, s0, s1, p0, p1);
+        x[cc] = pack_bf16x2(p0, p1);
+      }
     } else {
 #pragma unroll
       for (int cc = 0; cc < BN / 2; cc++) {
@@ -584,7 +647,7 @@ __device__ void softmax_slot(const FwdParams& P, const Unit& u, int s, uint8_t* 
     }
     l += s0 + s1;
     // P (bf16, two per column) replaces the first BN/2 columns of S.
-    tmem_st32(t_s, x);
+    if (!(SPLIT_PST && !poly)) tmem_st32(t_s, x);
     tmem_st32(t_s + 32, x + 32);
     tmem_wait_st();
     if (__any_sync(0xffffffffu, need) && it > 0) {
