@@ -84,11 +84,10 @@ def test_bwd_rejects_bad_arguments(ta, kw, status):
 
 
 def test_bwd_workspace_size(ta):
-    """D (fp32 per query row) and the transposed fp32 dQ accumulator [B*Hq, d, Lq rounded up to 4],
-    each padded to 256 bytes."""
+    """D (fp32 per query row) and the fp32 dQ accumulator [B*Hq, Lq, d], each padded to 256 bytes."""
     n = ta.bwd_workspace_size(2, 4, 2, 101, 50, 64)
     rows = 2 * 4 * 101
-    acc = 2 * 4 * 64 * 104
+    acc = rows * 64
     assert n == -(-rows * 4 // 256) * 256 + -(-acc * 4 // 256) * 256
     assert ta.bwd_workspace_size(0, 4, 2, 100, 50, 64) == 0
     assert ta.bwd_workspace_size(1, 3, 2, 100, 50, 64) == 0

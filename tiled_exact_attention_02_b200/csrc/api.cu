@@ -288,7 +288,7 @@ size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int Lq, int Lk, int d) {
   if (B == 0 || Hq == 0 || Lq == 0) return 0;
   const size_t rows = (size_t)B * Hq * Lq;
   const size_t dsz = (rows * 4 + 255) / 256 * 256;                                    // D, fp32
-  const size_t dq = ((size_t)B * Hq * d * bwd_lq_pad(Lq) * 4 + 255) / 256 * 256;  // dQ^T accumulator, fp32
+  const size_t dq = ((size_t)B * Hq * Lq * d * 4 + 255) / 256 * 256;                // dQ accumulator, fp32
   return dsz + dq;
 }
 
@@ -313,7 +313,7 @@ int attn_bwd_preprocess(const void* o, const void* dO, int B, int Hq, int Lq, in
   float *dvec, *dq_acc;
   if ((st = split_workspace(B, Hq, Lq, d, workspace, workspace_bytes, &dvec, &dq_acc)) != ATTN_OK) return st;
   const cudaError_t e = launch_bwd_pre(o, dO, dvec, dq_acc, (int64_t)B * Hq * Lq, d,
-                                       (int64_t)B * Hq * d * bwd_lq_pad(Lq), static_cast<cudaStream_t>(stream));
+                                       (int64_t)B * Hq * Lq * d, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? ATTN_OK : cuda_fail("attn_bwd_preprocess launch", e);
 }
 
@@ -367,16 +367,16 @@ static int bwd_main_impl(const void* q, const void* k, const void* v, const floa
   P.lse = lse;
   P.dvec = dvec;
   P.dq_acc = dq_acc;
-  P.lq_pad = bwd_lq_pad(Lq);
   if (d == 128) {
-    // dQ^T accumulator as a 2-D fp32 tensor [B*Hq*d rows, Lq columns] (row pitch lq_pad):
-    // each step's 128 x 64 tile is added as two 128-row x 32-column boxes.
-    cuuint64_t dims[2] = {(cuuint64_t)Lq, (cuuint64_t)B * Hq * d};
-    cuuint64_t strides[1] = {(cuuint64_t)P.lq_pad * 4};
-    cuuint32_t box[2] = {32, 128};
-    cuuint32_t es[2] = {1, 1};
-    const CUresult r = enc(&P.tm_dq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, dq_acc, dims, strides, box, es,
-                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+    // dQ accumulator as a 3-D fp32 tensor [B*Hq, Lq, d]: each step's 64-query
+    // tile is added as two boxes of 32 query rows x 128 d (rows past a head's
+    // Lq fall outside the tensor and are dropped).
+    cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)Lq, (cuuint64_t)B * Hq};
+    cuuint64_t strides[2] = {(cuuint64_t)d * 4, (cuuint64_t)Lq * d * 4};
+    cuuint32_t box[3] = {128, 32, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    const CUresult r = enc(&P.tm_dq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, dq_acc, dims, strides, box, es,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return cu_fail("cuTensorMapEncodeTiled dQ", r);
   }
@@ -419,7 +419,7 @@ int attn_bwd_finalize(void* dq, int B, int Hq, int Lq, int d, float scale, void*
   if (!dq || !aligned16(dq)) return ATTN_ERR_INVALID_ARG;
   float *dvec, *dq_acc;
   if ((st = split_workspace(B, Hq, Lq, d, workspace, workspace_bytes, &dvec, &dq_acc)) != ATTN_OK) return st;
-  const cudaError_t e = launch_bwd_post(dq_acc, dq, B * Hq, Lq, bwd_lq_pad(Lq), d, scale, static_cast<cudaStream_t>(stream));
+  const cudaError_t e = launch_bwd_post(dq_acc, dq, (int64_t)B * Hq * Lq * d, scale, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? ATTN_OK : cuda_fail("attn_bwd_finalize launch", e);
 }
 

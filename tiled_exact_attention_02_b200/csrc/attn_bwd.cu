@@ -13,9 +13,9 @@
 //             the query heads of the GQA group and the query tiles that see
 //             its keys, accumulating dK and dV in tensor memory for the whole
 //             loop and adding each step's dQ contribution into the fp32
-//             accumulator (d = 128: TMA tensor reduce-add from a swizzled
-//             staging tile; d = 64: coalesced red.global)
-//   bwd_post  dQ = scale * accumulator, rounded to bf16
+//             accumulator [B*Hq, Lq, d] (d = 128: TMA tensor reduce-add from a
+//             staging tile; d = 64: vector red.global from registers)
+//   bwd_post  dQ = scale * accumulator, rounded to bf16 (element-wise)
 //
 // bwd_main works in the transposed orientation, keys on the 128 TMEM lanes:
 //   S^T = K Q^T and dP^T = V dO^T     (M = 128 keys, N = BM query rows)
@@ -57,7 +57,7 @@ struct Cfg {
   static constexpr bool TS = D == 128;
   static constexpr int NQS = 3;                   // Q/dO ring stages
   // d = 128: the dQ^T tile of a step leaves through two 16 KB halves of a
-  // 128-byte-swizzled staging area and a TMA tensor reduce-add.
+  // staging area ([32 query rows][128 d] fp32 each) and a TMA tensor reduce-add.
   static constexpr int STG_BYTES = D == 128 ? 2 * 16384 : 0;
   static constexpr int KV_TILE = BN * D * 2;
   static constexpr int Q_TILE = BM * D * 2;
@@ -78,7 +78,7 @@ struct Cfg {
   static constexpr uint32_t T_PT = T_DQ + 64, T_DST = T_PT + BM / 2;  // bf16 pairs (TS only)
   static_assert(T_DQ + 64 <= 512 && (!TS || T_DST + BM / 2 <= 512), "tensor memory budget");
   static_assert(SMEM <= 232448, "shared memory budget");
-  static_assert(OFF_STG % 1024 == 0, "staging must be 1024-byte aligned for the 128-byte swizzle");
+  static_assert(OFF_STG % 1024 == 0, "staging must be 1024-byte aligned");
 };
 
 // Barriers.  The MMA issuer pays for every wait and commit with tensor-core
@@ -534,25 +534,27 @@ __device__ void grad_rows(const BwdParams& P, const Unit& u, uint8_t* smem, Bars
 }
 
 // ------------------------------------------------------------------ dQ drain
-// Moves each step's fp32 dQ tile out of tensor memory into the accumulator,
-// which is stored transposed, [head][d][q] (row pitch lq_pad), so that the
-// values a lane holds are contiguous in it:
-//   d = 128 (dQ^T in TMEM, lane = d, 64 query columns): the lane writes its
-//     row as 16-byte pieces into a 128-byte-swizzled staging half (32
-//     queries x 128 rows = 16 KB, conflict-free), and one thread adds the
-//     half into the accumulator with a TMA tensor reduce-add (element-wise
-//     atomic in L2); two halves alternate so staging overlaps the reduce.
-//   d = 64 (dQ in TMEM, lane = query, 64 d columns): per column, the lanes
-//     hold 32 consecutive queries, so red.global covers 128 bytes per warp.
-__device__ __forceinline__ void red_add_f32(float* p, float v) {
-  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
+// Moves each step's fp32 dQ tile out of tensor memory into the accumulator
+// [B*Hq, Lq, d] (the layout of dQ itself, so the final pass is element-wise):
+//   d = 128 (dQ^T in TMEM, lane = d, 64 query columns): lane t writes element
+//     (q, t) of a row-major staging half [32 queries][128 d] (for each q the
+//     warp's 32 lanes fill 128 contiguous bytes: no bank conflict), and one
+//     thread adds the half into the accumulator with a TMA tensor reduce-add
+//     (element-wise atomic in L2; rows past Lq are clipped by the tensor's
+//     bounds); two halves alternate so staging overlaps the reduce.
+//   d = 64 (dQ in TMEM, lane = query, 64 d columns): the lane's row is 256
+//     contiguous bytes of the accumulator, added with 16 vector red.global.
+__device__ __forceinline__ void red_add_v4_f32(float* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(__uint_as_float(a)),
+               "f"(__uint_as_float(b)), "f"(__uint_as_float(c)), "f"(__uint_as_float(d))
+               : "memory");
 }
 
-__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* map, const void* src, int c0, int c1) {
+__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* map, const void* src, int c0, int c1, int c2) {
   asm volatile(
-      "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+      "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
           reinterpret_cast<uint64_t>(map)),
-      "r"(smem_u32(src)), "r"(c0), "r"(c1)
+      "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
 }
 // Wait until at most one committed bulk group still reads shared memory.
@@ -591,29 +593,27 @@ __device__ void dq_drain(const BwdParams& P, const Unit& u, uint8_t* smem, Bars&
         const int b = half & 1, use = half >> 1;
         // The reduce of this buffer's previous use must have read it.
         if (use > 0 && !mbar_wait(&bars.stg_free[b], (use - 1) & 1, g, 31)) return;
-        uint8_t* row = stg + b * 16384 + t * 128;
+        float* col = reinterpret_cast<float*>(stg + b * 16384) + t;
 #pragma unroll
-        for (int c = 0; c < 8; c++)
-          *reinterpret_cast<uint4*>(row + (((uint32_t)c ^ (uint32_t)(t & 7)) << 4)) =
-              make_uint4(r[32 * hh + 4 * c], r[32 * hh + 4 * c + 1], r[32 * hh + 4 * c + 2], r[32 * hh + 4 * c + 3]);
+        for (int qq = 0; qq < 32; qq++) col[qq * 128] = __uint_as_float(r[32 * hh + qq]);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars.stg_full[b]);
         if (t == 0) {
           if (!mbar_wait(&bars.stg_full[b], use & 1, g, 32)) return;
-          // Columns past Lq are clipped by the tensor bounds.
-          tma_reduce_add_2d(&P.tm_dq, stg + b * 16384, q0 + 32 * hh, bh * D);
+          // Query rows past Lq are clipped by the tensor bounds.
+          tma_reduce_add_3d(&P.tm_dq, stg + b * 16384, 0, q0 + 32 * hh, bh);
           bulk_commit();
           bulk_wait_read_1();  // the previous half has been read
           if (half > 0) mbar_arrive(&bars.stg_free[(half - 1) & 1]);
         }
       }
     } else {
-      // Lane t holds dQ row q0 + t: column c goes to accumulator row (bh, c).
+      // Lane t holds dQ row q0 + t.
       if (q0 + t < p.Lq) {
-        float* colp = P.dq_acc + (size_t)bh * D * P.lq_pad + q0 + t;
+        float* rowp = P.dq_acc + ((size_t)bh * p.Lq + q0 + t) * D;
 #pragma unroll
-        for (int c = 0; c < 64; c++) red_add_f32(colp + (size_t)c * P.lq_pad, __uint_as_float(r[c]));
+        for (int c = 0; c < 16; c++) red_add_v4_f32(rowp + 4 * c, r[4 * c], r[4 * c + 1], r[4 * c + 2], r[4 * c + 3]);
       }
     }
   }
@@ -734,60 +734,25 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const uint16_t* __restrict
   for (int64_t x = tid; x < acc_floats / 4; x += stride) z[x] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
-// dQ[bh, q, :] = scale * acc[bh, :, q], rounded to bf16.  One CTA transposes a
-// 64-query x d tile through shared memory: reads run along q (16 bytes per
-// thread: lq_pad is a multiple of 4 and the accumulator is 256-byte aligned,
-// so every 4-query group below lq_pad is one aligned float4), writes along d.
-// Accumulator columns in [Lq, lq_pad) were zeroed by the preprocess and are
-// read but never written out.
-template <int D>
-__global__ void __launch_bounds__(256) bwd_post_kernel(const float* __restrict__ acc, uint16_t* __restrict__ dq, int Lq,
-                                                       int lq_pad, float scale) {
-  __shared__ float tile[D][65];
-  const int bh = blockIdx.y;
-  const int q0 = blockIdx.x * 64;
-  const float* src = acc + (size_t)bh * D * lq_pad;
-  for (int idx = threadIdx.x; idx < D * 16; idx += 256) {
-    const int dd = idx / 16, qv = idx % 16;
-    const int q = q0 + 4 * qv;
-    float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (q < lq_pad) f = *reinterpret_cast<const float4*>(src + (size_t)dd * lq_pad + q);
-    tile[dd][4 * qv] = f.x;
-    tile[dd][4 * qv + 1] = f.y;
-    tile[dd][4 * qv + 2] = f.z;
-    tile[dd][4 * qv + 3] = f.w;
-  }
-  __syncthreads();
-  constexpr int CH = D / 8;  // 16-byte output chunks per row
-  for (int idx = threadIdx.x; idx < 64 * CH; idx += 256) {
-    const int qq = idx / CH, c = idx % CH;
-    const int q = q0 + qq;
-    if (q < Lq) {
-      uint4 w;
-      w.x = pack_bf16x2(tile[c * 8 + 0][qq] * scale, tile[c * 8 + 1][qq] * scale);
-      w.y = pack_bf16x2(tile[c * 8 + 2][qq] * scale, tile[c * 8 + 3][qq] * scale);
-      w.z = pack_bf16x2(tile[c * 8 + 4][qq] * scale, tile[c * 8 + 5][qq] * scale);
-      w.w = pack_bf16x2(tile[c * 8 + 6][qq] * scale, tile[c * 8 + 7][qq] * scale);
-      *reinterpret_cast<uint4*>(dq + ((size_t)bh * Lq + q) * D + c * 8) = w;
-    }
-  }
-}
-
-// out = bf16(acc), 8 elements (two float4 in, one uint4 out) per thread and
-// iteration; a tail of fewer than 8 elements is converted one by one.
+// out = bf16(scale * acc), 8 elements (two float4 in, one uint4 out) per
+// thread and iteration; a tail of fewer than 8 elements is converted one by
+// one.  With scale = the softmax scale and acc the dQ accumulator this is the
+// last backward phase (dQ = scale * dS K); with scale = 1 it rounds an fp32
+// accumulator (ring attention's dK / dV).
 __global__ void __launch_bounds__(256) f32_to_bf16_kernel(const float* __restrict__ acc, uint16_t* __restrict__ out,
-                                                          int64_t n) {
+                                                          int64_t n, float scale) {
   const int64_t n8 = n / 8;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; x < n8; x += stride) {
     const float4 a = reinterpret_cast<const float4*>(acc)[2 * x];
     const float4 b = reinterpret_cast<const float4*>(acc)[2 * x + 1];
     reinterpret_cast<uint4*>(out)[x] =
-        make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
+        make_uint4(pack_bf16x2(a.x * scale, a.y * scale), pack_bf16x2(a.z * scale, a.w * scale),
+                   pack_bf16x2(b.x * scale, b.y * scale), pack_bf16x2(b.z * scale, b.w * scale));
   }
   if (blockIdx.x == 0 && threadIdx.x < n - n8 * 8) {
     const int64_t i = n8 * 8 + threadIdx.x;
-    out[i] = (uint16_t)(pack_bf16x2(acc[i], 0.f) & 0xFFFFu);
+    out[i] = (uint16_t)(pack_bf16x2(acc[i] * scale, 0.f) & 0xFFFFu);
   }
 }
 
@@ -817,22 +782,15 @@ cudaError_t launch_bwd_pre(const void* o, const void* dO, float* dvec, float* dq
   return cudaGetLastError();
 }
 
-cudaError_t launch_bwd_post(const float* dq_acc, void* dq, int BH, int Lq, int lq_pad, int d, float scale,
-                            cudaStream_t stream) {
-  if (BH <= 0 || Lq <= 0) return cudaSuccess;
-  const dim3 grid((Lq + 63) / 64, BH);
-  if (d == 128)
-    bwd::bwd_post_kernel<128><<<grid, 256, 0, stream>>>(dq_acc, static_cast<uint16_t*>(dq), Lq, lq_pad, scale);
-  else
-    bwd::bwd_post_kernel<64><<<grid, 256, 0, stream>>>(dq_acc, static_cast<uint16_t*>(dq), Lq, lq_pad, scale);
+cudaError_t launch_bwd_post(const float* dq_acc, void* dq, int64_t n, float scale, cudaStream_t stream) {
+  if (n <= 0) return cudaSuccess;
+  const int grid = elementwise_grid(n / 8 > 0 ? n / 8 : 1);
+  bwd::f32_to_bf16_kernel<<<grid, 256, 0, stream>>>(dq_acc, static_cast<uint16_t*>(dq), n, scale);
   return cudaGetLastError();
 }
 
 cudaError_t launch_f32_to_bf16(const float* acc, void* out, size_t n, cudaStream_t stream) {
-  if (n == 0) return cudaSuccess;
-  const int grid = elementwise_grid((int64_t)(n / 8) > 0 ? (int64_t)(n / 8) : 1);
-  bwd::f32_to_bf16_kernel<<<grid, 256, 0, stream>>>(acc, static_cast<uint16_t*>(out), (int64_t)n);
-  return cudaGetLastError();
+  return launch_bwd_post(acc, out, (int64_t)n, 1.f, stream);
 }
 
 template <int D>

@@ -526,11 +526,40 @@ __device__ void softmax_slot(const FwdParams& P, const Unit& u, int s, uint8_t* 
     if (!mbar_wait(&bars.s_full[s], it & 1, g, 20 + s)) return;
     tc_fence_after();
     uint32_t x[BN];
-    // Element-wise mask only on tiles that straddle this row's visible range.
+    // Element-wise mask only on tiles that straddle this row's visible range
+    // (a per-row condition: it never guards a tcgen05 instruction, which the
+    // whole warp must execute together).
     const int key0 = j * BN;
     const bool masked = key0 < key_lo || key0 + BN > key_hi;
+    auto mask_cols = [&](int c0, int c1) {
+      if (W && (gh_hi > 0 || gt_hi > gt_lo)) {
+        // Global keys on top of the band (rare: only global-token masks).
+#pragma unroll
+        for (int cc = c0; cc < c1; cc++) {
+          const int key = key0 + cc;
+          const bool vis = (unsigned)(key - key_lo) < (unsigned)(key_hi - key_lo) || key < gh_hi ||
+                           (unsigned)(key - gt_lo) < (unsigned)(gt_hi - gt_lo);
+          if (!vis) x[cc] = __float_as_uint(-INFINITY);
+        }
+      } else {
+#pragma unroll
+        for (int cc = c0; cc < c1; cc++) {
+          const int key = key0 + cc;
+          if (key < key_lo || key >= key_hi) x[cc] = __float_as_uint(-INFINITY);
+        }
+      }
+    };
     float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
-    if (PIPE_LD && !masked) {
+    auto max_cols = [&](int c0, int c1) {
+#pragma unroll
+      for (int cc = c0; cc < c1; cc += 8) {
+        mx0 = max3(mx0, __uint_as_float(x[cc]), __uint_as_float(x[cc + 1]));
+        mx1 = max3(mx1, __uint_as_float(x[cc + 2]), __uint_as_float(x[cc + 3]));
+        mx2 = max3(mx2, __uint_as_float(x[cc + 4]), __uint_as_float(x[cc + 5]));
+        mx3 = max3(mx3, __uint_as_float(x[cc + 6]), __uint_as_float(x[cc + 7]));
+      }
+    };
+    if constexpr (PIPE_LD) {
       // Max of the first half while the second half is still being loaded.
       tmem_ld32p(t_s, x);
       tmem_ld32p(t_s + 32, x + 32);
@@ -539,52 +568,19 @@ __device__ void softmax_slot(const FwdParams& P, const Unit& u, int s, uint8_t* 
       tmem_reg_fence32(x + 32);
       tmem_ld32p(t_s + 64, x + 64);
       tmem_ld32p(t_s + 96, x + 96);
-#pragma unroll
-      for (int cc = 0; cc < BN / 2; cc += 8) {
-        mx0 = max3(mx0, __uint_as_float(x[cc]), __uint_as_float(x[cc + 1]));
-        mx1 = max3(mx1, __uint_as_float(x[cc + 2]), __uint_as_float(x[cc + 3]));
-        mx2 = max3(mx2, __uint_as_float(x[cc + 4]), __uint_as_float(x[cc + 5]));
-        mx3 = max3(mx3, __uint_as_float(x[cc + 6]), __uint_as_float(x[cc + 7]));
-      }
+      if (masked) mask_cols(0, BN / 2);
+      max_cols(0, BN / 2);
       tmem_wait_ld();
       tmem_reg_fence32(x + 64);
       tmem_reg_fence32(x + 96);
-#pragma unroll
-      for (int cc = BN / 2; cc < BN; cc += 8) {
-        mx0 = max3(mx0, __uint_as_float(x[cc]), __uint_as_float(x[cc + 1]));
-        mx1 = max3(mx1, __uint_as_float(x[cc + 2]), __uint_as_float(x[cc + 3]));
-        mx2 = max3(mx2, __uint_as_float(x[cc + 4]), __uint_as_float(x[cc + 5]));
-        mx3 = max3(mx3, __uint_as_float(x[cc + 6]), __uint_as_float(x[cc + 7]));
-      }
+      if (masked) mask_cols(BN / 2, BN);
+      max_cols(BN / 2, BN);
     } else {
 #pragma unroll
-    for (int q = 0; q < BN / 32; q++) tmem_ld32p(t_s + 32 * q, x + 32 * q);
-    tmem_wait_ld();
-    if (masked) {
-      if (W && (gh_hi > 0 || gt_hi > gt_lo)) {
-        // Global keys on top of the band (rare: only global-token masks).
-#pragma unroll
-        for (int cc = 0; cc < BN; cc++) {
-          const int key = key0 + cc;
-          const bool vis = (unsigned)(key - key_lo) < (unsigned)(key_hi - key_lo) || key < gh_hi ||
-                           (unsigned)(key - gt_lo) < (unsigned)(gt_hi - gt_lo);
-          if (!vis) x[cc] = __float_as_uint(-INFINITY);
-        }
-      } else {
-#pragma unroll
-        for (int cc = 0; cc < BN; cc++) {
-          const int key = key0 + cc;
-          if (key < key_lo || key >= key_hi) x[cc] = __float_as_uint(-INFINITY);
-        }
-      }
-    }
-#pragma unroll
-    for (int cc = 0; cc < BN; cc += 8) {
-      mx0 = max3(mx0, __uint_as_float(x[cc]), __uint_as_float(x[cc + 1]));
-      mx1 = max3(mx1, __uint_as_float(x[cc + 2]), __uint_as_float(x[cc + 3]));
-      mx2 = max3(mx2, __uint_as_float(x[cc + 4]), __uint_as_float(x[cc + 5]));
-      mx3 = max3(mx3, __uint_as_float(x[cc + 6]), __uint_as_float(x[cc + 7]));
-    }
+      for (int q = 0; q < BN / 32; q++) tmem_ld32p(t_s + 32 * q, x + 32 * q);
+      tmem_wait_ld();
+      if (masked) mask_cols(0, BN);
+      max_cols(0, BN);
     }
     const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
     const float m_cand = mx == -INFINITY ? -INFINITY : mx * c;

@@ -41,9 +41,8 @@ struct BwdParams {
   Problem prob;
   const float* lse;   // fp32 [B, Hq, Lq], natural log (forward output)
   const float* dvec;  // fp32 [B, Hq, Lq], D_i = dO_i . O_i (workspace)
-  float* dq_acc;      // fp32 [B*Hq, d, lq_pad]: dQ transposed, summed over key tiles (workspace)
-  int lq_pad;         // row pitch of dq_acc in floats (Lq rounded up to a multiple of 4)
-  CUtensorMap tm_dq;  // dq_acc as 2-D [B*Hq*d rows, Lq cols], box 32 x 128, 128-byte swizzle (d = 128)
+  float* dq_acc;      // fp32 [B*Hq, Lq, d]: dQ / scale summed over key tiles (workspace)
+  CUtensorMap tm_dq;  // dq_acc as 3-D [B*Hq, Lq, d], box 128 x 32 x 1, no swizzle (d = 128)
   void* dk;           // bf16 [B, Hkv, Lk, d]
   void* dv;           // bf16 [B, Hkv, Lk, d]
   // Accumulate mode (both non-null): dK (already scaled) and dV are added into
@@ -90,14 +89,13 @@ inline cudaError_t once_per_device(std::atomic<unsigned char> (&done)[kMaxDevice
 inline int bwd_block_m(int d) { return d == 128 ? 64 : 128; }
 
 // Workspace layout of the backward: D (fp32 [B*Hq*Lq], padded to 256 bytes), then
-// the transposed dQ accumulator fp32 [B*Hq, d, lq_pad].
-inline int bwd_lq_pad(int Lq) { return (Lq + 3) / 4 * 4; }
+// the dQ accumulator fp32 [B*Hq, Lq, d].
 
 cudaError_t launch_bwd_pre(const void* o, const void* dO, float* dvec, float* dq_acc, int64_t rows, int d,
                            int64_t acc_floats, cudaStream_t stream);
 cudaError_t launch_bwd(const BwdParams& P, cudaStream_t stream);
-cudaError_t launch_bwd_post(const float* dq_acc, void* dq, int BH, int Lq, int lq_pad, int d, float scale,
-                            cudaStream_t stream);
+// dq = bf16(scale * dq_acc), n elements.
+cudaError_t launch_bwd_post(const float* dq_acc, void* dq, int64_t n, float scale, cudaStream_t stream);
 // out[i] = bf16(acc[i]) (round to nearest even), n elements.
 cudaError_t launch_f32_to_bf16(const float* acc, void* out, size_t n, cudaStream_t stream);
 
