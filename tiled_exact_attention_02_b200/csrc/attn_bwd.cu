@@ -42,6 +42,13 @@
 namespace tea {
 namespace bwd {
 
+#ifndef TEA_DQ_RED
+#define TEA_DQ_RED 0
+#endif
+// d = 128: 1 adds each step's dQ with red.global from the drain warps'
+// registers (no shared-memory staging); 0 stages it for a TMA reduce-add.
+constexpr bool DQ_RED = TEA_DQ_RED != 0;
+
 constexpr int BN = 128;  // keys per CTA
 constexpr int THREADS = 512;
 constexpr int KPANEL = 16384;  // 128 rows x 128 bytes
@@ -58,7 +65,7 @@ struct Cfg {
   static constexpr int NQS = 3;                   // Q/dO ring stages
   // d = 128: the dQ^T tile of a step leaves through two 16 KB halves of a
   // staging area ([32 query rows][128 d] fp32 each) and a TMA tensor reduce-add.
-  static constexpr int STG_BYTES = D == 128 ? 2 * 16384 : 0;
+  static constexpr int STG_BYTES = (D == 128 && !DQ_RED) ? 2 * 16384 : 0;
   static constexpr int KV_TILE = BN * D * 2;
   static constexpr int Q_TILE = BM * D * 2;
   static constexpr int Q_PANEL = BM * 128;
@@ -544,6 +551,9 @@ __device__ void grad_rows(const BwdParams& P, const Unit& u, uint8_t* smem, Bars
 //     bounds); two halves alternate so staging overlaps the reduce.
 //   d = 64 (dQ in TMEM, lane = query, 64 d columns): the lane's row is 256
 //     contiguous bytes of the accumulator, added with 16 vector red.global.
+__device__ __forceinline__ void red_add_f32(float* p, float v) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
+}
 __device__ __forceinline__ void red_add_v4_f32(float* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(__uint_as_float(a)),
                "f"(__uint_as_float(b)), "f"(__uint_as_float(c)), "f"(__uint_as_float(d))
@@ -587,7 +597,15 @@ __device__ void dq_drain(const BwdParams& P, const Unit& u, uint8_t* smem, Bars&
     __syncwarp();
     if (lane == 0) mbar_arrive(&bars.grad_ready[(i + 1) & 1]);  // dQ TMEM free for step i+1
     const int bh = u.b * p.Hq + h;
-    if constexpr (D == 128) {
+    if constexpr (D == 128 && DQ_RED) {
+      // Lane t holds column t of the 64 query rows: for each row the warp's
+      // 32 lanes add 128 contiguous bytes.
+      float* colp = P.dq_acc + ((size_t)bh * p.Lq + q0) * D + t;
+      const int nq = imin(64, p.Lq - q0);
+#pragma unroll
+      for (int qq = 0; qq < 64; qq++)
+        if (qq < nq) red_add_f32(colp + (size_t)qq * D, __uint_as_float(r[qq]));
+    } else if constexpr (D == 128) {
 #pragma unroll
       for (int hh = 0; hh < 2; hh++, half++) {
         const int b = half & 1, use = half >> 1;
@@ -617,7 +635,7 @@ __device__ void dq_drain(const BwdParams& P, const Unit& u, uint8_t* smem, Bars&
       }
     }
   }
-  if (D == 128 && t == 0) bulk_wait_all();  // every reduce complete before the CTA exits
+  if (D == 128 && !DQ_RED && t == 0) bulk_wait_all();  // every reduce complete before the CTA exits
 }
 
 // ------------------------------------------------------------------ kernel

@@ -43,59 +43,6 @@ constexpr int THREADS = 384;
 constexpr int PANEL = 16384;   // one 128-row x 128-byte swizzled panel
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
 
-// Part of the exponentials run on the FMA pipe instead of the special-function
-// unit, which is otherwise the busiest pipe of the softmax: 2^x = 2^n * p(f)
-// with n = round(x) (Cody-Waite reduction: adding 1.5 * 2^23 rounds to an
-// integer and leaves n in the low mantissa bits), f = x - n in [-1/2, 1/2], p
-// the degree-4 polynomial minimising the relative error of 2^f there (Remez
-// exchange; coefficients from gen_exp2_poly.py, error < 3e-6), and 2^n
-// applied by adding n to the exponent field.  Arguments are clamped at -126
-// (p(f) may sit just below 1, exponent field 126, so n >= -126 keeps the sum
-// from wrapping into the sign bit);
-// only tiles without masked entries use it, so a masked -inf never gets here.
-constexpr float EXP2_C0 = 0.9999992847442627f;  // 0x3f7ffff4
-constexpr float EXP2_C1 = 0.6931217908859253f;  // 0x3f31706e
-constexpr float EXP2_C2 = 0.240247443318367f;  // 0x3e76036d
-constexpr float EXP2_C3 = 0.05591785907745361f;  // 0x3d650a20
-constexpr float EXP2_C4 = 0.009570102207362652f;  // 0x3c1ccbeb
-// One pair of columns in POLY_EVERY uses the polynomial (0: none).  Measured
-// on the causal 4096 workload: 4 -> 0.309 ms, 8 -> 0.302 ms, 0 -> 0.297 ms;
-// this softmax is bound by latency, not by the exponential unit.
-#ifndef TEA_POLY_EVERY
-#define TEA_POLY_EVERY 0
-#endif
-constexpr int POLY_EVERY = TEA_POLY_EVERY;
-constexpr int POLY_MOD = POLY_EVERY > 0 ? POLY_EVERY : 1;
-// Softmax pipelining inside one key tile:
-//   PIPE_LD    the row max of the first 64 columns runs while the TMEM load
-//              of the last 64 is in flight;
-//   SPLIT_PST  the bf16 P of the first 64 keys is stored to TMEM while the
-//              exponentials of the last 64 are computed.
-#ifndef TEA_PIPE_LD
-#define TEA_PIPE_LD 0
-#endif
-#ifndef TEA_SPLIT_PST
-#define TEA_SPLIT_PST 0
-#endif
-constexpr bool PIPE_LD = TEA_PIPE_LD != 0;
-constexpr bool SPLIT_PST = TEA_SPLIT_PST != 0;
-
-__device__ __forceinline__ void exp2_poly2(float& r0, float& r1, float x0, float x1) {
-  constexpr float MAGIC = 12582912.0f;  // 1.5 * 2^23
-  x0 = fmaxf(x0, -126.f);
-  x1 = fmaxf(x1, -126.f);
-  float t0, t1, n0, n1, f0, f1, p0, p1;
-  add2(t0, t1, x0, x1, MAGIC, MAGIC);
-  add2(n0, n1, t0, t1, -MAGIC, -MAGIC);
-  fma2(f0, f1, n0, n1, -1.f, -1.f, x0, x1);
-  fma2(p0, p1, EXP2_C4, EXP2_C4, f0, f1, EXP2_C3, EXP2_C3);
-  fma2(p0, p1, p0, p1, f0, f1, EXP2_C2, EXP2_C2);
-  fma2(p0, p1, p0, p1, f0, f1, EXP2_C1, EXP2_C1);
-  fma2(p0, p1, p0, p1, f0, f1, EXP2_C0, EXP2_C0);
-  r0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
-  r1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
-}
-
 template <int D>
 struct Cfg {
   static constexpr int PANELS = D / 64;
@@ -559,29 +506,11 @@ __device__ void softmax_slot(const FwdParams& P, const Unit& u, int s, uint8_t* 
         mx3 = max3(mx3, __uint_as_float(x[cc + 6]), __uint_as_float(x[cc + 7]));
       }
     };
-    if constexpr (PIPE_LD) {
-      // Max of the first half while the second half is still being loaded.
-      tmem_ld32p(t_s, x);
-      tmem_ld32p(t_s + 32, x + 32);
-      tmem_wait_ld();
-      tmem_reg_fence32(x);
-      tmem_reg_fence32(x + 32);
-      tmem_ld32p(t_s + 64, x + 64);
-      tmem_ld32p(t_s + 96, x + 96);
-      if (masked) mask_cols(0, BN / 2);
-      max_cols(0, BN / 2);
-      tmem_wait_ld();
-      tmem_reg_fence32(x + 64);
-      tmem_reg_fence32(x + 96);
-      if (masked) mask_cols(BN / 2, BN);
-      max_cols(BN / 2, BN);
-    } else {
 #pragma unroll
-      for (int q = 0; q < BN / 32; q++) tmem_ld32p(t_s + 32 * q, x + 32 * q);
-      tmem_wait_ld();
-      if (masked) mask_cols(0, BN);
-      max_cols(0, BN);
-    }
+    for (int q = 0; q < BN / 32; q++) tmem_ld32p(t_s + 32 * q, x + 32 * q);
+    tmem_wait_ld();
+    if (masked) mask_cols(0, BN);
+    max_cols(0, BN);
     const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
     const float m_cand = mx == -INFINITY ? -INFINITY : mx * c;
     const float m_new = fmaxf(m, m_cand);
@@ -594,56 +523,18 @@ __device__ void softmax_slot(const FwdParams& P, const Unit& u, int s, uint8_t* 
     const float m_sub = m == -INFINITY ? 0.f : m;
     float s0 = 0.f, s1 = 0.f;
     // P packed two per 32-bit word, written over x[0 .. BN/2) as it goes
-    // (x[2cc], x[2cc+1] are dead once read).  Tiles this warp sees without
-    // masking send one pair in POLY_EVERY to the FMA-pipe exponential.
-    const bool poly = POLY_EVERY > 0 && __all_sync(0xffffffffu, !masked);
-    if (poly) {
+    // (x[2cc], x[2cc+1] are dead once read).
 #pragma unroll
-      for (int cc = 0; cc < BN / 2; cc++) {
-        float a0, a1, p0, p1;
-        fma2(a0, a1, __uint_as_float(x[2 * cc]), __uint_as_float(x[2 * cc + 1]), c, c, -m_sub, -m_sub);
-        if (POLY_EVERY > 0 && cc % POLY_MOD == POLY_MOD - 1) {
-          exp2_poly2(p0, p1, a0, a1);
-        } else {
-          p0 = ex2_approx(a0);
-          p1 = ex2_approx(a1);
-        }
-        add2(s0, s1, s0, s1, p0, p1);
-        x[cc] = pack_bf16x2(p0, p1);
-      }
-    } else if (SPLIT_PST) {
-      // First 64 keys, then their P leaves for tensor memory while the last
-      // 64 keys' exponentials run.
-#pragma unroll
-      for (int cc = 0; cc < BN / 4; cc++) {
-        float a0, a1;
-        fma2(a0, a1, __uint_as_float(x[2 * cc]), __uint_as_float(x[2 * cc + 1]), c, c, -m_sub, -m_sub);
-        const float p0 = ex2_approx(a0), p1 = ex2_approx(a1);
-        add2(s0, s1, s0, s1, p0, p1);
-        x[cc] = pack_bf16x2(p0, p1);
-      }
-      tmem_st32(t_s, x);
-#pragma unroll
-      for (int cc = BN / 4; cc < BN / 2; cc++) {
-        float a0, a1;
-        fma2(a0, a1, __uint_as_float(x[2 * cc]), __uint_as_float(x[2 * cc + 1]), c, c, -m_sub, -m_sub);
-        const float p0 = ex2_approx(a0), p1 = ex2_approx(a1);
-        add2(s0, s1, s0, s1, p0, p1);
-        x[cc] = pack_bf16x2(p0, p1);
-      }
-    } else {
-#pragma unroll
-      for (int cc = 0; cc < BN / 2; cc++) {
-        float a0, a1;
-        fma2(a0, a1, __uint_as_float(x[2 * cc]), __uint_as_float(x[2 * cc + 1]), c, c, -m_sub, -m_sub);
-        const float p0 = ex2_approx(a0), p1 = ex2_approx(a1);
-        add2(s0, s1, s0, s1, p0, p1);
-        x[cc] = pack_bf16x2(p0, p1);
-      }
+    for (int cc = 0; cc < BN / 2; cc++) {
+      float a0, a1;
+      fma2(a0, a1, __uint_as_float(x[2 * cc]), __uint_as_float(x[2 * cc + 1]), c, c, -m_sub, -m_sub);
+      const float p0 = ex2_approx(a0), p1 = ex2_approx(a1);
+      add2(s0, s1, s0, s1, p0, p1);
+      x[cc] = pack_bf16x2(p0, p1);
     }
     l += s0 + s1;
     // P (bf16, two per column) replaces the first BN/2 columns of S.
-    if (!(SPLIT_PST && !poly)) tmem_st32(t_s, x);
+    tmem_st32(t_s, x);
     tmem_st32(t_s + 32, x + 32);
     tmem_wait_st();
     if (__any_sync(0xffffffffu, need) && it > 0) {
