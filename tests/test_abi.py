@@ -207,3 +207,37 @@ def _host(ta, buf=P << 4, nbytes=1 << 40, do=P, q=P, B=1, Hq=2, Hkv=2, Lq=8, Lk=
 ])
 def test_step_host_rejects_before_any_copy(ta, kw, status):
     assert _host(ta, **kw) == status
+
+
+# ------------------------------------------------------------------ ring-attention block calls
+def test_accumulate_calls_reject_bad_arguments(ta):
+    lib = ta.lib
+    ok = dict(B=1, Hq=2, Hkv=1, Lq=8, Lk=8, d=128)
+    args = lambda **kw: [dict(ok, **kw)[n] for n in ("B", "Hq", "Hkv", "Lq", "Lk", "d")]
+    # attn_fwd_accumulate: missing or misaligned accumulators, bad shapes, bad mask
+    assert lib.attn_fwd_accumulate(P, P, P, 0, P, *args(), 0.1, 1, 0, 1, None) == ta.ATTN_ERR_INVALID_ARG
+    assert lib.attn_fwd_accumulate(P, P, P, P, P + 4, *args(), 0.1, 1, 0, 1, None) == ta.ATTN_ERR_INVALID_ARG
+    assert lib.attn_fwd_accumulate(P, P, P, P, P, *args(d=96), 0.1, 1, 0, 1, None) == ta.ATTN_ERR_UNSUPPORTED
+    assert lib.attn_fwd_accumulate(P, P, P, P, P, *args(Hq=3, Hkv=2), 0.1, 1, 0, 1, None) == ta.ATTN_ERR_INVALID_ARG
+    assert lib.attn_fwd_accumulate(P, P, P, P, P, *args(), 0.1, 4, 0, 1, None) == ta.ATTN_ERR_INVALID_ARG
+    assert lib.attn_fwd_accumulate(0, 0, 0, P, P, *args(Lq=0), 0.1, 1, 0, 1, None) == ta.ATTN_OK
+    # attn_fwd_accumulate_finalize
+    assert lib.attn_fwd_accumulate_finalize(P, P, 0, P, 1, 2, 8, 128, None) == ta.ATTN_ERR_INVALID_ARG
+    assert lib.attn_fwd_accumulate_finalize(P, P, P, P, 1, 2, 8, 72, None) == ta.ATTN_ERR_UNSUPPORTED
+    assert lib.attn_fwd_accumulate_finalize(0, 0, 0, 0, 0, 2, 8, 128, None) == ta.ATTN_OK
+    # attn_bwd_accumulate: accumulators and workspace
+    ws = 1 << 20
+    assert lib.attn_bwd_accumulate(P, P, P, P, P, 0, P, *args(), 0.1, 1, 0, 1, P, ws, None) == ta.ATTN_ERR_INVALID_ARG
+    assert lib.attn_bwd_accumulate(P, P, P, P, P, P, P + 8, *args(), 0.1, 1, 0, 1, P, ws, None) == \
+        ta.ATTN_ERR_INVALID_ARG
+    assert lib.attn_bwd_accumulate(P, P, P, P, P, P, P, *args(), 0.1, 1, 0, 1, P, 16, None) == ta.ATTN_ERR_INVALID_ARG
+    assert lib.attn_bwd_accumulate(P, P, P, P, P, P, P, *args(), 0.1, 1, 0, 1, 0, ws, None) == ta.ATTN_ERR_INVALID_ARG
+    # attn_accumulator_to_bf16
+    assert lib.attn_accumulator_to_bf16(P, P, 0, None) == ta.ATTN_OK
+    assert lib.attn_accumulator_to_bf16(0, P, 16, None) == ta.ATTN_ERR_INVALID_ARG
+    assert lib.attn_accumulator_to_bf16(P + 4, P, 16, None) == ta.ATTN_ERR_INVALID_ARG
+
+
+def test_step_host_fail_hook_validates(ta):
+    assert ta.lib.attn_selftest_step_host_fail_at(-2) == ta.ATTN_ERR_INVALID_ARG
+    assert ta.lib.attn_selftest_step_host_fail_at(-1) == ta.ATTN_OK
