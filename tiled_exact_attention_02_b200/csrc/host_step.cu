@@ -24,7 +24,10 @@
 
 namespace {
 
-constexpr int kTargetChunks = 8;
+#ifndef TEA_STEP_CHUNKS
+#define TEA_STEP_CHUNKS 8
+#endif
+constexpr int kTargetChunks = TEA_STEP_CHUNKS;
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
