@@ -5,14 +5,17 @@ Each case draws its shape and mask from a fixed seed: batch 1-3, group size
 alignment none / top-left / bottom-right, an optional window, optional
 global keys or block-sparse mask, and optional per-sequence lengths.  The
 draws are plain numpy from the case index, so a failure names a reproducible
-problem.  Tolerances are those of the other parity tests.
+problem.  Tolerances are those of the other parity tests, with the O max-abs
+bound max(1e-2, 2^-8 max|V|) (see tests/_util.py o_maxabs_bound): random
+shapes reach rows of few keys with |V| near 3, where the bf16 rounding of P
+and of O alone can pass 1e-2.
 """
 
 import numpy as np
 import pytest
 
 import oracle
-from synth import make_shape_inputs
+from synth import bf16_bits_to_f32, make_shape_inputs
 from tests._util import check_grad, check_lse, check_o, to_dev, to_f64
 
 pytestmark = pytest.mark.gpu
@@ -68,7 +71,8 @@ def test_random_problem(ta, i):
     assert st == 0, f"device error {st} at site {site}"
     what = f"case {i}: B={B} Hq={Hq} Hkv={Hkv} Lq={Lq} Lk={Lk} d={d} causal={causal} window={window} {extra}"
     ro, rl = oracle.attn_fwd(x["q"], x["k"], x["v"], scale, causal, window, **extra)
-    check_o(to_f64(o), ro, what + " O")
+    vmax = float(np.max(np.abs(bf16_bits_to_f32(x["v"])))) if x["v"].size else 0.0
+    check_o(to_f64(o), ro, what + " O", vmax=vmax)
     check_lse(to_f64(lse), rl, what + " LSE")
     rq, rk, rv = oracle.attn_bwd(x["q"], x["k"], x["v"], x["do"], scale, causal, window, **extra)
     check_grad(to_f64(dq), rq, what + " dQ")
