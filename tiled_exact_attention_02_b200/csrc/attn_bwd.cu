@@ -24,10 +24,9 @@
 // so that one thread per key turns a row of S^T into P^T and dS^T, and the
 // bf16 P^T and dS^T, written once to shared memory, serve both as the K-major
 // A operand of dV/dK and as the MN-major operand of dQ.
-// Warp roles (512 threads): warp 0 TMA, warps 1 and 2 MMA issuers, warp 3
-// forwards the landing of each Q/dO tile to the issuers, warps 4-7 and 8-11
-// the per-key softmax gradient (each group takes half of a step's query
-// columns), warps 12-15 the dQ drain.  Tensor memory at d = 128:
+// Warp roles (512 threads): warp 0 TMA, warps 1 and 2 MMA issuers, warps 4-7
+// and 8-11 the per-key softmax gradient (each group takes half of a step's
+// query columns), warps 12-15 the dQ drain.  Tensor memory at d = 128:
 // S^T | dP^T | dV | dK | dQ^T | P^T | dS^T = 512 columns.  Q/dO tiles stream
 // through a 3-stage ring.
 #include <cuda.h>
@@ -84,10 +83,13 @@ struct Cfg {
 // Barriers.  The MMA issuer pays for every wait and commit with tensor-core
 // idle time (its issue queue is shallow), so each of its waits covers
 // everything the next MMA group needs:
-//   q_land[stage]    Q/dO of a step landed (TMA bytes; 1 arrival by the producer)
-//   sq_ready[stage]  Q/dO of a step landed (1 arrival by the landing forwarder,
-//                    after q_land) and the previous step's S^T/dP^T were read
-//                    out (8 gradient warps)
+//   q_land[stage]    Q/dO of a step landed (TMA bytes; 1 arrival by the
+//                    producer); it counts only the producer's copies, so the
+//                    producer can wait for exactly those before the CTA exits
+//   sq_ready[stage]  the previous step's S^T/dP^T were read out (8 gradient
+//                    warps); the S^T/dP^T issuer waits on q_land first (by
+//                    then the copy has almost always landed, so that wait is
+//                    off the critical path) and then on this
 //   grad_ready[2]    P^T/dS^T of a step written (8 gradient warps) and the
 //                    previous step's dQ read out of TMEM (4 drain warps)
 //   sdp_full         S^T/dP^T of a step complete
@@ -192,19 +194,6 @@ __device__ void producer(const BwdParams& P, const Unit& u, uint8_t* smem, Bars&
     mbar_wait_ignore_abort(&bars.q_land[j % C::NQS], (j / C::NQS) & 1, g);
 }
 
-// Passes the landing of each step's Q/dO tiles (q_land) on to sq_ready, which
-// also collects the gradient warps' arrivals: the issuer of S^T/dP^T then
-// waits on one barrier per step, and the producer keeps a barrier that counts
-// only its own copies, for an exact drain after an abort.
-template <int D>
-__device__ void land_forwarder(const Unit& u, Bars& bars, const WaitGuard& g) {
-  using C = Cfg<D>;
-  for (int i = 0; i < u.n_steps; i++) {
-    const int st = i % C::NQS;
-    if (!mbar_wait(&bars.q_land[st], (i / C::NQS) & 1, g, 2)) return;
-    mbar_arrive(&bars.sq_ready[st]);
-  }
-}
 
 // ------------------------------------------------------------------ MMA issuer
 // Two issuing threads keep the tensor core fed: each mbarrier wait costs the
@@ -259,6 +248,7 @@ __device__ void mma_issuer(const BwdParams& P, const Unit& u, uint8_t* smem, Bar
     if (!mbar_wait(&bars.kv_full, 0, g, 10)) goto done;
     for (int i = 0; i < u.n_steps; i++) {
       // Q/dO of step i landed and S^T/dP^T of step i-1 read out.
+      if (!mbar_wait(&bars.q_land[i % C::NQS], (i / C::NQS) & 1, g, 11)) goto done;
       if (!mbar_wait(&bars.sq_ready[i % C::NQS], (i / C::NQS) & 1, g, 12)) goto done;
       tc_fence_after();
       issue_sdp(i);
@@ -646,7 +636,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kernel(const __grid_const
     bars.abort_flag = 0;
     mbar_init(&bars.kv_full, 1);
     for (int s = 0; s < C::NQS; s++) {
-      mbar_init(&bars.sq_ready[s], 1 + 8);  // landing forwarder + 8 gradient warps
+      mbar_init(&bars.sq_ready[s], 8);  // 8 gradient warps
       mbar_init(&bars.q_empty[s], 1);
       mbar_init(&bars.q_land[s], 1);
     }
@@ -685,8 +675,6 @@ __global__ void __launch_bounds__(THREADS, 1) attn_bwd_kernel(const __grid_const
       if (lane == 0) mma_issuer<D, 0>(P, u, smem, bars, tmem, g);
     } else if (warp == 2) {
       if (lane == 0) mma_issuer<D, 1>(P, u, smem, bars, tmem, g);
-    } else {
-      if (lane == 0) land_forwarder<D>(u, bars, g);
     }
   } else if (warp < 12) {
     regs_set<RG, LAUNCH_REGS>();
