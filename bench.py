@@ -49,6 +49,9 @@ def parse():
     ap.add_argument("--all-configs", action="store_true",
                     help="time attn_fwd and the backward on every workload (one JSON line each); not the bench line")
     ap.add_argument("--workload", default=None, help="with --all-configs: only this workload")
+    ap.add_argument("--ring-blocks", type=int, default=0, metavar="N",
+                    help="time one rank's block kernels of ring attention over N ranks (zigzag cut), all steps "
+                         "run on this GPU without the exchange; not the bench line")
     return ap.parse_args()
 
 
@@ -334,12 +337,91 @@ def all_configs(args):
         torch.cuda.empty_cache()
 
 
+def ring_blocks(args):
+    """One rank's compute in ring attention over N ranks (the zigzag cut gives
+    every rank the same work): the forward and backward block calls of its N
+    steps, timed with CUDA events on this GPU, on a causal sequence of 32768
+    positions (B=1, Hq=32, Hkv=8, d=128).  The K/V chunks a rank would
+    receive are taken from the full tensors, so no exchange is timed.  The
+    monolithic forward and backward of the whole problem on this GPU, divided
+    by N, is the comparison: it is what one GPU's share would cost without
+    the cut into blocks."""
+    import numpy as np
+    import torch
+    import tiled_exact_attention_02_b200 as ta
+    from tiled_exact_attention_02_b200 import ring
+    from synth import Workload
+    N = args.ring_blocks
+    w = Workload("ring_causal_32768", 1, 32, 8, 32768, 32768, 128, True, backward=True, seed=49)
+    x = make_inputs(w)
+    dev = lambda bits: torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).cuda()
+    full = {n: dev(x[n]) for n in ("q", "k", "v", "do")}
+    sh = {n: [ring.shard(full[n], r, N, "zigzag") for r in range(N)] for n in full}
+    ops = ring.CudaOps(ta.lib)
+    r = 0  # every rank has the same work under the zigzag cut
+
+    def timed(fn, reps=5):
+        ts = []
+        for it in range(reps + 2):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            if it >= 2:
+                ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    state = {}
+
+    def fwd():
+        f = ring.RingForwardRank(sh["q"][r], r, N, "zigzag", True, w.scale, ops)
+        for t in range(N):
+            src = (r - t) % N
+            f.step(t, sh["k"][src], sh["v"][src])
+        state["o"], state["lse"] = f.result()
+
+    def bwd():
+        bw = ring.RingBackwardRank(sh["q"][r], state["o"], state["lse"], sh["do"][r], r, N, "zigzag", True, w.scale,
+                                   ops, k_like=sh["k"][r])
+        acc = [torch.empty(sh["k"][r].shape, dtype=torch.float32, device="cuda") for _ in range(2)]
+        for t in range(N):
+            src = (r - t) % N
+            bw.step(t, sh["k"][src], sh["v"][src], acc[0], acc[1])
+        bw.dq()
+        dk, dv = torch.empty_like(sh["k"][r]), torch.empty_like(sh["v"][r])
+        ops.to_bf16(acc[0], dk)
+        ops.to_bf16(acc[1], dv)
+
+    f_ms = timed(fwd)
+    b_ms = timed(bwd)
+    q, k, v, do = (full[n] for n in ("q", "k", "v", "do"))
+    o, lse = ta.attention(q, k, v, True, 0, w.scale)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(ta.bwd_workspace_size(w.B, w.Hq, w.Hkv, w.Lq, w.Lk, w.d), dtype=torch.uint8, device="cuda")
+    mf_ms = timed(lambda: ta.fwd(q, k, v, o, lse, True, 0, w.scale))
+    mb_ms = timed(lambda: ta.bwd(q, k, v, o, lse, do, dq, dk, dv, ws, True, 0, w.scale))
+    st, site = ta.device_error()
+    if st != 0:
+        raise SystemExit(f"device error {st} at site {site}")
+    fl_f, fl_b = w.fwd_flops() / N, w.bwd_flops() / N
+    print(json.dumps({
+        "ring_blocks": N, "layout": "zigzag", "workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.Lq,
+        "d": w.d, "causal": True, "rank_chunks_rows": w.Lq // (2 * N),
+        "rank_fwd_ms": f_ms, "rank_fwd_tflops": fl_f / f_ms / 1e9,
+        "rank_bwd_ms": b_ms, "rank_bwd_tflops": fl_b / b_ms / 1e9,
+        "monolithic_fwd_ms_over_N": mf_ms / N, "monolithic_bwd_ms_over_N": mb_ms / N,
+        "block_efficiency_fwd": (mf_ms / N) / f_ms, "block_efficiency_bwd": (mb_ms / N) / b_ms}), flush=True)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
     if args.all_configs:
         return all_configs(args)
+    if args.ring_blocks:
+        return ring_blocks(args)
 
     import torch
     if not torch.cuda.is_available():
