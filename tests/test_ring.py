@@ -366,3 +366,19 @@ def test_accumulate_entry_points_match_the_whole_problem():
     check_grad(to_f64(dq) / 2, rq, "dQ")  # every block's dQ was added twice
     check_grad(np.concatenate([d.double().cpu().numpy() for d in dks], axis=2), rk, "dK")
     check_grad(np.concatenate([d.double().cpu().numpy() for d in dvs], axis=2), rv, "dV")
+
+
+def test_single_process_ring_needs_no_process_group():
+    """Without torch.distributed initialised the ring has one rank: its one
+    step is the whole problem (float64 stand-ins, against the oracle)."""
+    ring = _ring()
+    x = make_shape_inputs(1, 2, 1, 40, 40, 8, seed=3, with_do=True)
+    full = {n: torch.from_numpy(bf16_bits_to_f32(x[n]).astype(np.float64)) for n in ("q", "k", "v", "do")}
+    q, k, v, do = (ring.shard(full[n], 0, 1, "zigzag") for n in ("q", "k", "v", "do"))
+    ops = F64Ops()
+    o, lse = ring.ring_attention_forward(q, k, v, causal=True, scale=8 ** -0.5, ops=ops)
+    dq, dk, dv = ring.ring_attention_backward(q, k, v, o, lse, do, causal=True, scale=8 ** -0.5, ops=ops)
+    ro, rl = oracle.attn_fwd(x["q"], x["k"], x["v"], 8 ** -0.5, True, 0)
+    rq, rk, rv = oracle.attn_bwd(x["q"], x["k"], x["v"], x["do"], 8 ** -0.5, True, 0)
+    for g, r in zip((o, lse, dq, dk, dv), (ro, rl, rq, rk, rv)):
+        np.testing.assert_allclose(ring.unshard([g], 1, "zigzag").numpy(), r, rtol=1e-10, atol=1e-12)

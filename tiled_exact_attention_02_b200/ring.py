@@ -260,6 +260,8 @@ class RingBackwardRank:
 
 def _ring_peers(group):
     import torch.distributed as dist
+    if group is None and not (dist.is_available() and dist.is_initialized()):
+        return 0, 1, 0, 0  # a single process: the ring has one rank and no exchange
     world = dist.get_world_size(group)
     rank = dist.get_rank(group)
     g = (lambda r: dist.get_global_rank(group, r)) if group is not None else (lambda r: r)
