@@ -385,6 +385,21 @@ ATTN_API int attn_get_device_error(void* stream, int* site);
 ATTN_API int attn_selftest_wait_timeout(int64_t limit_ns, void* stream);
 
 /*
+ * Self-test of the backward kernel's abort path: attn_bwd (arguments as
+ * there) in which the gradient warps withhold their arrival for step
+ * `stall_step` of every CTA that has that many steps, so the MMA issuer's
+ * bounded wait runs out after `limit_ns` (1 ns .. 10 s).  The CTA then lets
+ * every copy, MMA and reduce it started finish, frees its tensor memory and
+ * exits; attn_get_device_error() reports ATTN_ERR_TIMEOUT and the outputs are
+ * undefined.  Nothing faults or hangs on the GPU, and the context stays
+ * usable.  No counterpart on the pages: it exists to test failure handling.
+ */
+ATTN_API int attn_selftest_bwd_abort(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                                     const void* dO, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Lq,
+                                     int Lk, int d, float scale, int causal, int window, int stall_step,
+                                     int64_t limit_ns, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Self-test of attn_step_host's error path: the next attn_step_host call (on
  * any thread) behaves as if the copy in of chunk `chunk` had failed, after
  * the earlier chunks' copies and kernels were queued, and returns

@@ -94,6 +94,8 @@ def _load() -> ctypes.CDLL:
     lib.attn_bwd_accumulate.restype = i
     lib.attn_accumulator_to_bf16.argtypes = [vp, vp, sz, vp]
     lib.attn_accumulator_to_bf16.restype = i
+    lib.attn_selftest_bwd_abort.argtypes = [vp] * 9 + [i] * 6 + [f, i, i, i, ctypes.c_int64, vp, sz, vp]
+    lib.attn_selftest_bwd_abort.restype = i
     lib.attn_selftest_step_host_fail_at.argtypes = [i]
     lib.attn_selftest_step_host_fail_at.restype = i
     return lib

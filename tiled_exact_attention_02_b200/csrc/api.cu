@@ -324,7 +324,7 @@ static int bwd_main_impl(const void* q, const void* k, const void* v, const floa
                          void* dv, const int* lens_q, const int* lens_k, int B, int Hq, int Hkv, int Lq, int Lk, int d,
                          float scale, int causal, int window, int gh, int gt, int sb, void* workspace,
                          size_t workspace_bytes, void* stream, float* dk_acc = nullptr, float* dv_acc = nullptr,
-                         int dkv_init = 0) {
+                         int dkv_init = 0, int stall_at = 0, uint64_t limit_ns = kWaitLimitNs) {
   int st = check_shape(B, Hq, Hkv, Lq, Lk, d, scale, causal, window);
   if (st == ATTN_OK && (gh < 0 || gt < 0 || sb < 0 || sb > (1 << 28))) st = ATTN_ERR_INVALID_ARG;
   if (st != ATTN_OK) return st;
@@ -390,8 +390,9 @@ static int bwd_main_impl(const void* q, const void* k, const void* v, const floa
   P.scale = scale;
   P.scale_log2 = scale * 1.4426950408889634f;
   P.n_units = B * Hkv * ((Lk + 127) / 128);
+  P.stall_at = stall_at;
   if ((st = get_err_word(&P.err)) != ATTN_OK) return st;
-  P.limit_ns = kWaitLimitNs;
+  P.limit_ns = limit_ns;
   const cudaError_t e = launch_bwd(P, s);
   return e == cudaSuccess ? ATTN_OK : cuda_fail("attn_bwd_main launch", e);
 }
@@ -554,6 +555,23 @@ int attn_get_device_error(void* stream, int* site) {
   if (e != cudaSuccess) return cuda_fail("clear error word", e);
   if (site) *site = word >> 8;
   return (word & 0xFF) == DEV_TIMEOUT ? ATTN_ERR_TIMEOUT : ATTN_OK;
+}
+
+int attn_selftest_bwd_abort(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                            const void* dO, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Lq, int Lk, int d,
+                            float scale, int causal, int window, int stall_step, int64_t limit_ns, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  if (stall_step < 0 || limit_ns <= 0 || limit_ns > (int64_t)10000000000ll) return ATTN_ERR_INVALID_ARG;
+  int st = check_shape(B, Hq, Hkv, Lq, Lk, d, scale, causal, window);
+  if (st != ATTN_OK) return st;
+  if (B == 0 || Hq == 0 || Lq == 0 || Lk == 0) return ATTN_ERR_INVALID_ARG;
+  if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return ATTN_ERR_INVALID_ARG;
+  if ((st = attn_bwd_preprocess(o, dO, B, Hq, Lq, d, workspace, workspace_bytes, stream)) != ATTN_OK) return st;
+  if ((st = bwd_main_impl(q, k, v, lse, dO, dk, dv, nullptr, nullptr, B, Hq, Hkv, Lq, Lk, d, scale, causal, window, 0,
+                          0, 0, workspace, workspace_bytes, stream, nullptr, nullptr, 0, stall_step + 1,
+                          (uint64_t)limit_ns)) != ATTN_OK)
+    return st;
+  return attn_bwd_finalize(dq, B, Hq, Lq, d, scale, workspace, workspace_bytes, stream);
 }
 
 int attn_selftest_wait_timeout(int64_t limit_ns, void* stream) {

@@ -466,7 +466,7 @@ __device__ void grad_rows(const BwdParams& P, const Unit& u, uint8_t* smem, Bars
     fence_proxy_async_smem();  // generic-proxy stores -> tensor-core reads
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive(&bars.grad_ready[i & 1]);
+    if (lane == 0 && i + 1 != P.stall_at) mbar_arrive(&bars.grad_ready[i & 1]);
   }
 
   // Epilogue: group 0 writes dV, group 1 writes scale * dK for its key.
@@ -585,7 +585,7 @@ __device__ void dq_drain(const BwdParams& P, const Unit& u, uint8_t* smem, Bars&
       for (int hh = 0; hh < 2; hh++, half++) {
         const int b = half & 1, use = half >> 1;
         // The reduce of this buffer's previous use must have read it.
-        if (use > 0 && !mbar_wait(&bars.stg_free[b], (use - 1) & 1, g, 31)) return;
+        if (use > 0 && !mbar_wait(&bars.stg_free[b], (use - 1) & 1, g, 31)) goto out;
         float* col = reinterpret_cast<float*>(stg + b * 16384) + t;
 #pragma unroll
         for (int qq = 0; qq < 32; qq++) col[qq * 128] = __uint_as_float(r[32 * hh + qq]);
@@ -593,7 +593,7 @@ __device__ void dq_drain(const BwdParams& P, const Unit& u, uint8_t* smem, Bars&
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars.stg_full[b]);
         if (t == 0) {
-          if (!mbar_wait(&bars.stg_full[b], use & 1, g, 32)) return;
+          if (!mbar_wait(&bars.stg_full[b], use & 1, g, 32)) goto out;
           // Query rows past Lq are clipped by the tensor bounds.
           tma_reduce_add_3d(&P.tm_dq, stg + b * 16384, 0, q0 + 32 * hh, bh);
           bulk_commit();
@@ -610,7 +610,10 @@ __device__ void dq_drain(const BwdParams& P, const Unit& u, uint8_t* smem, Bars&
       }
     }
   }
-  if (D == 128 && t == 0) bulk_wait_all();  // every reduce complete before the CTA exits
+out:
+  // Every reduce this thread started is complete before the CTA may exit (also
+  // after an abort, so that no bulk copy still reads the staging buffer).
+  if (D == 128 && t == 0) bulk_wait_all();
 }
 
 // ------------------------------------------------------------------ kernel

@@ -51,6 +51,10 @@ struct BwdParams {
   float* dk_acc;
   float* dv_acc;
   int dkv_init;
+  // Self-test of the abort path (0 otherwise): with k > 0 the gradient warps
+  // withhold their arrival for step k - 1, so a bounded wait runs out and the
+  // kernel takes its abort path (attn_selftest_bwd_abort).
+  int stall_at;
   float scale;
   float scale_log2;
   int n_units;        // CTAs: B * Hkv * key tiles
