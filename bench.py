@@ -275,8 +275,10 @@ def run_reference(args):
 
 def all_configs(args):
     """Forward and backward times of every workload on one GPU (CUDA-event
-    medians), one JSON line each.  The backward runs with a dO drawn for the
-    workload when it has none.  Inputs of the small case fit in L2."""
+    medians; calls shorter than 1 ms timed in back-to-back groups), one JSON
+    line each.  The
+    backward runs with a dO drawn for the workload when it has none.  Inputs
+    of the small case fit in L2; the others are larger than L2."""
     import numpy as np
     import torch
     import tiled_exact_attention_02_b200 as ta
@@ -294,15 +296,27 @@ def all_configs(args):
         ws = torch.empty(ta.bwd_workspace_size(w.B, w.Hq, w.Hkv, w.Lq, w.Lk, w.d), dtype=torch.uint8, device="cuda")
 
         def timed(fn, n):
+            # Each sample brackets `rep` back-to-back calls (about 1 ms of work,
+            # at most 10 calls), so for short kernels the host work of one call
+            # overlaps the kernels of the one before it and the time is the
+            # device's; the sample's mean per call, median over samples.
+            fn()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            rep = max(1, min(10, int(1.0 / max(a.elapsed_time(b), 1e-3))))
             ts = []
             for it in range(n + 3):
                 a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 a.record()
-                fn()
+                for _ in range(rep):
+                    fn()
                 b.record()
                 torch.cuda.synchronize()
                 if it >= 3:
-                    ts.append(a.elapsed_time(b))
+                    ts.append(a.elapsed_time(b) / rep)
             return statistics.median(ts)
 
         n = max(5, min(args.steps, 50))

@@ -180,11 +180,16 @@ ATTN_API int attn_fwd_split(const void* q, const void* k, const void* v, void* o
  * problem or invalid sizes. */
 ATTN_API size_t attn_fwd_split_workspace_size(int B, int Hq, int Hkv, int Lq, int Lk, int d, int n_split);
 
-/* A slice count for this problem on the current device: the count with the
- * least estimated time when CTAs run in waves of one per SM and each costs its
- * slice's 128-key tiles plus about two tiles of fixed work; no slice shorter
- * than two tiles, at most 64; 1 when splitting would not help.  Host-only (no
- * launch). */
+/* A slice count for this problem on the current device; no slice shorter
+ * than two 128-key tiles, at most 64; 1 when splitting would not help.
+ * Host-only (no launch).
+ * - Few query rows per kv group (the units pack them into one slot that both
+ *   slots share: decoding): the most slices that still fit in one wave of one
+ *   CTA per SM.  These CTAs stream K/V at the HBM rate; a second wave only
+ *   adds fixed work and a tail.
+ * - Otherwise: the count with the least estimated time when CTAs run in waves
+ *   of one per SM and each costs its slice's key tiles plus about two tiles of
+ *   fixed work. */
 ATTN_API int attn_fwd_split_default(int B, int Hq, int Hkv, int Lq, int Lk, int d, int causal, int window);
 
 /*

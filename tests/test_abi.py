@@ -110,9 +110,18 @@ def test_fwd_split_default_is_in_range(ta):
     assert 1 <= d(8, 32, 8, 1, 32768, 128, 2, 0) <= 64
     assert d(2, 32, 32, 4096, 4096, 128, 1, 0) == 1     # a full grid does not
     assert d(1, 2, 2, 1, 100, 64, 2, 0) == 1            # a single key tile does not
-    # 16 queries per head over 32768 keys, G = 4: 32 packed units of 256 key tiles.  With 148 SMs (the
-    # default without a device) 9 slices (288 CTAs, two waves) give the least modelled time.
-    assert d(4, 32, 8, 16, 32768, 128, 2, 0) == 9
+    # Alternating-slot plans (few query rows per kv group) take the most slices that fit one wave of one CTA
+    # per SM (148 SMs, the default without a device).  16 queries per head over 32768 keys, G = 4: 32 packed
+    # units -> 4 slices (128 CTAs); 8 units -> 18; 64 units -> 2; 128 units -> 1.
+    assert d(4, 32, 8, 16, 32768, 128, 2, 0) == 4
+    assert d(1, 32, 8, 1, 32768, 128, 2, 0) == 18
+    assert d(8, 32, 8, 16, 32768, 128, 2, 0) == 2
+    assert d(16, 32, 8, 1, 4096, 128, 2, 0) == 1
+    # ... but never a slice shorter than two key tiles: 8 units over 1024 keys (8 tiles) -> 4.
+    assert d(1, 32, 8, 1, 1024, 128, 2, 0) == 4
+    # Units with two slots of different rows (128 queries per head, G = 4: 32 units of 256 key tiles) are
+    # compute-bound: the modelled waves give 9 slices (288 CTAs, two waves).
+    assert d(1, 32, 8, 128, 32768, 128, 2, 0) == 9
 
 
 def _split(ta, n_split=4, ws=P, wsb=1 << 20, **kw):
