@@ -103,10 +103,45 @@ __device__ __forceinline__ bool walk_has(const Segs& s, int j) {
   else return j >= s.lo[1] && j < s.hi[1];
 }
 
+// Key tiles of query rows [q0, q1) as a walk.  Without global tokens the walk
+// is the band alone (range 1), built directly: the general form's range
+// merging is a long chain of dependent integer operations that every thread
+// of a CTA runs before its first copy can start.
+template <bool W>
+__device__ __forceinline__ Segs tile_walk(const Problem& ps, int q0, int q1) {
+  if constexpr (W) {
+    return kv_tile_segs(ps, q0, q1, BN);
+  } else {
+    Segs s;
+    kv_tile_range(ps, q0, q1, BN, s.lo[1], s.hi[1]);
+    return s;
+  }
+}
+
+// The union of the two slots' walks (what the CTA streams); without global
+// tokens the tiles between the two bands' ends.
+template <bool W>
+__device__ __forceinline__ Segs union_walk(const Segs& a, const Segs& b) {
+  Segs u = a;
+  if constexpr (W) {
+    u.unite(b);
+  } else if (b.lo[1] < b.hi[1]) {
+    if (u.lo[1] < u.hi[1]) {
+      u.lo[1] = imin(u.lo[1], b.lo[1]);
+      u.hi[1] = imax(u.hi[1], b.hi[1]);
+    } else {
+      u.lo[1] = b.lo[1];
+      u.hi[1] = b.hi[1];
+    }
+  }
+  return u;
+}
+
 // Packed rows (short queries): row r of kv group (b, kvh) is query r % Lq of
 // head kvh*G + r / Lq, i.e. Q read as [B*Hkv, G*Lq, d]; each unit takes two
 // consecutive 128-row tiles of a group.  A tile inside one head sees the key
 // tiles of its own query rows, a tile across heads those of all Lq rows.
+template <bool W>
 __device__ __forceinline__ Unit decode_unit_packed(const FwdParams& P, int idx) {
   const Problem& p = P.prob;
   Unit u;
@@ -127,13 +162,12 @@ __device__ __forceinline__ Unit decode_unit_packed(const FwdParams& P, int idx) 
     if (r0 >= r1) {
       u.seg[s] = Segs{};
     } else if (r0 / p.Lq != (r1 - 1) / p.Lq) {
-      u.seg[s] = kv_tile_segs(ps, 0, p.Lq, BN);
+      u.seg[s] = tile_walk<W>(ps, 0, p.Lq);
     } else {
-      u.seg[s] = kv_tile_segs(ps, r0 % p.Lq, (r1 - 1) % p.Lq + 1, BN);
+      u.seg[s] = tile_walk<W>(ps, r0 % p.Lq, (r1 - 1) % p.Lq + 1);
     }
   }
-  u.useg = u.seg[0];
-  u.useg.unite(u.seg[1]);
+  u.useg = union_walk<W>(u.seg[0], u.seg[1]);
   return u;
 }
 
@@ -149,9 +183,10 @@ __device__ __forceinline__ void make_alternating(Unit& u) {
   u.useg = u.seg[0];
 }
 
+template <bool W>
 __device__ __forceinline__ Unit decode_unit(const FwdParams& P, int idx) {
   if (P.packed) {
-    Unit u = decode_unit_packed(P, idx);
+    Unit u = decode_unit_packed<W>(P, idx);
     u.alt = 0;
     if (P.alternate) make_alternating(u);
     return u;
@@ -188,10 +223,9 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& P, int idx) {
   }
   u.kvh = u.head[0] / G;
   const Problem ps = seq_problem(p, u.b);  // this sequence's lengths (padded batches)
-  u.seg[0] = kv_tile_segs(ps, u.q0[0], u.q0[0] + BM, BN);
-  u.seg[1] = kv_tile_segs(ps, u.q0[1], u.q0[1] + BM, BN);
-  u.useg = u.seg[0];
-  u.useg.unite(u.seg[1]);
+  u.seg[0] = tile_walk<W>(ps, u.q0[0], u.q0[0] + BM);
+  u.seg[1] = tile_walk<W>(ps, u.q0[1], u.q0[1] + BM);
+  u.useg = union_walk<W>(u.seg[0], u.seg[1]);
   u.alt = 0;
   if (P.alternate) make_alternating(u);
   return u;
@@ -205,11 +239,11 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& P, int idx) {
 template <bool W>
 __device__ __forceinline__ Unit decode_unit_split(const FwdParams& P, int idx) {
   if (P.n_split <= 1) {
-    Unit u = decode_unit(P, idx);
+    Unit u = decode_unit<W>(P, idx);
     u.split = 0;
     return u;
   }
-  Unit u = decode_unit(P, idx / P.n_split);
+  Unit u = decode_unit<W>(P, idx / P.n_split);
   u.split = idx % P.n_split;
   const int n = walk_count<W>(u.useg);
   const int p0 = (int)((long long)u.split * n / P.n_split);
