@@ -82,20 +82,24 @@ struct Unit {
   Segs useg;         // their union: the tiles the CTA streams
   int split;         // key-range slice of a split problem (0 otherwise)
   int alt;           // 1: both slots hold the same rows and take alternate key tiles of one range
+  int down;          // 1: the walk runs from its last tile down (block-sparse masks, no global tokens)
 };
 
 // Walk accessors.  W = false (no global tokens): the walk is the band alone,
 // which kv_tile_segs always keeps in range 1, so every accessor is the plain
-// contiguous-range arithmetic and the rest of Segs is dead code.
+// contiguous-range arithmetic and the rest of Segs is dead code.  Under a
+// block-sparse mask the band is walked from its last tile down (`down`): on a
+// B200 that measured 8% faster for 64-row blocks, while the causal and
+// window workloads measured the same or slower that way, so they walk up.
 template <bool W>
 __device__ __forceinline__ int walk_count(const Segs& s) {
   if constexpr (W) return s.count();
   else return s.hi[1] > s.lo[1] ? s.hi[1] - s.lo[1] : 0;
 }
 template <bool W>
-__device__ __forceinline__ int walk_at(const Segs& s, int t) {
+__device__ __forceinline__ int walk_at(const Segs& s, int t, bool down) {
   if constexpr (W) return s.at(t);
-  else return s.lo[1] + t;
+  else return down ? s.hi[1] - 1 - t : s.lo[1] + t;
 }
 template <bool W>
 __device__ __forceinline__ bool walk_has(const Segs& s, int j) {
@@ -187,6 +191,7 @@ template <bool W>
 __device__ __forceinline__ Unit decode_unit(const FwdParams& P, int idx) {
   if (P.packed) {
     Unit u = decode_unit_packed<W>(P, idx);
+    u.down = !W && P.prob.sparse_block > 0;
     u.alt = 0;
     if (P.alternate) make_alternating(u);
     return u;
@@ -226,6 +231,7 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& P, int idx) {
   u.seg[0] = tile_walk<W>(ps, u.q0[0], u.q0[0] + BM);
   u.seg[1] = tile_walk<W>(ps, u.q0[1], u.q0[1] + BM);
   u.useg = union_walk<W>(u.seg[0], u.seg[1]);
+  u.down = !W && P.prob.sparse_block > 0;
   u.alt = 0;
   if (P.alternate) make_alternating(u);
   return u;
@@ -248,8 +254,13 @@ __device__ __forceinline__ Unit decode_unit_split(const FwdParams& P, int idx) {
   const int n = walk_count<W>(u.useg);
   const int p0 = (int)((long long)u.split * n / P.n_split);
   const int p1 = (int)((long long)(u.split + 1) * n / P.n_split);
-  const int a = p0 < p1 ? walk_at<W>(u.useg, p0) : 0;
-  const int b = p0 < p1 ? walk_at<W>(u.useg, p1 - 1) + 1 : 0;
+  // Tiles between the slice's first and last (either order, as the walk runs).
+  int a = 0, b = 0;
+  if (p0 < p1) {
+    const int ja = walk_at<W>(u.useg, p0, u.down), jb = walk_at<W>(u.useg, p1 - 1, u.down);
+    a = imin(ja, jb);
+    b = imax(ja, jb) + 1;
+  }
   u.useg.clip(a, b);
   u.seg[0].clip(a, b);
   u.seg[1].clip(a, b);
@@ -260,7 +271,8 @@ __device__ __forceinline__ Unit decode_unit_split(const FwdParams& P, int idx) {
 // positions s, s + 2, ... of the one contiguous range.
 template <bool W>
 __device__ __forceinline__ bool active(const Unit& u, int s, int j) {
-  if (!W && u.alt) return walk_has<W>(u.seg[s], j) && ((j - u.seg[s].lo[1]) & 1) == s;
+  if (!W && u.alt)
+    return walk_has<W>(u.seg[s], j) && ((u.down ? u.seg[s].hi[1] - 1 - j : j - u.seg[s].lo[1]) & 1) == s;
   return walk_has<W>(u.seg[s], j);
 }
 template <bool W>
@@ -270,7 +282,8 @@ __device__ __forceinline__ int slot_count(const Unit& u, const Segs& sg, int s) 
 }
 template <bool W>
 __device__ __forceinline__ int slot_at(const Unit& u, const Segs& sg, int s, int i) {
-  return (!W && u.alt) ? sg.lo[1] + 2 * i + s : walk_at<W>(sg, i);
+  if (!W && u.alt) return u.down ? sg.hi[1] - 1 - (2 * i + s) : sg.lo[1] + 2 * i + s;
+  return walk_at<W>(sg, i, u.down);
 }
 
 // ------------------------------------------------------------------ producer
@@ -292,7 +305,7 @@ __device__ void producer(const FwdParams& P, const Unit& u, uint8_t* smem, Bars&
   int issued = 0;
   const int un = walk_count<W>(u.useg);
   for (int t = 0; t < un; t++) {
-    const int j = walk_at<W>(u.useg, t);
+    const int j = walk_at<W>(u.useg, t, u.down);
     for (int which = 0; which < 2; which++) {
       const int r = 2 * t + which;
       const int st = r % C::NST;
@@ -357,7 +370,7 @@ __device__ void mma_issuer(const FwdParams& P, const Unit& u, uint8_t* smem, Bar
 
   {
     // Prologue: S for the first tile of the walk.
-    const int j0 = walk_at<W>(u.useg, 0);
+    const int j0 = walk_at<W>(u.useg, 0, u.down);
     if (!mbar_wait(&bars.kv_full[stage_of(0, 0)], phase_of(0, 0), g, 11)) goto out;
     tc_fence_after();
 #pragma unroll
@@ -367,10 +380,10 @@ __device__ void mma_issuer(const FwdParams& P, const Unit& u, uint8_t* smem, Bar
   }
 
   for (int t = 0; t < un; t++) {
-    const int j = walk_at<W>(u.useg, t);
+    const int j = walk_at<W>(u.useg, t, u.down);
     if (!mbar_wait(&bars.kv_full[stage_of(t, 1)], phase_of(t, 1), g, 12)) goto out;
     const bool next = t + 1 < un;
-    const int jn = next ? walk_at<W>(u.useg, t + 1) : -1;
+    const int jn = next ? walk_at<W>(u.useg, t + 1, u.down) : -1;
     if (next) {
       if (!mbar_wait(&bars.kv_full[stage_of(t + 1, 0)], phase_of(t + 1, 0), g, 13)) goto out;
     }
@@ -719,8 +732,10 @@ __device__ void softmax_slot(const FwdParams& P, const Unit& u, int s, uint8_t* 
 // ------------------------------------------------------------------ kernel
 // W: the problem has global tokens (the key-tile walk may have several ranges).
 // A: alternating slots (launched only for plans that use them, so the other
-// variants carry none of that code).
-template <int D, bool W, bool A>
+// variants carry none of that code).  DN: the walk runs downwards (block-sparse
+// masks; a compile-time choice, since a run-time direction cost about 5% on
+// the causal workloads).
+template <int D, bool W, bool A, bool DN>
 __global__ void __launch_bounds__(THREADS, 1) attn_fwd_kernel(const __grid_constant__ FwdParams P) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -730,6 +745,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_kernel(const __grid_const
   const int lane = threadIdx.x % 32;
   Unit u = decode_unit_split<W>(P, blockIdx.x);
   if (!A || W) u.alt = 0;
+  u.down = DN;  // equal to the decoded value; a constant lets the compiler drop the other direction
   const WaitGuard g{P.err, &bars.abort_flag, P.limit_ns, 0};
 
   if (threadIdx.x == 0) {
@@ -870,22 +886,24 @@ void fwd_plan(const Problem& p, int* n_units, int* pair_heads, int* packed, int*
   if (has_global(p)) *alternate = 0;
 }
 
-template <int D, bool W, bool A>
+template <int D, bool W, bool A, bool DN = false>
 static cudaError_t launch_fwd_d(const FwdParams& P, cudaStream_t stream) {
   constexpr int smem = fwd::Cfg<D>::SMEM;
   static std::atomic<unsigned char> ready[kMaxDevices];
   cudaError_t e = once_per_device(ready, [] {
-    return cudaFuncSetAttribute(fwd::attn_fwd_kernel<D, W, A>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    return cudaFuncSetAttribute(fwd::attn_fwd_kernel<D, W, A, DN>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   });
   if (e != cudaSuccess) return e;
-  fwd::attn_fwd_kernel<D, W, A><<<P.n_units * imax(1, P.n_split), fwd::THREADS, smem, stream>>>(P);
+  fwd::attn_fwd_kernel<D, W, A, DN><<<P.n_units * imax(1, P.n_split), fwd::THREADS, smem, stream>>>(P);
   return cudaGetLastError();
 }
 
 template <int D>
 static cudaError_t launch_fwd_dd(const FwdParams& P, cudaStream_t stream) {
   if (has_global(P.prob)) return launch_fwd_d<D, true, false>(P, stream);
-  return P.alternate ? launch_fwd_d<D, false, true>(P, stream) : launch_fwd_d<D, false, false>(P, stream);
+  const bool down = P.prob.sparse_block > 0;  // as decode_unit sets Unit::down
+  if (P.alternate) return down ? launch_fwd_d<D, false, true, true>(P, stream) : launch_fwd_d<D, false, true>(P, stream);
+  return down ? launch_fwd_d<D, false, false, true>(P, stream) : launch_fwd_d<D, false, false>(P, stream);
 }
 
 cudaError_t launch_fwd(const FwdParams& P, cudaStream_t stream) {
