@@ -148,11 +148,13 @@ __device__ __forceinline__ Unit decode_unit(const BwdParams& P, int idx) {
 }
 
 // Step i of a unit: query head h (global head index) and first query row q0.
+// Each head's query tiles are taken from the last down (under a causal mask
+// the diagonal tile comes last); measured about 1% faster than upwards.
 template <int D>
 __device__ __forceinline__ void step_of(const Unit& u, int i, int& h, int& q0) {
   const int g = i / u.nq;
   h = u.kvh * u.G + g;
-  q0 = (u.qt_lo + i % u.nq) * Cfg<D>::BM;
+  q0 = (u.qt_lo + u.nq - 1 - i % u.nq) * Cfg<D>::BM;
 }
 
 // ------------------------------------------------------------------ producer
