@@ -220,11 +220,17 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& P, int idx) {
     u.head[1] = 2 * hp + 1;
     u.q0[0] = u.q0[1] = qi * BM;
   } else {
-    // Two consecutive row tiles of one head.
+    // Two consecutive row tiles of one head.  The later tile (under a causal
+    // mask the one that sees one more key tile) takes slot 0, whose MMAs the
+    // issuer takes first at each key tile: measured about 2.5% faster on a
+    // causal 4096 workload.  Block-sparse masks (walked downwards) measured
+    // 10% faster the other way round, and with alternating slots slot 0 must
+    // hold the unit's only tile.
+    const bool later_first = !P.alternate && p.sparse_block == 0;
     u.b = hu / p.Hq;
     u.head[0] = u.head[1] = hu % p.Hq;
-    u.q0[0] = qi * 2 * BM;
-    u.q0[1] = qi * 2 * BM + BM;
+    u.q0[0] = qi * 2 * BM + (later_first ? BM : 0);
+    u.q0[1] = qi * 2 * BM + (later_first ? 0 : BM);
   }
   u.kvh = u.head[0] / G;
   const Problem ps = seq_problem(p, u.b);  // this sequence's lengths (padded batches)
