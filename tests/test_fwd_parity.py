@@ -179,6 +179,10 @@ SPARSE = [
     (2, 8, 2, 16, 2000, 128, 2, 0, 300, 1, 0, 0),
     (1, 2, 2, 100, 3000, 128, 0, 0, 256, 4, 0, 0),
     (1, 2, 2, 600, 600, 128, 0, 0, 64, 1, 2, 3),
+    # Two row tiles per unit (no alternating slots) cut into key-range slices: the
+    # slices of a walk that runs downwards.
+    (1, 2, 2, 700, 900, 128, 0, 0, 64, 3, 0, 0),
+    (2, 4, 4, 520, 520, 64, 1, 0, 100, 2, 0, 0),
 ]
 
 
