@@ -176,21 +176,29 @@ __host__ __device__ inline void row_key_range(const Problem& p, int i, int& key_
   }
 }
 
-// Key tiles [lo, hi) (tiles of bn keys) holding any key visible to any query
-// row in [q0, q1).  Empty range: lo == hi == 0.
-__host__ __device__ inline void kv_tile_range(const Problem& p, int q0, int q1, int bn, int& lo, int& hi) {
+// Keys [key_lo, key_hi) spanning every key visible to any query row in
+// [q0, q1) (the band; global keys not included).  Empty: key_lo >= key_hi.
+__host__ __device__ inline void kv_key_range(const Problem& p, int q0, int q1, int& key_lo, int& key_hi) {
   q1 = imin(q1, p.Lq);
-  lo = hi = 0;
+  key_lo = key_hi = 0;
   if (q0 >= q1) return;
   const int off = diag_off(p);
   // The last row reaches furthest forward, the first row furthest back.
-  int key_hi = p.causal ? imin(p.Lk, q1 + off) : (p.window > 0 ? imin(p.Lk, q1 - 1 + p.window) : p.Lk);
-  int key_lo = p.window > 0 ? imax(0, q0 + off - p.window + 1) : 0;
+  key_hi = p.causal ? imin(p.Lk, q1 + off) : (p.window > 0 ? imin(p.Lk, q1 - 1 + p.window) : p.Lk);
+  key_lo = p.window > 0 ? imax(0, q0 + off - p.window + 1) : 0;
   if (p.sparse_block > 0) {
     // Both ends of every mask's key range only grow with the row.
     key_lo = imax(key_lo, sparse_key_lo(p, q0));
     key_hi = imin(key_hi, sparse_key_hi(p, q1 - 1));
   }
+}
+
+// Key tiles [lo, hi) (tiles of bn keys) holding any key visible to any query
+// row in [q0, q1).  Empty range: lo == hi == 0.
+__host__ __device__ inline void kv_tile_range(const Problem& p, int q0, int q1, int bn, int& lo, int& hi) {
+  int key_lo, key_hi;
+  kv_key_range(p, q0, q1, key_lo, key_hi);
+  lo = hi = 0;
   if (key_lo >= key_hi) return;
   lo = key_lo / bn;
   hi = cdiv(key_hi, bn);

@@ -83,6 +83,7 @@ struct Unit {
   int split;         // key-range slice of a split problem (0 otherwise)
   int alt;           // 1: both slots hold the same rows and take alternate key tiles of one range
   int down;          // 1: the walk runs from its last tile down (block-sparse masks, no global tokens)
+  int koff;          // key tile j holds keys [j*BN + koff, (j+1)*BN + koff) (block-sparse masks; else 0)
 };
 
 // Walk accessors.  W = false (no global tokens): the walk is the band alone,
@@ -112,14 +113,37 @@ __device__ __forceinline__ bool walk_has(const Segs& s, int j) {
 // merging is a long chain of dependent integer operations that every thread
 // of a CTA runs before its first copy can start.
 template <bool W>
-__device__ __forceinline__ Segs tile_walk(const Problem& ps, int q0, int q1) {
+__device__ __forceinline__ Segs tile_walk(const Problem& ps, int q0, int q1, int koff) {
   if constexpr (W) {
     return kv_tile_segs(ps, q0, q1, BN);
   } else {
     Segs s;
-    kv_tile_range(ps, q0, q1, BN, s.lo[1], s.hi[1]);
+    int key_lo, key_hi;
+    kv_key_range(ps, q0, q1, key_lo, key_hi);
+    if (key_lo < key_hi) {
+      s.lo[1] = (key_lo - koff) / BN;
+      s.hi[1] = cdiv(key_hi - koff, BN);
+    }
     return s;
   }
+}
+
+// Offset of the key-tile grid.  Under a block-sparse mask the band of a row
+// tile starts on a block boundary, which need not be a tile boundary: 64-row
+// blocks give 128-row tiles a band of 256 keys starting 64 keys before a tile
+// boundary, three tiles on the aligned grid but two on a grid shifted by 64.
+// So the grid starts at the unit's first visible key (mod BN); copies of the
+// keys before 0 or past Lk read the tensor map's zero fill and are masked.
+// Other masks keep the aligned grid.  koff <= every slot's first key.
+template <bool W, bool DN>
+__device__ __forceinline__ int grid_offset(const Problem& ps, int qa0, int qb0, int qa1, int qb1) {
+  if (W || !DN || ps.sparse_block <= 0) return 0;
+  int a0, b0, a1, b1;
+  kv_key_range(ps, qa0, qb0, a0, b0);
+  kv_key_range(ps, qa1, qb1, a1, b1);
+  if (a0 >= b0 && a1 >= b1) return 0;
+  const int lo = a0 >= b0 ? a1 : (a1 >= b1 ? a0 : imin(a0, a1));
+  return lo % BN;
 }
 
 // The union of the two slots' walks (what the CTA streams); without global
@@ -145,7 +169,7 @@ __device__ __forceinline__ Segs union_walk(const Segs& a, const Segs& b) {
 // head kvh*G + r / Lq, i.e. Q read as [B*Hkv, G*Lq, d]; each unit takes two
 // consecutive 128-row tiles of a group.  A tile inside one head sees the key
 // tiles of its own query rows, a tile across heads those of all Lq rows.
-template <bool W>
+template <bool W, bool DN>
 __device__ __forceinline__ Unit decode_unit_packed(const FwdParams& P, int idx) {
   const Problem& p = P.prob;
   Unit u;
@@ -157,6 +181,9 @@ __device__ __forceinline__ Unit decode_unit_packed(const FwdParams& P, int idx) 
   u.kvh = grp % p.Hkv;
   const int qi = idx % nq;
   const Problem ps = seq_problem(p, u.b);
+  // Query rows of each slot's tile: its own rows inside one head, all Lq rows
+  // of a head when it spans several.
+  int qa[2], qb[2];
 #pragma unroll
   for (int s = 0; s < 2; s++) {
     const int r0 = (2 * qi + s) * BM;
@@ -164,13 +191,18 @@ __device__ __forceinline__ Unit decode_unit_packed(const FwdParams& P, int idx) 
     u.head[s] = u.kvh * G;
     u.q0[s] = r0;
     if (r0 >= r1) {
-      u.seg[s] = Segs{};
+      qa[s] = qb[s] = 0;
     } else if (r0 / p.Lq != (r1 - 1) / p.Lq) {
-      u.seg[s] = tile_walk<W>(ps, 0, p.Lq);
+      qa[s] = 0;
+      qb[s] = p.Lq;
     } else {
-      u.seg[s] = tile_walk<W>(ps, r0 % p.Lq, (r1 - 1) % p.Lq + 1);
+      qa[s] = r0 % p.Lq;
+      qb[s] = (r1 - 1) % p.Lq + 1;
     }
   }
+  u.koff = grid_offset<W, DN>(ps, qa[0], qb[0], qa[1], qb[1]);
+#pragma unroll
+  for (int s = 0; s < 2; s++) u.seg[s] = qa[s] < qb[s] ? tile_walk<W>(ps, qa[s], qb[s], u.koff) : Segs{};
   u.useg = union_walk<W>(u.seg[0], u.seg[1]);
   return u;
 }
@@ -187,11 +219,11 @@ __device__ __forceinline__ void make_alternating(Unit& u) {
   u.useg = u.seg[0];
 }
 
-template <bool W>
+template <bool W, bool DN>
 __device__ __forceinline__ Unit decode_unit(const FwdParams& P, int idx) {
   if (P.packed) {
-    Unit u = decode_unit_packed<W>(P, idx);
-    u.down = !W && P.prob.sparse_block > 0;
+    Unit u = decode_unit_packed<W, DN>(P, idx);
+    u.down = DN;
     u.alt = 0;
     if (P.alternate) make_alternating(u);
     return u;
@@ -234,10 +266,11 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& P, int idx) {
   }
   u.kvh = u.head[0] / G;
   const Problem ps = seq_problem(p, u.b);  // this sequence's lengths (padded batches)
-  u.seg[0] = tile_walk<W>(ps, u.q0[0], u.q0[0] + BM);
-  u.seg[1] = tile_walk<W>(ps, u.q0[1], u.q0[1] + BM);
+  u.koff = grid_offset<W, DN>(ps, u.q0[0], u.q0[0] + BM, u.q0[1], u.q0[1] + BM);
+  u.seg[0] = tile_walk<W>(ps, u.q0[0], u.q0[0] + BM, u.koff);
+  u.seg[1] = tile_walk<W>(ps, u.q0[1], u.q0[1] + BM, u.koff);
   u.useg = union_walk<W>(u.seg[0], u.seg[1]);
-  u.down = !W && P.prob.sparse_block > 0;
+  u.down = DN;
   u.alt = 0;
   if (P.alternate) make_alternating(u);
   return u;
@@ -248,14 +281,14 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& P, int idx) {
 // [k*n/ns, (k+1)*n/ns) of the union walk (n tiles), i.e. the tiles between
 // the first and last of them, in each slot's walk as well.  An empty slice
 // leaves both slots empty.
-template <bool W>
+template <bool W, bool DN>
 __device__ __forceinline__ Unit decode_unit_split(const FwdParams& P, int idx) {
   if (P.n_split <= 1) {
-    Unit u = decode_unit<W>(P, idx);
+    Unit u = decode_unit<W, DN>(P, idx);
     u.split = 0;
     return u;
   }
-  Unit u = decode_unit<W>(P, idx / P.n_split);
+  Unit u = decode_unit<W, DN>(P, idx / P.n_split);
   u.split = idx % P.n_split;
   const int n = walk_count<W>(u.useg);
   const int p0 = (int)((long long)u.split * n / P.n_split);
@@ -320,7 +353,7 @@ __device__ void producer(const FwdParams& P, const Unit& u, uint8_t* smem, Bars&
       mbar_arrive_expect_tx(&bars.kv_full[st], C::TILE);
       for (int pnl = 0; pnl < C::PANELS; pnl++)
         tma_load_3d(smem + C::OFF_KV + st * C::TILE + pnl * PANEL, which ? &P.tm_v : &P.tm_k, &bars.kv_full[st],
-                    pnl * 64, j * BN, u.b * p.Hkv + u.kvh);
+                    pnl * 64, j * BN + u.koff, u.b * p.Hkv + u.kvh);
       issued = r + 1;
     }
   }
@@ -529,7 +562,7 @@ __device__ void softmax_slot(const FwdParams& P, const Unit& u, int s, uint8_t* 
     // Element-wise mask only on tiles that straddle this row's visible range
     // (a per-row condition: it never guards a tcgen05 instruction, which the
     // whole warp must execute together).
-    const int key0 = j * BN;
+    const int key0 = j * BN + u.koff;
     const bool masked = key0 < key_lo || key0 + BN > key_hi;
     auto mask_cols = [&](int c0, int c1) {
       if (W && (gh_hi > 0 || gt_hi > gt_lo)) {
@@ -749,9 +782,9 @@ __global__ void __launch_bounds__(THREADS, 1) attn_fwd_kernel(const __grid_const
   Bars& bars = *reinterpret_cast<Bars*>(smem + C::OFF_BAR);
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  Unit u = decode_unit_split<W>(P, blockIdx.x);
+  Unit u = decode_unit_split<W, DN>(P, blockIdx.x);
   if (!A || W) u.alt = 0;
-  u.down = DN;  // equal to the decoded value; a constant lets the compiler drop the other direction
+
   const WaitGuard g{P.err, &bars.abort_flag, P.limit_ns, 0};
 
   if (threadIdx.x == 0) {
